@@ -1,0 +1,243 @@
+/*
+ * df11.h - C ABI of the B200 (sm_100a) exponent-Huffman BF16 weight codec.
+ *
+ * What the codec does (mlx-dfloat, PyPI page, intro and its bit diagram): a
+ * BF16 weight is s | eeeeeeee | mmmmmmm; the 8 exponent bits are replaced by
+ * a variable-length prefix code and the sign and 7 fraction bits are kept as
+ * one raw byte, so that decoding gives back the original bits exactly. The
+ * codebook is built deterministically from the exponent frequencies
+ * (df11pack, GitHub page, intro and "Licence"), codes have a maximum length
+ * (mlx-dfloat, "Try it": the "max-code" group), the decoder uses lookup tables
+ * and a block index (df11pack, "What is checked": --luts=correct,
+ * --index idx8) and the stream is cut into independently decodable chunks
+ * (df11pack, "Use": --safe and verify decode units and chunks). The pages do
+ * not give a container layout; this header defines it.
+ *
+ * Container of one tensor of n weights (all sizes from df_plan):
+ *   stream  n_chunks*C bytes of code bits, most significant bit first (the
+ *           first code bit is bit 7 of byte 0), zero after the last code,
+ *           then 16 zero bytes. n_chunks = max(1, ceil(total_bits / 8C)).
+ *   gaps    one 5-bit field per chunk, MSB first, zero padded (at least one
+ *           byte, to a multiple of 16 bytes). gap[j] = (first code start at
+ *           or after bit 8Cj) - 8Cj, where the end of the stream counts as a
+ *           code start; a code belongs to the chunk that holds its first bit.
+ *   block_offsets  n_blocks+1 uint64: offsets[b] = number of codes that start
+ *           before bit 8*C*T*b; offsets[n_blocks] = n. n_blocks = ceil(n_chunks/T).
+ *   sm      n bytes: sm[i] = (w >> 8 & 0x80) | (w & 0x7F).
+ *   lengths 256 code lengths (0 = symbol absent), canonical codes: symbols in
+ *           (length, symbol) order, code = (previous + 1) << (length step).
+ * C (chunk_bytes, a multiple of 16) and T (threads_per_block, a multiple of
+ * 32) are per-tensor parameters; the defaults are C = 32 and T = 256.
+ *
+ * Conventions for every function:
+ *   - returns a df_status; nothing is thrown across the ABI;
+ *   - device pointers are owned by the caller; the library allocates no device
+ *     memory and frees nothing; workspaces are passed in;
+ *   - kernels are launched asynchronously on `stream`, a cudaStream_t passed
+ *     as void* (NULL = the legacy default stream); a DF_OK return means the
+ *     launch was accepted, not that the data was valid: decode-time data
+ *     errors are reported through the optional device error word `d_err`
+ *     (DF_EFLAG_* bits OR-ed in; the caller zeroes it) and df_read_error;
+ *   - no function keeps global mutable state except the per-thread last CUDA
+ *     error returned by df_last_cuda_error.
+ */
+#ifndef DF11_H
+#define DF11_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int df_status;
+#define DF_OK 0
+#define DF_ERR_INVALID_ARG 1 /* a null, misaligned or inconsistent argument     */
+#define DF_ERR_CUDA 2        /* a CUDA call failed; see df_last_cuda_error()   */
+#define DF_ERR_CORRUPT 3     /* the device error word reported corrupt data     */
+#define DF_ERR_UNSUPPORTED 4 /* valid but outside this build's limits           */
+#define DF_ERR_WORKSPACE 5   /* workspace too small                             */
+
+/* bits of the device error word */
+#define DF_EFLAG_BAD_CODE 1u      /* decode: a bit pattern no code starts with        */
+#define DF_EFLAG_COUNT 2u         /* decode: codes in a block != its offset difference */
+#define DF_EFLAG_OFFSETS 4u       /* decode: block offsets out of range               */
+#define DF_EFLAG_ENC_TOTAL 16u    /* encode: stream length != the planned total_bits   */
+#define DF_EFLAG_ENC_SYMBOL 32u   /* encode: an exponent without a code                */
+
+#define DF_DEFAULT_CHUNK_BYTES 32u
+#define DF_DEFAULT_THREADS_PER_BLOCK 256u
+#define DF_DEFAULT_MAX_LEN 32u
+#define DF_MAX_WEIGHTS (1ull << 48) /* n above this is DF_ERR_UNSUPPORTED */
+
+/* A code table. Built by df_build_code from an exponent histogram. */
+typedef struct df_code {
+    uint32_t max_len;    /* the length limit the code was built with (1..32) */
+    uint32_t n_symbols;  /* exponents with a code                            */
+    uint32_t min_len;    /* shortest code length (0 when n_symbols == 0)     */
+    uint32_t n_tables;   /* 256-entry decode tables (see df_build_lut)       */
+    uint8_t lengths[256];
+    uint32_t codes[256]; /* canonical code of each exponent, right-aligned   */
+} df_code;
+
+/* Exact sizes of one tensor's container and of the encode workspace. */
+typedef struct df_sizes {
+    uint64_t total_bits, n_chunks, stream_bytes, gap_bytes, n_blocks, offsets_bytes, sm_bytes;
+    uint64_t container_bytes; /* stream + gaps + offsets + sm + 256 lengths + 64-byte header */
+    uint64_t encode_ws_bytes; /* device workspace df_encode needs                           */
+} df_sizes;
+
+/* Descriptor of one compressed tensor for decoding. Device pointers are
+ * read only; lut is the device copy of df_build_lut's output. */
+typedef struct df_tensor {
+    uint64_t n;
+    uint64_t total_bits;
+    uint32_t chunk_bytes;
+    uint32_t threads_per_block;
+    uint32_t max_len;
+    uint32_t n_tables;
+    const uint8_t* stream;         /* 16-byte aligned                 */
+    const uint8_t* gaps;
+    const uint64_t* block_offsets; /* 8-byte aligned                  */
+    const uint8_t* sm;             /* 8-byte aligned for vector loads  */
+    const uint32_t* lut;           /* 16-byte aligned                 */
+    uint8_t lengths[256];          /* host copy of the code lengths   */
+} df_tensor;
+
+/* Host plan of a grouped decode, filled by df_decode_batch_prepare. */
+typedef struct df_batch_plan {
+    void* d_ws;              /* the workspace holding the device table  */
+    uint32_t count;          /* tensors with n > 0                      */
+    uint32_t threads_per_block;
+    uint32_t chunk_bytes;
+    uint32_t smem_tables;    /* decode tables staged in shared memory   */
+    uint32_t stage_bytes;    /* exponent staging bytes per block        */
+    uint32_t smem_bytes;     /* dynamic shared memory per block         */
+    uint64_t total_blocks;
+} df_batch_plan;
+
+/* Human-readable name of a status. Static string; never NULL. */
+const char* df_status_string(df_status s);
+
+/* The cudaError_t of the last failing CUDA call made by this thread inside
+ * the library (0 if none). */
+int df_last_cuda_error(void);
+
+/* ---- code construction (host only) ---------------------------------------
+ * df_build_code: optimal prefix code over the exponents with hist[e] > 0 and
+ * no code longer than max_len (1..32), by package-merge (Larmore and
+ * Hirschberg 1990) with ties resolved as: items sorted by (count, exponent), an
+ * item before a package of equal weight. One exponent gets length 1 (code 0);
+ * an empty histogram gives an empty code. Then canonical codes.
+ * Source: df11pack (GitHub page), intro and "Licence" (deterministic codebook
+ * from frequencies); mlx-dfloat (PyPI page), "Try it" (a maximum code length).
+ * Errors: DF_ERR_INVALID_ARG for null pointers; DF_ERR_UNSUPPORTED when
+ * max_len is outside 1..32 or 2^max_len is below the number of exponents.
+ */
+df_status df_build_code(const uint64_t hist[256], uint32_t max_len, df_code* out);
+
+/* df_code_from_lengths: the canonical code for given code lengths (0 = no
+ * code), e.g. the lengths stored in a container. Errors: DF_ERR_INVALID_ARG
+ * (null, a length above max_len, or lengths that break Kraft's inequality
+ * sum 2^-l <= 1); DF_ERR_UNSUPPORTED (max_len outside 1..32). */
+df_status df_code_from_lengths(const uint8_t lengths[256], uint32_t max_len, df_code* out);
+
+/* Number of uint32 words df_build_lut writes: 256 per table plus 64 words
+ * holding the 256 code-length bytes. 0 for a NULL code. */
+size_t df_lut_words(const df_code* code);
+
+/* df_build_lut: derive the decode tables of a code into host memory `lut`
+ * (lut_words >= df_lut_words(code)). Table 0 is indexed by the next 8 stream
+ * bits; an entry holds up to three whole codes that fit in those 8 bits
+ * (symbols in bits 0-23, their count in bits 24-25, the bits they use in bits
+ * 26-31), or, for a longer code, count 0 and the index of a next-level table
+ * (bits 0-15) indexed by the following 8 bits, at most four levels for 32-bit
+ * codes. Entries no code reaches are zero. The caller copies the words to the
+ * device and passes them as df_tensor.lut. Source: df11pack, "What is
+ * checked" (--luts=correct zero-fills unreachable table entries).
+ * Errors: DF_ERR_INVALID_ARG (null, too small, or a code that is not prefix free).
+ */
+df_status df_build_lut(const df_code* code, uint32_t* lut, size_t lut_words);
+
+/* df_plan: exact sizes of the container for n weights with exponent
+ * histogram hist under `code`, and of df_encode's workspace.
+ * Errors: DF_ERR_INVALID_ARG (null; hist total != n; an exponent present in
+ * hist without a code; chunk_bytes not a multiple of 16 in 16..4096;
+ * threads_per_block not a multiple of 32 in 32..1024); DF_ERR_UNSUPPORTED
+ * (n > DF_MAX_WEIGHTS). */
+df_status df_plan(const df_code* code, const uint64_t hist[256], uint64_t n, uint32_t chunk_bytes,
+                  uint32_t threads_per_block, df_sizes* out);
+
+/* ---- encode (device) ---------------------------------------------------------
+ * df_histogram: d_hist256[e] = number of weights of d_in[0..n) whose exponent
+ * bits (w >> 7 & 0xFF) equal e. Overwrites d_hist256 (256 uint64, device,
+ * 8-byte aligned). d_in: n uint16 BF16 bit patterns on the device, 2-byte
+ * aligned (16-byte alignment takes the vector path). Source: df11pack, intro
+ * (codebook from exponent frequencies). Errors: DF_ERR_INVALID_ARG,
+ * DF_ERR_CUDA.
+ */
+df_status df_histogram(const uint16_t* d_in, uint64_t n, uint64_t* d_hist256, void* stream);
+
+/* df_encode: write the container of d_in[0..n) under `code`: d_stream
+ * (sizes.stream_bytes, 16-byte aligned), d_gaps (sizes.gap_bytes, 4-byte
+ * aligned), d_block_offsets (n_blocks+1 uint64), d_sm (n bytes). The bytes
+ * equal those of the layout above for the same code. d_ws: device workspace
+ * of at least sizes.encode_ws_bytes (16-byte aligned). total_bits is the
+ * value df_plan returned for the same input; a mismatch, or an exponent
+ * without a code, sets DF_EFLAG_ENC_* in d_err (nullable). Source:
+ * mlx-dfloat, intro bit diagram (what is coded and what is kept raw).
+ * Errors: DF_ERR_INVALID_ARG, DF_ERR_WORKSPACE, DF_ERR_CUDA.
+ */
+df_status df_encode(const df_code* code, const uint16_t* d_in, uint64_t n, uint64_t total_bits,
+                    uint32_t chunk_bytes, uint32_t threads_per_block, uint8_t* d_stream, uint8_t* d_gaps,
+                    uint64_t* d_block_offsets, uint8_t* d_sm, void* d_ws, size_t ws_bytes, uint32_t* d_err,
+                    void* stream);
+
+/* ---- decode (device) ---------------------------------------------------------
+ * df_decode: d_out[0..t->n) = the original BF16 bit patterns (uint16, device;
+ * 16-byte alignment takes the vector store path). One CUDA block per T
+ * chunks: the decode tables and the block's stream slice are staged in shared
+ * memory, each thread counts the codes that start in its chunk, a block scan
+ * turns the counts into output positions, a second pass writes the exponents
+ * to a shared-memory stage, and the block merges them with the sign|fraction
+ * bytes into 16-byte stores. Source: mlx-dfloat, intro and "Status" (blockwise
+ * GPU decode back to identical bits); df11pack, "Use" (chunks).
+ * Data errors set DF_EFLAG_* in d_err (nullable) and skip the affected
+ * block's stores. Errors: DF_ERR_INVALID_ARG, DF_ERR_UNSUPPORTED (a layout
+ * whose block needs more shared memory than the device has), DF_ERR_CUDA.
+ */
+df_status df_decode(const df_tensor* t, uint16_t* d_out, uint32_t* d_err, void* stream);
+
+/* Device workspace bytes df_decode_batch needs for `count` tensors. */
+size_t df_decode_batch_workspace(uint32_t count);
+
+/* df_decode_batch_prepare: validate `count` descriptors (host array) and
+ * their outputs (host array of device pointers), write the device table into
+ * d_ws (asynchronously on `stream`; the host arrays may be reused on return)
+ * and fill *plan. All tensors must share chunk_bytes and threads_per_block.
+ * Errors: DF_ERR_INVALID_ARG, DF_ERR_WORKSPACE, DF_ERR_UNSUPPORTED, DF_ERR_CUDA. */
+df_status df_decode_batch_prepare(const df_tensor* tensors, uint16_t* const* d_outs, uint32_t count, void* d_ws,
+                                  size_t ws_bytes, df_batch_plan* plan, void* stream);
+
+/* df_decode_batch_run: decode every tensor of a prepared table in one launch
+ * (one CUDA block per format block over all tensors; block -> tensor by a
+ * binary search of the prefix sum of block counts). The workspace must hold
+ * the prepared table until the launch has run. Errors: DF_ERR_INVALID_ARG,
+ * DF_ERR_CUDA. */
+df_status df_decode_batch_run(const df_batch_plan* plan, uint32_t* d_err, void* stream);
+
+/* df_decode_batch: prepare + run. */
+df_status df_decode_batch(const df_tensor* tensors, uint16_t* const* d_outs, uint32_t count, void* d_ws,
+                          size_t ws_bytes, uint32_t* d_err, void* stream);
+
+/* df_read_error: wait for `stream`, copy the device error word to *flags
+ * (nullable) and return DF_ERR_CORRUPT if any bit is set, else DF_OK.
+ * Errors: DF_ERR_INVALID_ARG, DF_ERR_CUDA. */
+df_status df_read_error(const uint32_t* d_err, void* stream, uint32_t* flags);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DF11_H */

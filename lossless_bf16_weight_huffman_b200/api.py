@@ -1,0 +1,140 @@
+"""Python binding of the C ABI: one function per entry point of include/df11.h,
+same names, argument marshalling only. Device buffers are torch CUDA tensors
+(PyTorch supplies memory and streams); every computation runs in libdf11.so.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+import torch
+
+from ._native import DfBatchPlan, DfCode, DfSizes, DfTensor, check, lib
+
+
+def _stream_ptr(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dev(t: torch.Tensor | None, name: str):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor (there is no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _hist_array(hist) -> np.ndarray:
+    h = np.ascontiguousarray(np.asarray(hist, dtype=np.uint64).reshape(-1))
+    if h.size != 256:
+        raise ValueError("hist must have 256 entries")
+    return h
+
+
+def df_status_string(status: int) -> str:
+    return lib().df_status_string(status).decode()
+
+
+def df_last_cuda_error() -> int:
+    return int(lib().df_last_cuda_error())
+
+
+def df_build_code(hist, max_len: int = 32) -> DfCode:
+    h = _hist_array(hist)
+    code = DfCode()
+    check("df_build_code", lib().df_build_code(h.ctypes.data, max_len, ctypes.byref(code)))
+    return code
+
+
+def df_code_from_lengths(lengths, max_len: int = 32) -> DfCode:
+    arr = np.ascontiguousarray(np.asarray(lengths, dtype=np.uint8).reshape(-1))
+    if arr.size != 256:
+        raise ValueError("lengths must have 256 entries")
+    code = DfCode()
+    check("df_code_from_lengths", lib().df_code_from_lengths(arr.ctypes.data, max_len, ctypes.byref(code)))
+    return code
+
+
+def df_lut_words(code: DfCode) -> int:
+    return int(lib().df_lut_words(ctypes.byref(code)))
+
+
+def df_build_lut(code: DfCode) -> np.ndarray:
+    words = df_lut_words(code)
+    out = np.zeros(words, np.uint32)
+    check("df_build_lut", lib().df_build_lut(ctypes.byref(code), out.ctypes.data, words))
+    return out
+
+
+def df_plan(code: DfCode, hist, n: int, chunk_bytes: int = 32, threads_per_block: int = 256) -> DfSizes:
+    h = _hist_array(hist)
+    z = DfSizes()
+    check("df_plan", lib().df_plan(ctypes.byref(code), h.ctypes.data, n, chunk_bytes, threads_per_block,
+                                   ctypes.byref(z)))
+    return z
+
+
+def df_histogram(d_in: torch.Tensor, d_hist256: torch.Tensor, stream=None) -> None:
+    check("df_histogram", lib().df_histogram(_dev(d_in, "d_in"), d_in.numel(), _dev(d_hist256, "d_hist256"),
+                                             _stream_ptr(stream)))
+
+
+def df_encode(code: DfCode, d_in: torch.Tensor, total_bits: int, chunk_bytes: int, threads_per_block: int,
+              d_stream: torch.Tensor, d_gaps: torch.Tensor, d_block_offsets: torch.Tensor, d_sm: torch.Tensor,
+              d_ws: torch.Tensor, d_err: torch.Tensor | None = None, stream=None) -> None:
+    ws_bytes = d_ws.numel() * d_ws.element_size() if d_ws is not None else 0
+    check("df_encode", lib().df_encode(
+        ctypes.byref(code), _dev(d_in, "d_in"), d_in.numel(), total_bits, chunk_bytes, threads_per_block,
+        _dev(d_stream, "d_stream"), _dev(d_gaps, "d_gaps"), _dev(d_block_offsets, "d_block_offsets"),
+        _dev(d_sm, "d_sm"), _dev(d_ws, "d_ws"), ws_bytes, _dev(d_err, "d_err"), _stream_ptr(stream)))
+
+
+def df_decode(t: DfTensor, d_out: torch.Tensor, d_err: torch.Tensor | None = None, stream=None) -> None:
+    check("df_decode", lib().df_decode(ctypes.byref(t), _dev(d_out, "d_out"), _dev(d_err, "d_err"),
+                                       _stream_ptr(stream)))
+
+
+def df_decode_batch_workspace(count: int) -> int:
+    return int(lib().df_decode_batch_workspace(count))
+
+
+def _batch_arrays(tensors, d_outs):
+    if len(tensors) != len(d_outs):
+        raise ValueError("one output per tensor")
+    arr = (DfTensor * max(1, len(tensors)))(*tensors)
+    outs = (ctypes.c_void_p * max(1, len(d_outs)))(*[_dev(o, "d_outs[i]").value for o in d_outs])
+    return arr, outs
+
+
+def df_decode_batch_prepare(tensors, d_outs, d_ws: torch.Tensor, stream=None) -> DfBatchPlan:
+    arr, outs = _batch_arrays(tensors, d_outs)
+    plan = DfBatchPlan()
+    ws_bytes = d_ws.numel() * d_ws.element_size()
+    check("df_decode_batch_prepare", lib().df_decode_batch_prepare(
+        arr, outs, len(tensors), _dev(d_ws, "d_ws"), ws_bytes, ctypes.byref(plan), _stream_ptr(stream)))
+    return plan
+
+
+def df_decode_batch_run(plan: DfBatchPlan, d_err: torch.Tensor | None = None, stream=None) -> None:
+    check("df_decode_batch_run", lib().df_decode_batch_run(ctypes.byref(plan), _dev(d_err, "d_err"),
+                                                           _stream_ptr(stream)))
+
+
+def df_decode_batch(tensors, d_outs, d_ws: torch.Tensor, d_err: torch.Tensor | None = None, stream=None) -> None:
+    arr, outs = _batch_arrays(tensors, d_outs)
+    ws_bytes = d_ws.numel() * d_ws.element_size()
+    check("df_decode_batch", lib().df_decode_batch(arr, outs, len(tensors), _dev(d_ws, "d_ws"), ws_bytes,
+                                                   _dev(d_err, "d_err"), _stream_ptr(stream)))
+
+
+def df_read_error(d_err: torch.Tensor, stream=None) -> int:
+    """Return the device error word (0 = clean); waits for the stream."""
+    flags = ctypes.c_uint32(0)
+    status = lib().df_read_error(_dev(d_err, "d_err"), _stream_ptr(stream), ctypes.byref(flags))
+    if status not in (0, 3):
+        check("df_read_error", status)
+    return int(flags.value)

@@ -1,0 +1,170 @@
+"""Tensor-level helpers over the C ABI: compress a BF16 CUDA tensor into a
+container held in torch CUDA buffers, and decode one or many containers.
+
+PyTorch only allocates memory here; every step of the codec runs in
+libdf11.so (df_histogram, df_encode, df_decode, df_decode_batch_*). Building
+the code table is host work done by df_build_code / df_build_lut in the same
+library. There is no CPU fallback: CPU tensors are rejected.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from . import api
+from ._native import DfTensor
+
+DEFAULT_MAX_LEN = 32
+DEFAULT_CHUNK_BYTES = 32
+DEFAULT_THREADS_PER_BLOCK = 256
+
+
+def _as_u16(w: torch.Tensor) -> torch.Tensor:
+    if not w.is_cuda:
+        raise TypeError("compress takes a CUDA tensor (there is no CPU path)")
+    if w.dtype not in (torch.bfloat16, torch.int16, torch.uint16):
+        raise TypeError(f"expected BF16 bit patterns (bfloat16/int16/uint16), got {w.dtype}")
+    return w.contiguous().reshape(-1).view(torch.int16)
+
+
+class Compressed:
+    """One tensor's container in device memory."""
+
+    def __init__(self, *, n, shape, code, lut, sizes, chunk_bytes, threads_per_block, stream, gaps, offsets, sm):
+        self.n = int(n)
+        self.shape = tuple(shape)
+        self.code = code
+        self.lut = lut
+        self.sizes = sizes
+        self.chunk_bytes = chunk_bytes
+        self.threads_per_block = threads_per_block
+        self.stream = stream
+        self.gaps = gaps
+        self.offsets = offsets
+        self.sm = sm
+        self._desc = None
+
+    @property
+    def total_bits(self) -> int:
+        return self.sizes["total_bits"]
+
+    @property
+    def container_bytes(self) -> int:
+        return self.sizes["container_bytes"]
+
+    @property
+    def ratio(self) -> float:
+        return self.container_bytes / (2 * self.n) if self.n else 1.0
+
+    @property
+    def lengths(self) -> np.ndarray:
+        return np.frombuffer(bytes(self.code.lengths), np.uint8).copy()
+
+    def read_bytes(self) -> int:
+        """Bytes a full decode must read: the stream, gaps, offsets and sm bytes."""
+        z = self.sizes
+        return z["stream_bytes"] + z["gap_bytes"] + z["offsets_bytes"] + z["sm_bytes"]
+
+    def descriptor(self) -> DfTensor:
+        if self._desc is None:
+            d = DfTensor()
+            d.n = self.n
+            d.total_bits = self.total_bits
+            d.chunk_bytes = self.chunk_bytes
+            d.threads_per_block = self.threads_per_block
+            d.max_len = self.code.max_len
+            d.n_tables = self.code.n_tables
+            d.stream = self.stream.data_ptr()
+            d.gaps = self.gaps.data_ptr()
+            d.block_offsets = self.offsets.data_ptr()
+            d.sm = self.sm.data_ptr() if self.n else self.stream.data_ptr()
+            d.lut = self.lut.data_ptr()
+            d.lengths[:] = self.code.lengths[:]
+            self._desc = d
+        return self._desc
+
+    @classmethod
+    def from_host(cls, *, lengths, max_len, total_bits, n, stream, gaps, offsets, sm, shape=None,
+                  chunk_bytes=DEFAULT_CHUNK_BYTES, threads_per_block=DEFAULT_THREADS_PER_BLOCK,
+                  device="cuda"):
+        """Upload a container whose parts are host arrays (e.g. read from a file)."""
+        code = api.df_code_from_lengths(lengths, max_len)
+        lut = torch.from_numpy(api.df_build_lut(code).view(np.int32)).to(device)
+        hist_free = {
+            "total_bits": int(total_bits),
+            "stream_bytes": int(np.asarray(stream).size),
+            "gap_bytes": int(np.asarray(gaps).size),
+            "offsets_bytes": 8 * int(np.asarray(offsets).size),
+            "sm_bytes": int(n),
+        }
+        hist_free["container_bytes"] = (hist_free["stream_bytes"] + hist_free["gap_bytes"] +
+                                        hist_free["offsets_bytes"] + int(n) + 256 + 64)
+        t = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a).view(dt)).to(device)  # noqa: E731
+        sm_arr = np.asarray(sm, np.uint8)
+        return cls(n=n, shape=shape or (n,), code=code, lut=lut, sizes=hist_free, chunk_bytes=chunk_bytes,
+                   threads_per_block=threads_per_block, stream=t(np.asarray(stream, np.uint8), np.uint8),
+                   gaps=t(np.asarray(gaps, np.uint8), np.uint8),
+                   offsets=t(np.asarray(offsets, np.uint64), np.int64),
+                   sm=t(sm_arr if sm_arr.size else np.zeros(16, np.uint8), np.uint8))
+
+
+def compress(w: torch.Tensor, max_len: int = DEFAULT_MAX_LEN, chunk_bytes: int = DEFAULT_CHUNK_BYTES,
+             threads_per_block: int = DEFAULT_THREADS_PER_BLOCK, d_err: torch.Tensor | None = None,
+             stream=None) -> Compressed:
+    """Histogram on the GPU, code build on the host, encode on the GPU."""
+    x = _as_u16(w)
+    dev = x.device
+    n = x.numel()
+    hist_d = torch.empty(256, dtype=torch.int64, device=dev)
+    api.df_histogram(x, hist_d, stream)
+    hist = hist_d.cpu().numpy().view(np.uint64)
+    code = api.df_build_code(hist, max_len)
+    lut = torch.from_numpy(api.df_build_lut(code).view(np.int32)).to(dev)
+    z = api.df_plan(code, hist, n, chunk_bytes, threads_per_block).as_dict()
+    stream_buf = torch.empty(z["stream_bytes"], dtype=torch.uint8, device=dev)
+    gaps = torch.empty(z["gap_bytes"], dtype=torch.uint8, device=dev)
+    offsets = torch.empty(z["n_blocks"] + 1, dtype=torch.int64, device=dev)
+    sm = torch.empty(max(n, 16), dtype=torch.uint8, device=dev)
+    ws = torch.empty(max(z["encode_ws_bytes"], 16), dtype=torch.uint8, device=dev)
+    api.df_encode(code, x, z["total_bits"], chunk_bytes, threads_per_block, stream_buf, gaps, offsets,
+                  sm, ws, d_err, stream)
+    return Compressed(n=n, shape=tuple(w.shape), code=code, lut=lut, sizes=z, chunk_bytes=chunk_bytes,
+                      threads_per_block=threads_per_block, stream=stream_buf, gaps=gaps, offsets=offsets, sm=sm)
+
+
+def decompress(c: Compressed, out: torch.Tensor | None = None, d_err: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+    """Decode into `out` (BF16 or 16-bit integer CUDA tensor of c.n elements)."""
+    if out is None:
+        out = torch.empty(c.shape, dtype=torch.bfloat16, device=c.stream.device)
+    if out.numel() != c.n:
+        raise ValueError("output size differs from the container's")
+    api.df_decode(c.descriptor(), out.view(torch.int16).reshape(-1) if c.n else out, d_err, stream)
+    return out
+
+
+class BatchDecoder:
+    """A grouped decode of many containers, prepared once and launched many
+    times (one kernel launch per run)."""
+
+    def __init__(self, comps: list[Compressed], outs: list[torch.Tensor] | None = None, stream=None):
+        if not comps:
+            raise ValueError("no tensors")
+        dev = comps[0].stream.device
+        self.comps = comps
+        self.outs = outs if outs is not None else [
+            torch.empty(c.shape, dtype=torch.bfloat16, device=dev) for c in comps]
+        self.ws = torch.empty(api.df_decode_batch_workspace(len(comps)), dtype=torch.uint8, device=dev)
+        descs = [c.descriptor() for c in comps]
+        flat = [o.view(torch.int16).reshape(-1) for o in self.outs]
+        self.plan = api.df_decode_batch_prepare(descs, flat, self.ws, stream)
+
+    def run(self, d_err: torch.Tensor | None = None, stream=None) -> list[torch.Tensor]:
+        api.df_decode_batch_run(self.plan, d_err, stream)
+        return self.outs
+
+
+def decompress_batch(comps: list[Compressed], outs: list[torch.Tensor] | None = None,
+                     d_err: torch.Tensor | None = None, stream=None) -> list[torch.Tensor]:
+    dec = BatchDecoder(comps, outs, stream)
+    return dec.run(d_err, stream)

@@ -1,0 +1,370 @@
+// Encode path: exponent histogram, per-tile code-length sums, a scan of the
+// tile sums into bit offsets, and a warp-level bit packer.
+//
+// What is coded (mlx-dfloat, PyPI page, intro bit diagram): the 8 exponent
+// bits of each BF16 weight become a variable-length code; the sign and the 7
+// fraction bits become one raw byte. The codebook comes from the exponent
+// frequencies (df11pack, GitHub page, intro). The stream layout (MSB-first
+// bits, C-byte chunks with 5-bit start gaps, per-block output offsets) is the
+// one df11.h defines.
+//
+// Tiles of 4096 weights: 8 warps x 16 steps x 32 lanes. In a step each lane
+// holds one weight's code; a warp shuffle scan gives each code its bit
+// offset, and every 32-bit stream word the step touches is assembled with one
+// warp OR-reduction. Words inside a warp's range are written whole; the first
+// and last word of a warp's range (shared with its neighbours) are OR-ed in
+// atomically into the zeroed stream.
+#include <cuda_runtime.h>
+
+#include <cstring>
+
+#include "df_internal.h"
+
+namespace df {
+namespace {
+
+constexpr uint32_t kTile = 4096;
+constexpr uint32_t kEncThreads = 256;
+constexpr uint32_t kSteps = kTile / kEncThreads;  // 16 steps of 32 weights per warp
+
+__device__ __forceinline__ uint32_t bswap32(uint32_t x) { return __byte_perm(x, 0, 0x0123); }
+
+__global__ void __launch_bounds__(256) hist_kernel(const uint16_t* __restrict__ in, uint64_t n, int vec,
+                                                   unsigned long long* __restrict__ hist) {
+    __shared__ uint32_t sh[8][256];
+    const uint32_t warp = threadIdx.x >> 5;
+    for (uint32_t i = threadIdx.x; i < 8 * 256; i += blockDim.x) (&sh[0][0])[i] = 0;
+    __syncthreads();
+    const uint64_t stride = static_cast<uint64_t>(gridDim.x) * blockDim.x;
+    uint64_t done = 0;
+    if (vec) {
+        const uint64_t n8 = n / 8;
+        const uint4* in4 = reinterpret_cast<const uint4*>(in);
+        for (uint64_t i = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8; i += stride) {
+            const uint4 v = __ldg(in4 + i);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                atomicAdd(&sh[warp][(w[k] >> 7) & 0xFFu], 1u);
+                atomicAdd(&sh[warp][(w[k] >> 23) & 0xFFu], 1u);
+            }
+        }
+        done = n8 * 8;
+    }
+    for (uint64_t i = done + static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride)
+        atomicAdd(&sh[warp][(__ldg(in + i) >> 7) & 0xFFu], 1u);
+    __syncthreads();
+    for (uint32_t s = threadIdx.x; s < 256; s += blockDim.x) {
+        uint32_t c = 0;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) c += sh[w][s];
+        if (c) atomicAdd(hist + s, static_cast<unsigned long long>(c));
+    }
+}
+
+struct EncTables {
+    uint32_t codes[256];
+    uint8_t lengths[256];
+};
+
+// Sum of code lengths of each tile of 4096 weights.
+__global__ void __launch_bounds__(kEncThreads) tile_bits_kernel(const uint16_t* __restrict__ in, uint64_t n,
+                                                                EncTables tab, uint64_t* __restrict__ tile_bits,
+                                                                uint32_t* d_err) {
+    __shared__ uint8_t s_len[256];
+    __shared__ uint32_t s_red[kEncThreads / 32];
+    for (uint32_t i = threadIdx.x; i < 256; i += blockDim.x) s_len[i] = tab.lengths[i];
+    __syncthreads();
+    const uint64_t base = static_cast<uint64_t>(blockIdx.x) * kTile;
+    uint32_t sum = 0;
+    bool missing = false;
+#pragma unroll 4
+    for (uint32_t k = 0; k < kSteps; ++k) {
+        const uint64_t i = base + k * kEncThreads + threadIdx.x;
+        if (i < n) {
+            const uint32_t l = s_len[(__ldg(in + i) >> 7) & 0xFFu];
+            missing |= (l == 0);
+            sum += l;
+        }
+    }
+    if (__syncthreads_or(missing) && threadIdx.x == 0 && d_err) atomicOr(d_err, DF_EFLAG_ENC_SYMBOL);
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, d);
+    if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = sum;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t t = 0;
+        for (uint32_t w = 0; w < kEncThreads / 32; ++w) t += s_red[w];
+        tile_bits[blockIdx.x] = t;
+    }
+}
+
+// Exclusive scan of the tile sums (one block): tile_base[0..tiles].
+__global__ void __launch_bounds__(1024) tile_scan_kernel(const uint64_t* __restrict__ tile_bits, uint64_t tiles,
+                                                         uint64_t* __restrict__ tile_base, uint64_t want_total,
+                                                         uint64_t* __restrict__ offsets, uint64_t n_blocks,
+                                                         uint64_t n, uint32_t* d_err) {
+    __shared__ uint64_t s_w[32];
+    __shared__ uint64_t s_carry;
+    if (threadIdx.x == 0) s_carry = 0;
+    __syncthreads();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (uint64_t start = 0; start < tiles; start += blockDim.x) {
+        const uint64_t i = start + threadIdx.x;
+        const uint64_t v = i < tiles ? tile_bits[i] : 0;
+        uint64_t x = v;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const uint64_t u = __shfl_up_sync(0xFFFFFFFFu, x, d);
+            if (lane >= d) x += u;
+        }
+        if (lane == 31) s_w[warp] = x;
+        __syncthreads();
+        if (warp == 0) {
+            uint64_t y = lane < static_cast<int>(blockDim.x >> 5) ? s_w[lane] : 0;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const uint64_t u = __shfl_up_sync(0xFFFFFFFFu, y, d);
+                if (lane >= d) y += u;
+            }
+            s_w[lane] = y;
+        }
+        __syncthreads();
+        const uint64_t carry = s_carry;
+        const uint64_t incl = x + (warp > 0 ? s_w[warp - 1] : 0);
+        if (i < tiles) tile_base[i] = carry + incl - v;
+        __syncthreads();
+        if (threadIdx.x == 0) s_carry = carry + s_w[(blockDim.x >> 5) - 1];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        tile_base[tiles] = s_carry;
+        if (s_carry != want_total && d_err) atomicOr(d_err, DF_EFLAG_ENC_TOTAL);
+        offsets[0] = 0;
+        offsets[n_blocks] = n;
+    }
+}
+
+struct PackArgs {
+    const uint16_t* in;
+    uint64_t n;
+    const uint64_t* tile_base;
+    uint32_t* stream32;   // the stream as 32-bit words (zeroed)
+    uint32_t* gaps32;     // the gap fields as 32-bit words (zeroed)
+    uint64_t* offsets;
+    uint8_t* sm;
+    uint64_t total_bits;
+    uint64_t n_chunks;
+    uint64_t stream_words;  // words the stream buffer holds: writes beyond are refused
+    uint32_t chunk_bits;
+    uint32_t threads_per_block;
+    uint32_t* err;
+};
+
+__device__ __forceinline__ void or_gap(uint32_t* gaps32, uint64_t j, uint32_t g) {
+    const uint64_t q = 5 * j;
+    const uint32_t o = static_cast<uint32_t>(q & 31);
+    uint32_t* w = gaps32 + (q >> 5);
+    if (o <= 27) {
+        atomicOr(w, bswap32(g << (27 - o)));
+    } else {
+        atomicOr(w, bswap32(g >> (o - 27)));
+        atomicOr(w + 1, bswap32(g << (59 - o)));
+    }
+}
+
+// This lane's bits of stream word W: the code occupies [ls, ls+l).
+__device__ __forceinline__ uint32_t word_part(uint64_t ls, uint32_t l, uint32_t code, uint64_t W) {
+    const uint64_t w0 = 32 * W;
+    if (l == 0 || ls >= w0 + 32 || ls + l <= w0) return 0;
+    const uint64_t v = static_cast<uint64_t>(code) << (64 - l);
+    if (ls >= w0) return static_cast<uint32_t>(v >> (32 + (ls - w0)));
+    return static_cast<uint32_t>((v << (w0 - ls)) >> 32);
+}
+
+__global__ void __launch_bounds__(kEncThreads) pack_kernel(PackArgs a, EncTables tab) {
+    __shared__ uint32_t s_code[256];
+    __shared__ uint8_t s_len[256];
+    __shared__ uint64_t s_wsum[kEncThreads / 32];
+    for (uint32_t i = threadIdx.x; i < 256; i += blockDim.x) {
+        s_code[i] = tab.codes[i];
+        s_len[i] = tab.lengths[i];
+    }
+    __syncthreads();
+    const uint32_t lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint64_t wbase = static_cast<uint64_t>(blockIdx.x) * kTile + warp * (kSteps * 32);
+
+    // bits of this warp's 512 weights
+    uint32_t mine = 0;
+#pragma unroll 4
+    for (uint32_t s = 0; s < kSteps; ++s) {
+        const uint64_t i = wbase + s * 32 + lane;
+        if (i < a.n) mine += s_len[(__ldg(a.in + i) >> 7) & 0xFFu];
+    }
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) mine += __shfl_xor_sync(0xFFFFFFFFu, mine, d);
+    if (lane == 0) s_wsum[warp] = mine;
+    __syncthreads();
+    uint64_t pos = a.tile_base[blockIdx.x];
+    for (uint32_t w = 0; w < warp; ++w) pos += s_wsum[w];
+    if (s_wsum[warp] == 0) return;  // nothing of this warp's range is in the tensor
+
+    const uint64_t first_word = pos >> 5;
+    uint64_t cur_word = first_word;
+    uint32_t carry = 0;
+    for (uint32_t s = 0; s < kSteps; ++s) {
+        const uint64_t i = wbase + s * 32 + lane;
+        uint32_t l = 0, code = 0;
+        if (i < a.n) {
+            const uint16_t x = __ldg(a.in + i);
+            const uint32_t e = (x >> 7) & 0xFFu;
+            l = s_len[e];
+            code = s_code[e];
+            a.sm[i] = static_cast<uint8_t>(((x >> 8) & 0x80u) | (x & 0x7Fu));
+        }
+        uint32_t incl = l;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const uint32_t u = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+            if (lane >= static_cast<uint32_t>(d)) incl += u;
+        }
+        const uint32_t step_bits = __shfl_sync(0xFFFFFFFFu, incl, 31);
+        const uint64_t ls = pos + incl - l;
+        // chunk index: the code that crosses (or ends on) a chunk boundary owns it
+        if (l) {
+            const uint64_t le = ls + l;
+            const uint64_t j = le / a.chunk_bits;
+            if (j > ls / a.chunk_bits && j < a.n_chunks) {
+                or_gap(a.gaps32, j, static_cast<uint32_t>(le - j * a.chunk_bits));
+                if (j % a.threads_per_block == 0) a.offsets[j / a.threads_per_block] = i + 1;
+            }
+        }
+        if (step_bits) {
+            const uint64_t fw = pos >> 5, lw = (pos + step_bits - 1) >> 5;
+            for (uint64_t W = fw; W <= lw; ++W) {
+                const uint32_t word = __reduce_or_sync(0xFFFFFFFFu, word_part(ls, l, code, W));
+                if (W == cur_word) {
+                    carry |= word;
+                } else {
+                    if (lane == 0) {
+                        if (cur_word >= a.stream_words) {
+                            if (a.err) atomicOr(a.err, DF_EFLAG_ENC_TOTAL);
+                        } else if (cur_word == first_word) {
+                            atomicOr(a.stream32 + cur_word, bswap32(carry));
+                        } else {
+                            a.stream32[cur_word] = bswap32(carry);
+                        }
+                    }
+                    cur_word = W;
+                    carry = word;
+                }
+            }
+        }
+        pos += step_bits;
+    }
+    if (lane == 0) {
+        if (cur_word < a.stream_words)
+            atomicOr(a.stream32 + cur_word, bswap32(carry));
+        else if (a.err)
+            atomicOr(a.err, DF_EFLAG_ENC_TOTAL);
+    }
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+df_status sm_count(int* sms) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return DF_OK;
+}
+
+}  // namespace
+}  // namespace df
+
+using namespace df;
+
+extern "C" {
+
+df_status df_histogram(const uint16_t* d_in, uint64_t n, uint64_t* d_hist256, void* stream) {
+    if (!d_hist256 || (n && !d_in) || !aligned(d_in, 2) || !aligned(d_hist256, 8)) return DF_ERR_INVALID_ARG;
+    if (n > DF_MAX_WEIGHTS) return DF_ERR_UNSUPPORTED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(d_hist256, 0, 256 * sizeof(uint64_t), s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (n == 0) return DF_OK;
+    int sms = 0;
+    df_status st = sm_count(&sms);
+    if (st != DF_OK) return st;
+    // at most 2^30 weights per block keeps the 32-bit shared counters exact
+    uint64_t grid = (n + 256ull * 8 * 4 - 1) / (256ull * 8 * 4);
+    const uint64_t cap = static_cast<uint64_t>(sms) * 8;
+    if (grid > cap) grid = cap;
+    const uint64_t floor_blocks = (n >> 30) + 1;
+    if (grid < floor_blocks) grid = floor_blocks;
+    hist_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(d_in, n, aligned(d_in, 16) ? 1 : 0,
+                                                          reinterpret_cast<unsigned long long*>(d_hist256));
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e);
+    return DF_OK;
+}
+
+df_status df_encode(const df_code* code, const uint16_t* d_in, uint64_t n, uint64_t total_bits,
+                    uint32_t chunk_bytes, uint32_t tpb, uint8_t* d_stream, uint8_t* d_gaps,
+                    uint64_t* d_block_offsets, uint8_t* d_sm, void* d_ws, size_t ws_bytes, uint32_t* d_err,
+                    void* stream) {
+    if (!code || !d_stream || !d_gaps || !d_block_offsets || (n && (!d_in || !d_sm))) return DF_ERR_INVALID_ARG;
+    if (chunk_bytes < 16 || chunk_bytes > 4096 || chunk_bytes % 16 || tpb < 32 || tpb > 1024 || tpb % 32)
+        return DF_ERR_INVALID_ARG;
+    if (!aligned(d_stream, 16) || !aligned(d_gaps, 4) || !aligned(d_block_offsets, 8) || !aligned(d_in, 2))
+        return DF_ERR_INVALID_ARG;
+    if (n > DF_MAX_WEIGHTS) return DF_ERR_UNSUPPORTED;
+    const uint64_t cbits = 8ull * chunk_bytes;
+    const uint64_t n_chunks = total_bits ? (total_bits + cbits - 1) / cbits : 1;
+    const uint64_t stream_bytes = n_chunks * chunk_bytes + 16;
+    const uint64_t gap_bytes = (((5 * n_chunks + 7) / 8) + 1 + 15) & ~15ull;
+    const uint64_t n_blocks = (n_chunks + tpb - 1) / tpb;
+    const uint64_t tiles = (n + kTile - 1) / kTile;
+    const uint64_t need_ws = 16 * (tiles + 2) + 256;
+    if (n && (ws_bytes < need_ws || !d_ws)) return DF_ERR_WORKSPACE;
+    if (n && !aligned(d_ws, 16)) return DF_ERR_INVALID_ARG;
+    if (tiles > 0x7FFFFFFFull) return DF_ERR_UNSUPPORTED;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(d_stream, 0, stream_bytes, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(d_gaps, 0, gap_bytes, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(d_block_offsets, 0, 8 * (n_blocks + 1), s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (n == 0) return DF_OK;  // empty stream, zero gap, offsets {0, 0}
+
+    EncTables tab;
+    std::memcpy(tab.codes, code->codes, sizeof(tab.codes));
+    std::memcpy(tab.lengths, code->lengths, sizeof(tab.lengths));
+    uint64_t* tile_bits = static_cast<uint64_t*>(d_ws);
+    uint64_t* tile_base = tile_bits + tiles;
+    tile_bits_kernel<<<static_cast<unsigned>(tiles), kEncThreads, 0, s>>>(d_in, n, tab, tile_bits, d_err);
+    tile_scan_kernel<<<1, 1024, 0, s>>>(tile_bits, tiles, tile_base, total_bits, d_block_offsets, n_blocks, n,
+                                         d_err);
+    PackArgs a;
+    a.in = d_in;
+    a.n = n;
+    a.tile_base = tile_base;
+    a.stream32 = reinterpret_cast<uint32_t*>(d_stream);
+    a.gaps32 = reinterpret_cast<uint32_t*>(d_gaps);
+    a.offsets = d_block_offsets;
+    a.sm = d_sm;
+    a.total_bits = total_bits;
+    a.n_chunks = n_chunks;
+    a.stream_words = stream_bytes / 4;
+    a.err = d_err;
+    a.chunk_bits = static_cast<uint32_t>(cbits);
+    a.threads_per_block = tpb;
+    pack_kernel<<<static_cast<unsigned>(tiles), kEncThreads, 0, s>>>(a, tab);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e);
+    return DF_OK;
+}
+
+}  // extern "C"

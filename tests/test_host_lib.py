@@ -1,0 +1,207 @@
+"""Host side of the CUDA library, on the CPU: the exported symbols, the code
+build against the oracle, size planning against the oracle, and the decode
+tables (walked here by a plain-Python model of the kernel's table steps)
+against the oracle's decoded output. No CUDA call is made.
+"""
+import math
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from lossless_bf16_weight_huffman_b200 import _native, api, synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from lossless_bf16_weight_huffman_b200 import build
+
+    build.build_native()
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "df11.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(df_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_function():
+    names = header_functions()
+    assert len(names) >= 15
+    lib = _native.lib()
+    for name in names:
+        assert hasattr(lib, name), name
+    assert sorted(_native.EXPORTS) == names
+
+
+def test_struct_sizes_match_header_layout():
+    import ctypes
+
+    assert ctypes.sizeof(_native.DfCode) == 16 + 256 + 1024
+    assert ctypes.sizeof(_native.DfSizes) == 9 * 8
+    assert ctypes.sizeof(_native.DfTensor) == 16 + 16 + 5 * 8 + 256
+    assert ctypes.sizeof(_native.DfBatchPlan) == 8 + 6 * 4 + 8
+
+
+def _random_hist(rng, kind):
+    h = np.zeros(256, np.uint64)
+    k = int(rng.integers(1, 257))
+    syms = rng.choice(256, size=k, replace=False)
+    if kind == 0:
+        h[syms] = rng.integers(1, 1000, size=k)
+    elif kind == 1:  # heavy tail: long codes
+        h[syms] = (rng.pareto(0.5, size=k) * 50).astype(np.uint64) + 1
+    elif kind == 2:  # many equal counts: ties everywhere
+        h[syms] = rng.integers(1, 4, size=k)
+    elif kind == 3:  # geometric, like real exponents
+        h[syms] = (2.0 ** rng.uniform(0, 40, size=k)).astype(np.uint64) + 1
+    else:  # one dominant symbol and a flat tail
+        h[syms] = 1
+        h[syms[0]] = int(rng.integers(1, 10**9))
+    return h
+
+
+def test_build_code_matches_oracle_on_many_histograms():
+    rng = np.random.default_rng(1234)
+    checked = 0
+    for trial in range(10000):
+        h = _random_hist(rng, trial % 5)
+        k = int((h > 0).sum())
+        lo = max(1, math.ceil(math.log2(k))) if k > 1 else 1
+        max_len = int(rng.integers(lo, 33))
+        want = oracle.package_merge(h, max_len)
+        code = api.df_build_code(h, max_len)
+        got = np.frombuffer(bytes(code.lengths), np.uint8)
+        assert (got == want).all(), (trial, max_len)
+        codes = np.frombuffer(bytes(code.codes), np.uint32)
+        assert (codes == oracle.canonical_codes(want)).all(), trial
+        checked += 1
+    assert checked == 10000
+
+
+def test_build_code_limits():
+    h = np.ones(256, np.uint64)
+    with pytest.raises(_native.DfError):
+        api.df_build_code(h, 7)
+    with pytest.raises(_native.DfError):
+        api.df_build_code(h, 33)
+    code = api.df_build_code(np.zeros(256, np.uint64))
+    assert code.n_symbols == 0 and code.n_tables == 1
+    with pytest.raises(_native.DfError):  # Kraft sum 3/2
+        api.df_code_from_lengths(np.array([1, 1, 1] + [0] * 253, np.uint8))
+
+
+@pytest.mark.parametrize("chunk_bytes,tpb", [(16, 32), (32, 256), (64, 128), (4096, 1024)])
+def test_plan_matches_oracle_sizes(chunk_bytes, tpb):
+    rng = np.random.default_rng(5)
+    for _ in range(200):
+        h = _random_hist(rng, 3)
+        code = api.df_build_code(h, 32)
+        n = int(h.sum())
+        z = api.df_plan(code, h, n, chunk_bytes, tpb).as_dict()
+        want = oracle.sizes(n, oracle.total_bits(h, oracle.package_merge(h, 32)), chunk_bytes, tpb)
+        for key, val in want.items():
+            assert z[key] == val, key
+    with pytest.raises(_native.DfError):
+        api.df_plan(code, h, n + 1, chunk_bytes, tpb)
+    with pytest.raises(_native.DfError):
+        api.df_plan(code, h, n, 24, tpb)
+
+
+# ---------------------------------------------------------------- the decode tables
+
+
+def table_walk_decode(stream, total_bits, n, gaps_fields, offsets, lut, n_tables, chunk_bytes, tpb):
+    """Plain-Python model of the kernel's per-chunk table walk: every chunk is
+    decoded from its start + gap up to its end, codes taken from the root
+    entry (up to three per step while 8 bits remain before the end) or from
+    the next-level tables; counts are checked against the block offsets."""
+    lengths = np.frombuffer(lut[n_tables * 256:].tobytes(), np.uint8)
+    bits = np.unpackbits(np.asarray(stream, np.uint8))
+    cb = 8 * chunk_bytes
+    n_chunks = len(gaps_fields)
+    out = []
+    counts = []
+
+    def window(p):
+        w = bits[p:p + 32]
+        v = 0
+        for b in w:
+            v = (v << 1) | int(b)
+        return v << (32 - len(w))
+
+    for j in range(n_chunks):
+        p = j * cb + int(gaps_fields[j])
+        end = min((j + 1) * cb, total_bits)
+        cnt = 0
+        while p < end:
+            win = window(p)
+            e = int(lut[win >> 24])
+            ns = (e >> 24) & 3
+            if ns == 0:
+                for lvl in (1, 2, 3):
+                    t = e & 0xFFFF
+                    assert t != 0, "unreachable entry"
+                    e = int(lut[t * 256 + ((win >> (24 - 8 * lvl)) & 0xFF)])
+                    if (e >> 24) & 3:
+                        break
+                out.append(e & 0xFF)
+                cnt += 1
+                p += e >> 26
+            elif p + 8 <= end:
+                for k in range(ns):
+                    out.append((e >> (8 * k)) & 0xFF)
+                cnt += ns
+                p += e >> 26
+            else:
+                out.append(e & 0xFF)
+                cnt += 1
+                p += int(lengths[e & 0xFF])
+        counts.append(cnt)
+    counts = np.array(counts)
+    per_block = [int(counts[b * tpb:(b + 1) * tpb].sum()) for b in range(len(offsets) - 1)]
+    assert per_block == list(np.diff(offsets.astype(np.int64)))
+    assert len(out) == n
+    return np.array(out, np.uint8)
+
+
+@pytest.mark.parametrize("case", ["normal", "heavy12", "single", "all256", "heavy9"])
+def test_tables_decode_oracle_streams(case):
+    rng = np.random.default_rng(99)
+    chunk_bytes, tpb, max_len = 16, 32, 32
+    if case == "normal":
+        w = synth.generate(synth.single_1024x4096()[0])[:6000]
+    elif case.startswith("heavy"):
+        w = synth.generate(synth.heavy_tail_64m()[0])
+        # keep rare exponents in the sample so long codes appear
+        e = (w >> 7) & 0xFF
+        rare = np.nonzero(np.bincount(e, minlength=256)[e] < 2000)[0][:300]
+        w = np.concatenate([w[:5000], w[rare]])
+        rng.shuffle(w)
+        max_len = int(case[5:])
+    elif case == "single":
+        w = (0x3F80 | rng.integers(0, 128, size=3000)).astype(np.uint16)
+    else:
+        w = ((np.arange(4096) % 256) << 7).astype(np.uint16)
+    enc = oracle.encode(w, max_len=max_len, chunk_bytes=chunk_bytes, threads_per_block=tpb)
+    code = api.df_code_from_lengths(enc.lengths, max_len)
+    lut = api.df_build_lut(code)
+    exps = table_walk_decode(enc.stream, enc.total_bits, enc.n, oracle.unpack_gaps(enc.gaps, enc.sizes["n_chunks"]),
+                             enc.offsets, lut, code.n_tables, chunk_bytes, tpb)
+    assert (exps == ((w >> 7) & 0xFF)).all()
+
+
+def test_unreachable_entries_are_zero():
+    h = np.zeros(256, np.uint64)
+    h[127] = 10  # one symbol: code '0', so every index starting with bit 1 is unreachable
+    code = api.df_build_code(h)
+    lut = api.df_build_lut(code)
+    assert (lut[128:256] == 0).all() and (lut[:128] != 0).all()
+    # a complete code reaches every root entry
+    code = api.df_build_code(np.arange(1, 257, dtype=np.uint64))
+    lut = api.df_build_lut(code)
+    assert (lut[:256] != 0).all()
