@@ -106,7 +106,7 @@ def test_decode_stream_ends_on_chunk_and_block_boundaries(n_chunks_exact):
     # 8-bit codes: n = 16 * chunks ends exactly on a 16-byte chunk boundary
     n = 16 * n_chunks_exact
     w = (((np.arange(n) * 11) % 256) << 7 | (np.arange(n) % 128)).astype(np.uint16)
-    enc = oracle.encode(w, chunk_bytes=16, threads_per_block=32)
+    enc = oracle.encode(w, chunk_bytes=16, threads_per_block=32, lengths=np.full(256, 8, np.uint8))
     assert enc.total_bits % 128 == 0
     c = from_oracle(enc)
     out, flags = gpu_decode(c)
