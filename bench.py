@@ -56,7 +56,9 @@ def parse():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--e2e-steps", type=int, default=3)
-    p.add_argument("--max-tensors", type=int, default=0, help="debug: use only the first N tensors")
+    p.add_argument("--workload", default="llama8b_shaped",
+                   choices=["llama8b_shaped", "llama_layer", "single_1024x4096", "heavy_tail_64m", "mixed_2000"],
+                   help="weight set to decode (the headline number is llama8b_shaped)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
 
@@ -228,6 +230,13 @@ def cpu_baseline_sample(specs):
     from lossless_bf16_weight_huffman_b200 import synth
 
     layer0 = [s for s in specs if s.name.startswith("layers.0.")]
+    if not layer0:  # another weight set: its first tensors, up to ~2e8 weights
+        layer0, tot = [], 0
+        for s in specs:
+            if tot >= 200_000_000:
+                break
+            layer0.append(s)
+            tot += s.numel
     encs = []
     for s in layer0:
         w = synth.generate(s)
@@ -239,7 +248,8 @@ def cpu_baseline_sample(specs):
         assert (out == w).all()
     dt = time.perf_counter() - t0
     return {"value": round(2 * n / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"layer 0 of the weight set ({n:,} weights), bit-serial decode, one host thread, "
+            "sample": f"{'layer 0' if layer0[0].name.startswith('layers.0.') else 'first tensors'} of the "
+                      f"weight set ({n:,} weights), bit-serial decode, one host thread, "
                       f"{dt:.1f} s"}
 
 
@@ -253,9 +263,7 @@ def run_gpu(args, world, rank, local):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream()
-    specs = synth.llama8b_shaped()
-    if args.max_tensors:
-        specs = specs[: args.max_tensors]
+    specs = synth.weight_set(args.workload)
     n_total = sum(s.numel for s in specs)
     max_n = max(s.numel for s in specs)
 
@@ -340,33 +348,32 @@ def run_gpu(args, world, rank, local):
     achieved = algo_bytes / (launch_ms / 1e3) / 1e9
     traffic = None
     rec = decode_traffic_record()
-    if rec and not args.max_tensors:
+    if rec and args.workload == "llama8b_shaped":
         traffic = int(rec["dram_bytes_per_weight"] * n_total)
 
-    # ---- (ii) layer by layer into one reused buffer
+    # ---- (ii) layer by layer into one reused buffer: the tensors of one decoder
+    # layer share a buffer; every other tensor (embedding, lm_head, ...) uses a
+    # second one
+    groups = []
+    for i, s in enumerate(specs):
+        parts = s.name.split(".")
+        key = ".".join(parts[:2]) if parts[0] == "layers" else None
+        if key is not None and groups and groups[-1][0] == key:
+            groups[-1][1].append(i)
+        else:
+            groups.append((key, [i]))
+    layer_need = max([sum(specs[j].numel for j in idx) for key, idx in groups if key] or [0])
+    other_need = max([specs[idx[0]].numel for key, idx in groups if not key] or [0])
+    layer_buf = torch.empty(layer_need, dtype=torch.int16, device=dev) if layer_need else None
+    other_buf = torch.empty(other_need, dtype=torch.int16, device=dev) if other_need else None
     layer_groups = []
-    layer_buf = None
-    vocab_buf = None
-    names = [s.name for s in specs]
-    i = 0
-    while i < len(specs):
-        if specs[i].name in ("embed_tokens", "lm_head"):
-            if vocab_buf is None:
-                vocab_buf = torch.empty(specs[i].numel, dtype=torch.int16, device=dev)
-            layer_groups.append(([i], [vocab_buf[: specs[i].numel]]))
-            i += 1
-            continue
-        prefix = specs[i].name.split(".")[0] + "." + specs[i].name.split(".")[1] + "."
-        idx = [j for j in range(i, len(specs)) if names[j].startswith(prefix)]
-        tot = sum(specs[j].numel for j in idx)
-        if layer_buf is None or layer_buf.numel() < tot:
-            layer_buf = torch.empty(tot, dtype=torch.int16, device=dev)
+    for key, idx in groups:
+        buf = layer_buf if key else other_buf
         views, off = [], 0
         for j in idx:
-            views.append(layer_buf[off: off + specs[j].numel])
+            views.append(buf[off: off + specs[j].numel])
             off += specs[j].numel
         layer_groups.append((idx, views))
-        i = idx[-1] + 1
     layer_decs = [codec.BatchDecoder([comps[j] for j in idx], views) for idx, views in layer_groups]
     for (idx, views), d in zip(layer_groups, layer_decs):  # verify each group once
         d.run(err)
@@ -395,8 +402,8 @@ def run_gpu(args, world, rank, local):
     for c in comps:
         host_parts.append({k: getattr(c, k).cpu().pin_memory() for k in ("stream", "gaps", "offsets")} |
                           {"sm": c.sm[: c.n].cpu().pin_memory()})
-    host_out = torch.empty(max_n if not layer_groups else max(
-        sum(comps[j].n for j in idx) for idx, _ in layer_groups), dtype=torch.int16, pin_memory=True)
+    host_out = torch.empty(max(sum(comps[j].n for j in idx) for idx, _ in layer_groups), dtype=torch.int16,
+                           pin_memory=True)
     h2d = sum(sum(p.numel() * p.element_size() for p in hp.values()) for hp in host_parts)
     d2h = bf16_bytes
 
@@ -453,8 +460,11 @@ def run_gpu(args, world, rank, local):
             "vs_baseline": None,
             "dtype": "u8",
             "data": "synthetic (seeded; Box-Muller normals rounded to BF16, shapes of an 8B Llama-style model)",
-            "config": {"workload": WORKLOAD, "weights": n_total, "tensors": len(specs), "chunk_bytes": 32,
-                       "threads_per_block": 256, "max_len": 32, "l2": "inputs (16 GB) larger than L2: no flush",
+            "config": {"workload": WORKLOAD if args.workload == "llama8b_shaped" else args.workload,
+                       "weights": n_total, "tensors": len(specs), "chunk_bytes": 32,
+                       "threads_per_block": 256, "max_len": 32,
+                       "l2": f"inputs ({(read_bytes + bf16_bytes) / 1e9:.2f} GB) larger than L2: no flush"
+                       if read_bytes + bf16_bytes > 2 * 126e6 else "L2-resident (no flush)",
                        "parallelism": f"{world} replica(s), no collective" if world > 1 else "1 GPU"},
             "weights_per_s": round(world * n_total * args.steps / (total_ms_max / 1e3), 1),
             "compressed_pct": round(100.0 * container / bf16_bytes, 4),
