@@ -150,10 +150,12 @@ size_t df_lut_words(const df_code* code);
 /* df_build_lut: derive the decode tables of a code into host memory `lut`
  * (lut_words >= df_lut_words(code)). Table 0 is indexed by the next 8 stream
  * bits; an entry holds up to three whole codes that fit in those 8 bits
- * (symbols in bits 0-23, their count in bits 24-25, the bits they use in bits
- * 26-31), or, for a longer code, count 0 and the index of a next-level table
- * (bits 0-15) indexed by the following 8 bits, at most four levels for 32-bit
- * codes. Entries no code reaches are zero. The caller copies the words to the
+ * (exponents in bits 0-23, their count in bits 24-25, the bits they use minus
+ * one in bits 26-28, the first code's length minus one in bits 29-31), or,
+ * for a longer code, count 0 and the index of a next-level table (bits 0-15)
+ * indexed by the following 8 bits, at most four levels for 32-bit codes. A
+ * next-level leaf holds one exponent (bits 0-7), its full code length (bits
+ * 8-13) and count 1. Entries no code reaches are zero. The caller copies the words to the
  * device and passes them as df_tensor.lut. Source: df11pack, "What is
  * checked" (--luts=correct zero-fills unreachable table entries).
  * Errors: DF_ERR_INVALID_ARG (null, too small, or a code that is not prefix free).

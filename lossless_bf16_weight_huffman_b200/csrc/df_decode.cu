@@ -6,7 +6,7 @@
 // The layout of the work below is this library's own, written for sm_100a:
 //
 //   one CUDA block = one format block = T chunks of C bytes of stream
-//   1. stage the decode tables, the code lengths and the block's stream slice
+//   1. stage the decode tables and the block's stream slice
 //      (byte-swapped to big-endian words) in shared memory
 //   2. count pass: thread t decodes the codes that start in chunk t
 //      (from chunk start + gap, up to the chunk end or the end of the stream)
@@ -14,8 +14,8 @@
 //   3. block scan of the counts: each thread's first output position
 //   4. check the block total against the block offsets (corrupt -> error bit)
 //   5. write pass: decode again, exponent bytes into a shared-memory stage
-//      placed so that stage index == output index mod 8
-//   6. merge with the sign|fraction bytes: 8 weights per 16-byte store
+//      placed so that stage index == output index mod 16
+//   6. merge with the sign|fraction bytes: 16 weights per pair of 16-byte stores
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -66,10 +66,11 @@ struct LaunchCfg {
 __device__ __forceinline__ uint32_t bswap32(uint32_t x) { return __byte_perm(x, 0, 0x0123); }
 
 // Next-level lookup for codes longer than 8 bits. `win` holds the 32 bits
-// starting at the code; returns the leaf entry, or 0 for an unreachable path.
-__device__ __noinline__ uint32_t descend(uint32_t win, uint32_t e, const uint32_t* s_lut, const uint32_t* g_lut,
-                                         uint32_t smem_tables) {
-#pragma unroll 1
+// starting at the code; returns the next-level leaf (exponent in bits 0-7,
+// length in bits 8-13, count 1), or 0 for a path no code takes.
+__device__ __forceinline__ uint32_t descend(uint32_t win, uint32_t e, const uint32_t* s_lut, const uint32_t* g_lut,
+                                            uint32_t smem_tables) {
+#pragma unroll
     for (int lvl = 1; lvl <= 3; ++lvl) {
         const uint32_t t = e & 0xFFFFu;
         if (t == 0) return 0;
@@ -104,57 +105,48 @@ struct BitWindow {
 };
 
 // Decode the codes that start in [p, end). kWrite=false counts them,
-// kWrite=true stores their exponents at stage[pos...]. Returns the count, or
-// sets *bad on an unreachable table entry.
+// kWrite=true also stores their exponents at stage[pos...]. Returns the
+// count; an unreachable table entry sets *bad and ends the chunk.
+// The loop runs in step across the warp (one vote per step) so that lanes
+// that took the long-code path rejoin the others at once.
 template <bool kWrite>
 __device__ __forceinline__ uint32_t decode_chunk(const uint32_t* s_words, uint32_t p, uint32_t end,
-                                                 const uint32_t* s_lut, const uint8_t* s_len, const uint32_t* g_lut,
-                                                 uint32_t smem_tables, uint8_t* stage, uint32_t pos, bool* bad) {
+                                                 const uint32_t* s_lut, const uint32_t* g_lut, uint32_t smem_tables,
+                                                 uint8_t* stage, uint32_t pos, bool* bad) {
     BitWindow bw;
     bw.init(s_words, p);
     uint32_t cnt = 0;
-    // whole-table steps while all 8 indexed bits lie before `end`
-    while (p + 8 <= end) {
-        const uint32_t win = bw.peek();
-        uint32_t e = s_lut[win >> 24];
-        uint32_t ns = (e >> kNsymShift) & 3u;
-        if (ns == 0) {
-            e = descend(win, e, s_lut, g_lut, smem_tables);
-            ns = (e >> kNsymShift) & 3u;
-            if (ns == 0) {
-                *bad = true;
-                return cnt;
+    for (;;) {
+        const bool act = p < end;
+        if (!__any_sync(0xFFFFFFFFu, act)) break;
+        if (act) {
+            const uint32_t win = bw.peek();
+            uint32_t e = s_lut[win >> 24];
+            uint32_t ns = (e >> kNsymShift) & 3u;
+            uint32_t nb;
+            if (ns == 0) {  // a code longer than 8 bits (or corrupt data)
+                e = descend(win, e, s_lut, g_lut, smem_tables);
+                ns = (e >> kNsymShift) & 3u;
+                nb = (e >> 8) & 63u;
+                if (ns == 0) {
+                    *bad = true;
+                    end = p;
+                }
+            } else if (p + 8 > end) {  // near the end: only the first code surely starts before it
+                ns = 1;
+                nb = (e >> 29) + 1;
+            } else {
+                nb = ((e >> 26) & 7u) + 1;
             }
-        }
-        if (kWrite) {
-            stage[pos + cnt] = static_cast<uint8_t>(e);
-            if (ns > 1) stage[pos + cnt + 1] = static_cast<uint8_t>(e >> 8);
-            if (ns > 2) stage[pos + cnt + 2] = static_cast<uint8_t>(e >> 16);
-        }
-        cnt += ns;
-        const uint32_t nb = e >> kNbitsShift;
-        p += nb;
-        bw.skip(nb);
-    }
-    // the last few bits: one code at a time
-    while (p < end) {
-        const uint32_t win = bw.peek();
-        uint32_t e = s_lut[win >> 24];
-        uint32_t nb;
-        if (((e >> kNsymShift) & 3u) == 0) {
-            e = descend(win, e, s_lut, g_lut, smem_tables);
-            if (((e >> kNsymShift) & 3u) == 0) {
-                *bad = true;
-                return cnt;
+            if (kWrite) {
+                if (ns > 0) stage[pos + cnt] = static_cast<uint8_t>(e);
+                if (ns > 1) stage[pos + cnt + 1] = static_cast<uint8_t>(e >> 8);
+                if (ns > 2) stage[pos + cnt + 2] = static_cast<uint8_t>(e >> 16);
             }
-            nb = e >> kNbitsShift;
-        } else {
-            nb = s_len[e & 0xFFu];
+            cnt += ns;
+            p += nb;
+            bw.skip(nb);
         }
-        if (kWrite) stage[pos + cnt] = static_cast<uint8_t>(e);
-        ++cnt;
-        p += nb;
-        bw.skip(nb);
     }
     return cnt;
 }
@@ -188,19 +180,16 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(Src src, LaunchCfg 
 
         // shared memory carve-up
         uint32_t* s_lut = reinterpret_cast<uint32_t*>(smem);
-        uint8_t* s_len = smem + static_cast<size_t>(cfg.smem_tables) * 1024;
-        uint32_t* s_words = reinterpret_cast<uint32_t*>(s_len + 256);
+        uint32_t* s_words = reinterpret_cast<uint32_t*>(smem + static_cast<size_t>(cfg.smem_tables) * 1024);
         const uint32_t slice_words = T * C / 4 + 4;
         uint32_t* s_warp = s_words + slice_words;
         uint8_t* s_stage = reinterpret_cast<uint8_t*>(s_warp + 32);
 
-        // 1. tables, lengths, stream slice
+        // 1. tables, stream slice
         {
             const uint4* src4 = reinterpret_cast<const uint4*>(td->lut);
             uint4* dst4 = reinterpret_cast<uint4*>(s_lut);
             for (uint32_t i = tid; i < stab * 64; i += T) dst4[i] = __ldg(src4 + i);
-            const uint4* len4 = reinterpret_cast<const uint4*>(td->lut + static_cast<size_t>(n_tables) * 256);
-            if (tid < 16) reinterpret_cast<uint4*>(s_len)[tid] = __ldg(len4 + tid);
             const uint64_t slice_byte0 = b * static_cast<uint64_t>(T) * C;
             const uint64_t stream_bytes = td->n_chunks * C + 16;
             const uint64_t avail = stream_bytes - slice_byte0;
@@ -239,7 +228,7 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(Src src, LaunchCfg 
 
         // 2. count pass
         bool bad = false;
-        const uint32_t cnt = decode_chunk<false>(s_words, p0, end, s_lut, s_len, td->lut, stab, nullptr, 0, &bad);
+        const uint32_t cnt = decode_chunk<false>(s_words, p0, end, s_lut, td->lut, stab, nullptr, 0, &bad);
 
         // 3. block scan
         const int lane = tid & 31, warp = tid >> 5;
@@ -257,7 +246,7 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(Src src, LaunchCfg 
         const uint32_t total = s_warp[nwarps - 1];
 
         // 4. consistency with the block index
-        const uint32_t align = static_cast<uint32_t>(out0 & 7);
+        const uint32_t align = static_cast<uint32_t>(out0 & 15);
         uint32_t flags = 0;
         if (out1 < out0 || out1 > td->n || out1 - out0 + align > cfg.stage_bytes ||
             (b + 1 == td->n_blocks && out1 != td->n))
@@ -272,38 +261,53 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(Src src, LaunchCfg 
         }
 
         // 5. write pass into the stage
-        decode_chunk<true>(s_words, p0, end, s_lut, s_len, td->lut, stab, s_stage, align + excl, &bad);
+        decode_chunk<true>(s_words, p0, end, s_lut, td->lut, stab, s_stage, align + excl, &bad);
         __syncthreads();
 
-        // 6. merge and store
+        // 6. merge and store: 16 weights per group (one 16-byte load of
+        // sign|fraction bytes, one of staged exponents, two 16-byte stores);
+        // two groups per thread per step keep two loads in flight
         const uint8_t* sm = td->sm;
         uint16_t* out = td->out;
-        const uint64_t gbase = out0 & ~7ull;  // stage index 0 <-> output gbase
-        const uint64_t ngroups = (out1 - gbase + 7) >> 3;
-        for (uint64_t gi = tid; gi < ngroups; gi += T) {
-            const uint64_t G = gbase + 8 * gi;
-            const uint32_t si = static_cast<uint32_t>(8 * gi);
-            if (td->vec_ok && G >= out0 && G + 8 <= out1) {
-                const uint2 s8 = *reinterpret_cast<const uint2*>(sm + G);
-                const uint2 e8 = *reinterpret_cast<const uint2*>(s_stage + si);
-                uint4 o;
-                {
-                    const uint32_t hi = (s8.x & 0x80808080u) | ((e8.x >> 1) & 0x7F7F7F7Fu);
-                    const uint32_t lo = ((e8.x << 7) & 0x80808080u) | (s8.x & 0x7F7F7F7Fu);
-                    o.x = __byte_perm(lo, hi, 0x5140);
-                    o.y = __byte_perm(lo, hi, 0x7362);
-                }
-                {
-                    const uint32_t hi = (s8.y & 0x80808080u) | ((e8.y >> 1) & 0x7F7F7F7Fu);
-                    const uint32_t lo = ((e8.y << 7) & 0x80808080u) | (s8.y & 0x7F7F7F7Fu);
-                    o.z = __byte_perm(lo, hi, 0x5140);
-                    o.w = __byte_perm(lo, hi, 0x7362);
-                }
-                *reinterpret_cast<uint4*>(out + G) = o;
-            } else {
-                for (uint32_t k = 0; k < 8; ++k) {
-                    const uint64_t i = G + k;
-                    if (i >= out0 && i < out1) out[i] = merge1(sm[i], s_stage[si + k]);
+        const uint64_t gbase = out0 & ~15ull;  // stage index 0 <-> output gbase
+        const uint64_t ngroups = (out1 - gbase + 15) >> 4;
+        const bool vec = td->vec_ok != 0;
+        for (uint64_t g0 = tid; g0 < ngroups; g0 += 2 * static_cast<uint64_t>(T)) {
+            uint4 s16[2];
+            bool full[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const uint64_t gi = g0 + static_cast<uint64_t>(u) * T;
+                const uint64_t G = gbase + 16 * gi;
+                full[u] = vec && gi < ngroups && G >= out0 && G + 16 <= out1;
+                if (full[u]) s16[u] = __ldg(reinterpret_cast<const uint4*>(sm + G));
+            }
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const uint64_t gi = g0 + static_cast<uint64_t>(u) * T;
+                if (gi >= ngroups) continue;
+                const uint64_t G = gbase + 16 * gi;
+                const uint32_t si = static_cast<uint32_t>(16 * gi);
+                if (full[u]) {
+                    const uint4 e16 = *reinterpret_cast<const uint4*>(s_stage + si);
+                    const uint32_t sw[4] = {s16[u].x, s16[u].y, s16[u].z, s16[u].w};
+                    const uint32_t ew[4] = {e16.x, e16.y, e16.z, e16.w};
+                    uint32_t o[8];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint32_t hi = (sw[k] & 0x80808080u) | ((ew[k] >> 1) & 0x7F7F7F7Fu);
+                        const uint32_t lo = ((ew[k] << 7) & 0x80808080u) | (sw[k] & 0x7F7F7F7Fu);
+                        o[2 * k] = __byte_perm(lo, hi, 0x5140);
+                        o[2 * k + 1] = __byte_perm(lo, hi, 0x7362);
+                    }
+                    uint4* dst = reinterpret_cast<uint4*>(out + G);
+                    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+                    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+                } else {
+                    for (uint32_t k = 0; k < 16; ++k) {
+                        const uint64_t i = G + k;
+                        if (i >= out0 && i < out1) out[i] = merge1(sm[i], s_stage[si + k]);
+                    }
                 }
             }
         }
@@ -356,19 +360,19 @@ df_status prepare(const df_tensor* t, uint16_t* out, Prepared* pr) {
     d.n_chunks = n_chunks;
     d.n_blocks = static_cast<uint32_t>(n_blocks);
     d.n_tables = t->n_tables;
-    d.vec_ok = aligned(t->sm, 8) && aligned(out, 16);
+    d.vec_ok = aligned(t->sm, 16) && aligned(out, 16);
     pr->dev = d;
     // a block holds at most 8CT/min_len codes, and never more than n
     uint64_t need = minl ? (cbits * T + minl - 1) / minl : 0;
     if (need > t->n) need = t->n;
-    need = (need + 8 + 15) & ~15ull;  // + alignment slack
+    need = (need + 16 + 15) & ~15ull;  // + alignment slack
     if (need > (1u << 30)) return DF_ERR_UNSUPPORTED;
     pr->stage_need = static_cast<uint32_t>(need);
     return DF_OK;
 }
 
 size_t smem_bytes(uint32_t tables, uint32_t C, uint32_t T, uint32_t stage) {
-    return static_cast<size_t>(tables) * 1024 + 256 + (static_cast<size_t>(T) * C / 4 + 4) * 4 + 32 * 4 + stage;
+    return static_cast<size_t>(tables) * 1024 + (static_cast<size_t>(T) * C / 4 + 4) * 4 + 32 * 4 + stage;
 }
 
 df_status device_limits(int* sms, int* max_smem) {

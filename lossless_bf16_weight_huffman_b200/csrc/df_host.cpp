@@ -209,10 +209,11 @@ df_status df_build_lut(const df_code* code, uint32_t* lut, size_t lut_words) {
         const uint32_t e0 = tables[x];
         uint32_t nsym = (e0 >> kNsymShift) & 3u;
         if (!nsym) {
-            lut[x] = e0;
+            lut[x] = e0;  // a link (count 0, table index) or an unreachable 0
             continue;
         }
-        uint32_t used = e0 >> kNbitsShift;
+        const uint32_t len0 = e0 >> kNbitsShift;
+        uint32_t used = len0;
         uint32_t syms = e0 & 0xFFu;
         while (nsym < 3 && used < 8) {
             const uint32_t y = (x << used) & 0xFFu;  // the unknown low bits read as 0
@@ -223,9 +224,13 @@ df_status df_build_lut(const df_code* code, uint32_t* lut, size_t lut_words) {
             used += l;
             ++nsym;
         }
-        lut[x] = lut_leaf(syms, nsym, used);
+        lut[x] = root_entry(syms, nsym, used, len0);
     }
-    std::memcpy(lut + 256, tables.data() + 256, (tables.size() - 256) * sizeof(uint32_t));
+    // next-level entries: one code each, with its full length
+    for (size_t i = 256; i < tables.size(); ++i) {
+        const uint32_t e = tables[i];
+        lut[i] = ((e >> kNsymShift) & 3u) ? sub_leaf(e & 0xFFu, e >> kNbitsShift) : e;
+    }
     std::memcpy(lut + static_cast<size_t>(code->n_tables) * 256, code->lengths, 256);
     return DF_OK;
 }

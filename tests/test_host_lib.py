@@ -118,9 +118,9 @@ def test_plan_matches_oracle_sizes(chunk_bytes, tpb):
 def table_walk_decode(stream, total_bits, n, gaps_fields, offsets, lut, n_tables, chunk_bytes, tpb):
     """Plain-Python model of the kernel's per-chunk table walk: every chunk is
     decoded from its start + gap up to its end, codes taken from the root
-    entry (up to three per step while 8 bits remain before the end) or from
-    the next-level tables; counts are checked against the block offsets."""
-    lengths = np.frombuffer(lut[n_tables * 256:].tobytes(), np.uint8)
+    entry (up to three per step while 8 bits remain before the end, else only
+    the first) or from the next-level tables; counts are checked against the
+    block offsets."""
     bits = np.unpackbits(np.asarray(stream, np.uint8))
     cb = 8 * chunk_bytes
     n_chunks = len(gaps_fields)
@@ -149,18 +149,19 @@ def table_walk_decode(stream, total_bits, n, gaps_fields, offsets, lut, n_tables
                     e = int(lut[t * 256 + ((win >> (24 - 8 * lvl)) & 0xFF)])
                     if (e >> 24) & 3:
                         break
+                assert (e >> 24) & 3 == 1
                 out.append(e & 0xFF)
                 cnt += 1
-                p += e >> 26
+                p += (e >> 8) & 63
             elif p + 8 <= end:
                 for k in range(ns):
                     out.append((e >> (8 * k)) & 0xFF)
                 cnt += ns
-                p += e >> 26
+                p += ((e >> 26) & 7) + 1
             else:
                 out.append(e & 0xFF)
                 cnt += 1
-                p += int(lengths[e & 0xFF])
+                p += (e >> 29) + 1
         counts.append(cnt)
     counts = np.array(counts)
     per_block = [int(counts[b * tpb:(b + 1) * tpb].sum()) for b in range(len(offsets) - 1)]
