@@ -107,13 +107,13 @@ typedef struct df_tensor {
 
 /* Host plan of a grouped decode, filled by df_decode_batch_prepare. */
 typedef struct df_batch_plan {
-    void* d_ws;              /* the workspace holding the device table  */
-    uint32_t count;          /* tensors with n > 0                      */
+    void* d_ws;                /* the workspace holding the device table      */
+    uint32_t count;            /* tensors with n > 0                          */
     uint32_t threads_per_block;
-    uint32_t chunk_bytes;
-    uint32_t smem_tables;    /* decode tables staged in shared memory   */
-    uint32_t stage_bytes;    /* exponent staging bytes per block        */
-    uint32_t smem_bytes;     /* dynamic shared memory per block         */
+    uint32_t words_per_chunk;  /* shared-memory words per chunk (widest C)    */
+    uint32_t region_bytes;     /* per-thread exponent region in shared memory */
+    uint32_t max_groups;       /* 16-weight output groups per block, at most  */
+    uint32_t smem_bytes;       /* dynamic shared memory per CUDA block        */
     uint64_t total_blocks;
 } df_batch_plan;
 
@@ -217,7 +217,8 @@ size_t df_decode_batch_workspace(uint32_t count);
 /* df_decode_batch_prepare: validate `count` descriptors (host array) and
  * their outputs (host array of device pointers), write the device table into
  * d_ws (asynchronously on `stream`; the host arrays may be reused on return)
- * and fill *plan. All tensors must share chunk_bytes and threads_per_block.
+ * and fill *plan. All tensors must share threads_per_block; chunk_bytes may
+ * differ (shared memory is sized for the widest).
  * Errors: DF_ERR_INVALID_ARG, DF_ERR_WORKSPACE, DF_ERR_UNSUPPORTED, DF_ERR_CUDA. */
 df_status df_decode_batch_prepare(const df_tensor* tensors, uint16_t* const* d_outs, uint32_t count, void* d_ws,
                                   size_t ws_bytes, df_batch_plan* plan, void* stream);

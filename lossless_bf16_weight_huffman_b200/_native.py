@@ -85,9 +85,9 @@ class DfBatchPlan(ctypes.Structure):
         ("d_ws", ctypes.c_void_p),
         ("count", ctypes.c_uint32),
         ("threads_per_block", ctypes.c_uint32),
-        ("chunk_bytes", ctypes.c_uint32),
-        ("smem_tables", ctypes.c_uint32),
-        ("stage_bytes", ctypes.c_uint32),
+        ("words_per_chunk", ctypes.c_uint32),
+        ("region_bytes", ctypes.c_uint32),
+        ("max_groups", ctypes.c_uint32),
         ("smem_bytes", ctypes.c_uint32),
         ("total_blocks", ctypes.c_uint64),
     ]

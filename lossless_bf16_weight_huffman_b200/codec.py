@@ -108,10 +108,17 @@ class Compressed:
                    sm=t(sm_arr if sm_arr.size else np.zeros(16, np.uint8), np.uint8))
 
 
-def compress(w: torch.Tensor, max_len: int = DEFAULT_MAX_LEN, chunk_bytes: int = DEFAULT_CHUNK_BYTES,
+def auto_chunk_bytes(code) -> int:
+    """32-byte chunks; 16 when the shortest code is 1 bit, so that no chunk
+    holds more than 128 codes (the decoder's per-thread region stays small)."""
+    return DEFAULT_CHUNK_BYTES if code.min_len >= 2 else 16
+
+
+def compress(w: torch.Tensor, max_len: int = DEFAULT_MAX_LEN, chunk_bytes: int | None = None,
              threads_per_block: int = DEFAULT_THREADS_PER_BLOCK, d_err: torch.Tensor | None = None,
              stream=None) -> Compressed:
-    """Histogram on the GPU, code build on the host, encode on the GPU."""
+    """Histogram on the GPU, code build on the host, encode on the GPU.
+    chunk_bytes=None picks auto_chunk_bytes(code)."""
     x = _as_u16(w)
     dev = x.device
     n = x.numel()
@@ -119,6 +126,8 @@ def compress(w: torch.Tensor, max_len: int = DEFAULT_MAX_LEN, chunk_bytes: int =
     api.df_histogram(x, hist_d, stream)
     hist = hist_d.cpu().numpy().view(np.uint64)
     code = api.df_build_code(hist, max_len)
+    if chunk_bytes is None:
+        chunk_bytes = auto_chunk_bytes(code)
     lut = torch.from_numpy(api.df_build_lut(code).view(np.int32)).to(dev)
     z = api.df_plan(code, hist, n, chunk_bytes, threads_per_block).as_dict()
     stream_buf = torch.empty(z["stream_bytes"], dtype=torch.uint8, device=dev)

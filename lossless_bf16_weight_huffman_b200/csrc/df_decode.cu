@@ -3,19 +3,25 @@
 // The pages fix what decoding restores (mlx-dfloat, PyPI page, intro: the
 // exponent code is undone and the raw sign|fraction byte put back, bit for bit)
 // and that it runs blockwise on the GPU (mlx-dfloat, "Status"; df11pack, intro).
-// The layout of the work below is this library's own, written for sm_100a:
+// The layout of the work below is this library's own, written for sm_100a.
 //
-//   one CUDA block = one format block = T chunks of C bytes of stream
-//   1. stage the decode tables and the block's stream slice
-//      (byte-swapped to big-endian words) in shared memory
-//   2. count pass: thread t decodes the codes that start in chunk t
-//      (from chunk start + gap, up to the chunk end or the end of the stream)
-//      through the 8-bit multi-code root table and counts them
-//   3. block scan of the counts: each thread's first output position
-//   4. check the block total against the block offsets (corrupt -> error bit)
-//   5. write pass: decode again, exponent bytes into a shared-memory stage
-//      placed so that stage index == output index mod 16
-//   6. merge with the sign|fraction bytes: 16 weights per pair of 16-byte stores
+// One CUDA block handles one format block (T chunks of C stream bytes) at a
+// time and loops over the blocks of all tensors of the launch:
+//   1. when the tensor changes, stage its 11-bit multi-code table (codes that
+//      lie wholly inside an 11-bit window: start mask, bits used, exponents)
+//      in shared memory; stage the block's stream slice, one chunk per thread,
+//      byte-swapped to big-endian words at an odd word stride (no bank
+//      conflicts between the threads' windows)
+//   2. one decode pass per thread over its chunk, from chunk start + gap to
+//      the chunk end: each table step yields up to 4 codes; their exponents
+//      go to the thread's own word-aligned shared-memory region with 32-bit
+//      stores; codes longer than 11 bits walk the 8-bit-indexed tables
+//   3. block scan of the code counts (warp shuffles + one shared array): the
+//      first output position of every thread; checked against the block index
+//   4. an owner map: for every group of 16 outputs, the thread whose region
+//      holds its first exponent
+//   5. merge: per group, 16 exponents gathered from the owner's region, one
+//      16-byte load of sign|fraction bytes, two 16-byte BF16 stores
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -28,7 +34,7 @@ namespace df {
 namespace {
 
 constexpr int kMaxThreads = 1024;
-constexpr uint32_t kSmemTableCap = 16;  // decode tables staged in shared memory
+constexpr uint32_t kWideN = 1u << kWideBits;
 
 struct SingleSrc {
     DevTensor t;
@@ -57,98 +63,34 @@ struct BatchSrc {
 };
 
 struct LaunchCfg {
-    uint32_t chunk_bytes;
-    uint32_t smem_tables;
-    uint32_t stage_bytes;
+    uint32_t words_per_chunk;  // shared-memory stride of a chunk (odd)
+    uint32_t region_bytes;     // private exponent region per thread (4 * odd)
+    uint32_t max_groups;       // owner-map entries
+    uint32_t pad;
     uint64_t total_blocks;
 };
 
 __device__ __forceinline__ uint32_t bswap32(uint32_t x) { return __byte_perm(x, 0, 0x0123); }
 
-// Next-level lookup for codes longer than 8 bits. `win` holds the 32 bits
-// starting at the code; returns the next-level leaf (exponent in bits 0-7,
-// length in bits 8-13, count 1), or 0 for a path no code takes.
-__device__ __forceinline__ uint32_t descend(uint32_t win, uint32_t e, const uint32_t* s_lut, const uint32_t* g_lut,
-                                            uint32_t smem_tables) {
-#pragma unroll
+// Codes longer than the wide window: walk the 8-bit-indexed tables (global
+// memory, cached). Returns the leaf (exponent bits 0-7, length bits 8-13,
+// count 1 in bits 24-25) or 0 for a bit pattern no code starts with.
+__device__ __noinline__ uint32_t long_code(uint32_t win, const uint32_t* __restrict__ hier) {
+    uint32_t e = __ldg(hier + (win >> 24));
+#pragma unroll 1
     for (int lvl = 1; lvl <= 3; ++lvl) {
+        if ((e >> kNsymShift) & 3u) return e;
         const uint32_t t = e & 0xFFFFu;
         if (t == 0) return 0;
-        const uint32_t idx = (win >> (24 - 8 * lvl)) & 0xFFu;
-        e = t < smem_tables ? s_lut[t * 256 + idx] : __ldg(g_lut + static_cast<size_t>(t) * 256 + idx);
-        if ((e >> kNsymShift) & 3u) return e;
+        e = __ldg(hier + static_cast<size_t>(t) * 256 + ((win >> (24 - 8 * lvl)) & 0xFFu));
     }
-    return 0;
+    return ((e >> kNsymShift) & 3u) ? e : 0;
 }
 
-struct BitWindow {
-    const uint32_t* words;
-    uint32_t wi, sh, cur, nxt;
-    __device__ __forceinline__ void init(const uint32_t* w, uint32_t p) {
-        words = w;
-        wi = p >> 5;
-        sh = p & 31;
-        cur = w[wi];
-        nxt = w[wi + 1];
-    }
-    // the 32 stream bits starting at the current position
-    __device__ __forceinline__ uint32_t peek() const { return __funnelshift_l(nxt, cur, sh); }
-    __device__ __forceinline__ void skip(uint32_t nb) {
-        sh += nb;
-        if (sh >= 32) {
-            sh -= 32;
-            cur = nxt;
-            ++wi;
-            nxt = words[wi + 1];
-        }
-    }
-};
-
-// Decode the codes that start in [p, end). kWrite=false counts them,
-// kWrite=true also stores their exponents at stage[pos...]. Returns the
-// count; an unreachable table entry sets *bad and ends the chunk.
-// The loop runs in step across the warp (one vote per step) so that lanes
-// that took the long-code path rejoin the others at once.
-template <bool kWrite>
-__device__ __forceinline__ uint32_t decode_chunk(const uint32_t* s_words, uint32_t p, uint32_t end,
-                                                 const uint32_t* s_lut, const uint32_t* g_lut, uint32_t smem_tables,
-                                                 uint8_t* stage, uint32_t pos, bool* bad) {
-    BitWindow bw;
-    bw.init(s_words, p);
-    uint32_t cnt = 0;
-    for (;;) {
-        const bool act = p < end;
-        if (!__any_sync(0xFFFFFFFFu, act)) break;
-        if (act) {
-            const uint32_t win = bw.peek();
-            uint32_t e = s_lut[win >> 24];
-            uint32_t ns = (e >> kNsymShift) & 3u;
-            uint32_t nb;
-            if (ns == 0) {  // a code longer than 8 bits (or corrupt data)
-                e = descend(win, e, s_lut, g_lut, smem_tables);
-                ns = (e >> kNsymShift) & 3u;
-                nb = (e >> 8) & 63u;
-                if (ns == 0) {
-                    *bad = true;
-                    end = p;
-                }
-            } else if (p + 8 > end) {  // near the end: only the first code surely starts before it
-                ns = 1;
-                nb = (e >> 29) + 1;
-            } else {
-                nb = ((e >> 26) & 7u) + 1;
-            }
-            if (kWrite) {
-                if (ns > 0) stage[pos + cnt] = static_cast<uint8_t>(e);
-                if (ns > 1) stage[pos + cnt + 1] = static_cast<uint8_t>(e >> 8);
-                if (ns > 2) stage[pos + cnt + 2] = static_cast<uint8_t>(e >> 16);
-            }
-            cnt += ns;
-            p += nb;
-            bw.skip(nb);
-        }
-    }
-    return cnt;
+// The 32 stream bits from bit p of a chunk whose big-endian words start at w.
+__device__ __forceinline__ uint32_t window(const uint32_t* w, uint32_t p) {
+    const uint32_t i = p >> 5;
+    return __funnelshift_l(w[i + 1], w[i], p);
 }
 
 __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v, int lane) {
@@ -165,149 +107,221 @@ __device__ __forceinline__ uint16_t merge1(uint8_t sm, uint8_t e) {
                                  (sm & 0x7Fu));
 }
 
+// 4 BF16 weights from 4 sign|fraction bytes and 4 exponent bytes: the high
+// byte of weight k is s | e >> 1, the low byte (e & 1) << 7 | fraction.
+__device__ __forceinline__ void merge4(uint32_t s, uint32_t e, uint32_t* o0, uint32_t* o1) {
+    const uint32_t hi = (s & 0x80808080u) | ((e >> 1) & 0x7F7F7F7Fu);
+    const uint32_t lo = ((e << 7) & 0x80808080u) | (s & 0x7F7F7F7Fu);
+    *o0 = __byte_perm(lo, hi, 0x5140);
+    *o1 = __byte_perm(lo, hi, 0x7362);
+}
+
 template <class Src>
-__global__ void __launch_bounds__(kMaxThreads) decode_kernel(Src src, LaunchCfg cfg, uint32_t* d_err) {
+__global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_constant__ Src src, const LaunchCfg cfg,
+                                                             uint32_t* d_err) {
     extern __shared__ __align__(16) uint8_t smem[];
     const uint32_t T = blockDim.x;
     const uint32_t tid = threadIdx.x;
-    const uint32_t C = cfg.chunk_bytes;
+    const int lane = tid & 31, warp = tid >> 5;
+    const uint32_t nwarps = T >> 5;
 
+    // shared memory carve-up (sizes in smem_bytes())
+    uint16_t* s_meta = reinterpret_cast<uint16_t*>(smem);
+    uint32_t* s_sym = reinterpret_cast<uint32_t*>(smem + 2 * kWideN);
+    uint32_t* s_words = s_sym + kWideN;
+    uint32_t* s_pos = s_words + T * cfg.words_per_chunk;
+    uint32_t* s_warp = s_pos + ((T + 1 + 3) & ~3u);
+    uint16_t* s_owner = reinterpret_cast<uint16_t*>(s_warp + 32);
+    uint8_t* s_priv = reinterpret_cast<uint8_t*>(s_owner) + ((cfg.max_groups * 2 + 15) & ~15u);
+    uint32_t* my_region = reinterpret_cast<uint32_t*>(s_priv + tid * cfg.region_bytes);
+    const uint32_t region_words = cfg.region_bytes / 4;
+
+    const DevTensor* staged = nullptr;
     for (uint64_t g = blockIdx.x; g < cfg.total_blocks; g += gridDim.x) {
         uint64_t b;
         const DevTensor* td = src.lookup(g, &b);
-        const uint32_t n_tables = td->n_tables;
-        const uint32_t stab = n_tables < cfg.smem_tables ? n_tables : cfg.smem_tables;
-
-        // shared memory carve-up
-        uint32_t* s_lut = reinterpret_cast<uint32_t*>(smem);
-        uint32_t* s_words = reinterpret_cast<uint32_t*>(smem + static_cast<size_t>(cfg.smem_tables) * 1024);
-        const uint32_t slice_words = T * C / 4 + 4;
-        uint32_t* s_warp = s_words + slice_words;
-        uint8_t* s_stage = reinterpret_cast<uint8_t*>(s_warp + 32);
-
-        // 1. tables, stream slice
-        {
-            const uint4* src4 = reinterpret_cast<const uint4*>(td->lut);
-            uint4* dst4 = reinterpret_cast<uint4*>(s_lut);
-            for (uint32_t i = tid; i < stab * 64; i += T) dst4[i] = __ldg(src4 + i);
-            const uint64_t slice_byte0 = b * static_cast<uint64_t>(T) * C;
-            const uint64_t stream_bytes = td->n_chunks * C + 16;
-            const uint64_t avail = stream_bytes - slice_byte0;
-            const uint32_t want16 = slice_words / 4;  // uint4 units
-            const uint32_t have16 = avail / 16 < want16 ? static_cast<uint32_t>(avail / 16) : want16;
-            const uint4* s4 = reinterpret_cast<const uint4*>(td->stream + slice_byte0);
-            uint4* d4 = reinterpret_cast<uint4*>(s_words);
-            for (uint32_t i = tid; i < want16; i += T) {
-                uint4 v = make_uint4(0, 0, 0, 0);
-                if (i < have16) v = __ldg(s4 + i);
-                v.x = bswap32(v.x);
-                v.y = bswap32(v.y);
-                v.z = bswap32(v.z);
-                v.w = bswap32(v.w);
-                d4[i] = v;
+        // 1. tables (when the tensor changes) and the stream slice
+        if (td != staged) {
+            const uint4* t4 = reinterpret_cast<const uint4*>(td->lut);
+            uint4* d4 = reinterpret_cast<uint4*>(smem);
+            for (uint32_t i = tid; i < kWideWords / 4; i += T) d4[i] = __ldg(t4 + i);
+            staged = td;
+        }
+        const uint32_t C = td->chunk_bytes;
+        const uint32_t wpc = C / 4 + 1;
+        uint32_t* my_words = s_words + tid * wpc;
+        const uint64_t chunk = b * T + tid;
+        uint32_t p = 0, end = 0;
+        if (chunk < td->n_chunks) {
+            const uint4* c4 = reinterpret_cast<const uint4*>(td->stream + chunk * C);
+            for (uint32_t k = 0; k < C / 16; ++k) {
+                const uint4 v = __ldg(c4 + k);
+                my_words[4 * k + 0] = bswap32(v.x);
+                my_words[4 * k + 1] = bswap32(v.y);
+                my_words[4 * k + 2] = bswap32(v.z);
+                my_words[4 * k + 3] = bswap32(v.w);
             }
+            my_words[C / 4] = bswap32(__ldg(reinterpret_cast<const uint32_t*>(td->stream + (chunk + 1) * C)));
+            const uint64_t q = 5 * chunk;
+            const uint32_t two = (static_cast<uint32_t>(__ldg(td->gaps + (q >> 3))) << 8) |
+                                 __ldg(td->gaps + (q >> 3) + 1);
+            const uint32_t cbits = 8 * C;
+            const uint64_t bit0 = chunk * cbits;
+            const uint64_t rem = td->total_bits > bit0 ? td->total_bits - bit0 : 0;
+            p = (two >> (11 - (q & 7))) & 31u;
+            end = static_cast<uint32_t>(rem < cbits ? rem : cbits);
         }
         const uint64_t out0 = td->offs[b];
         const uint64_t out1 = td->offs[b + 1];
         __syncthreads();
 
-        // this thread's chunk
-        const uint64_t chunk = b * T + tid;
-        const uint32_t cbits = 8 * C;
-        uint32_t p0 = 0, end = 0;
-        if (chunk < td->n_chunks) {
-            const uint64_t q = 5 * chunk;
-            const uint32_t two = (static_cast<uint32_t>(__ldg(td->gaps + (q >> 3))) << 8) |
-                                 __ldg(td->gaps + (q >> 3) + 1);
-            const uint32_t gap = (two >> (11 - (q & 7))) & 31u;
-            const uint64_t chunk_bit0 = chunk * cbits;
-            const uint64_t rem = td->total_bits > chunk_bit0 ? td->total_bits - chunk_bit0 : 0;
-            p0 = tid * cbits + gap;
-            end = tid * cbits + static_cast<uint32_t>(rem < cbits ? rem : cbits);
-        }
-
-        // 2. count pass
+        // 2. decode this thread's chunk into its region
+        uint32_t cnt = 0, nacc = 0, rw = 0;
+        uint64_t acc = 0;
         bool bad = false;
-        const uint32_t cnt = decode_chunk<false>(s_words, p0, end, s_lut, td->lut, stab, nullptr, 0, &bad);
+        const uint32_t rlim = region_words - 2;
+        for (;;) {  // whole windows before the chunk end
+            const bool act = p + kWideBits <= end && rw < rlim;
+            if (!__any_sync(0xFFFFFFFFu, act)) break;
+            if (act) {
+                const uint32_t win = window(my_words, p);
+                const uint32_t x = win >> (32 - kWideBits);
+                const uint32_t m = s_meta[x];
+                uint32_t sy = s_sym[x];
+                uint32_t used = m >> kWideBits, ns;
+                if (used == 0) {
+                    const uint32_t e = long_code(win, td->lut + kWideWords);
+                    ns = (e >> kNsymShift) & 3u;
+                    used = (e >> 8) & 63u;
+                    sy = e & 0xFFu;
+                    if (ns == 0) {
+                        bad = true;
+                        end = p;
+                    }
+                } else {
+                    ns = __popc(m & (kWideN - 1));
+                }
+                cnt += ns;
+                acc |= static_cast<uint64_t>(sy) << (8 * nacc);
+                nacc += ns;
+                if (nacc >= 4) {
+                    my_region[rw++] = static_cast<uint32_t>(acc);
+                    acc >>= 32;
+                    nacc -= 4;
+                }
+                p += used;
+            }
+        }
+        for (;;) {  // the last bits: count only the codes that start before the end
+            const bool act = p < end && rw < rlim;
+            if (!__any_sync(0xFFFFFFFFu, act)) break;
+            if (act) {
+                const uint32_t win = window(my_words, p);
+                const uint32_t x = win >> (32 - kWideBits);
+                const uint32_t m = s_meta[x];
+                uint32_t sy = s_sym[x];
+                uint32_t used = m >> kWideBits, ns, counted;
+                if (used == 0) {
+                    const uint32_t e = long_code(win, td->lut + kWideWords);
+                    ns = counted = (e >> kNsymShift) & 3u;
+                    used = (e >> 8) & 63u;
+                    sy = e & 0xFFu;
+                    if (ns == 0) {
+                        bad = true;
+                        end = p;
+                    }
+                } else {
+                    const uint32_t lim = end - p;  // < kWideBits here
+                    ns = __popc(m & (kWideN - 1));
+                    counted = __popc(m & ((1u << lim) - 1u));
+                }
+                cnt += counted;
+                acc |= static_cast<uint64_t>(sy) << (8 * nacc);
+                nacc += ns;
+                if (nacc >= 4) {
+                    my_region[rw++] = static_cast<uint32_t>(acc);
+                    acc >>= 32;
+                    nacc -= 4;
+                }
+                p += used;
+            }
+        }
+        if (p < end) bad = true;  // the region filled up: more codes than the layout allows
+        my_region[rw] = static_cast<uint32_t>(acc);
+        my_region[rw + 1] = static_cast<uint32_t>(acc >> 32);
 
-        // 3. block scan
-        const int lane = tid & 31, warp = tid >> 5;
+        // 3. block scan of the counts
         const uint32_t incl = warp_incl_scan(cnt, lane);
         if (lane == 31) s_warp[warp] = incl;
         __syncthreads();
-        const uint32_t nwarps = T >> 5;
         if (warp == 0) {
             uint32_t v = lane < static_cast<int>(nwarps) ? s_warp[lane] : 0;
             v = warp_incl_scan(v, lane);
             if (lane < static_cast<int>(nwarps)) s_warp[lane] = v;
         }
         __syncthreads();
-        const uint32_t excl = incl - cnt + (warp > 0 ? s_warp[warp - 1] : 0);
         const uint32_t total = s_warp[nwarps - 1];
-
-        // 4. consistency with the block index
         const uint32_t align = static_cast<uint32_t>(out0 & 15);
+        const uint32_t pos = align + incl - cnt + (warp > 0 ? s_warp[warp - 1] : 0);
+        s_pos[tid] = pos;
+        if (tid == T - 1) s_pos[T] = pos + cnt;
+
+        // consistency with the block index (uniform over the block)
         uint32_t flags = 0;
-        if (out1 < out0 || out1 > td->n || out1 - out0 + align > cfg.stage_bytes ||
+        if (out1 < out0 || out1 > td->n || (out1 - out0 + align + 15) / 16 > cfg.max_groups ||
             (b + 1 == td->n_blocks && out1 != td->n))
             flags |= DF_EFLAG_OFFSETS;
-        else if (static_cast<uint64_t>(total) != out1 - out0) flags |= DF_EFLAG_COUNT;
-        const bool any_bad = __syncthreads_or(bad) != 0;
-        if (any_bad) flags |= DF_EFLAG_BAD_CODE;
+        else if (static_cast<uint64_t>(total) != out1 - out0)
+            flags |= DF_EFLAG_COUNT;
+        if (__syncthreads_or(bad)) flags |= DF_EFLAG_BAD_CODE;
         if (flags) {
             if (tid == 0 && d_err) atomicOr(d_err, flags);
-            __syncthreads();  // s_warp and the stage are reused by the next block
+            __syncthreads();
             continue;
         }
 
-        // 5. write pass into the stage
-        decode_chunk<true>(s_words, p0, end, s_lut, td->lut, stab, s_stage, align + excl, &bad);
+        // 4. owner map: group gi (stage positions [16gi, 16gi+16)) belongs to
+        // the thread whose range holds max(16gi, align)
+        if (cnt) {
+            const uint32_t hi = pos + cnt;
+            if (pos <= align && align < hi) s_owner[0] = static_cast<uint16_t>(tid);
+            for (uint32_t gi = max((pos + 15) >> 4, 1u); 16 * gi < hi; ++gi) s_owner[gi] = static_cast<uint16_t>(tid);
+        }
         __syncthreads();
 
-        // 6. merge and store: 16 weights per group (one 16-byte load of
-        // sign|fraction bytes, one of staged exponents, two 16-byte stores);
-        // two groups per thread per step keep two loads in flight
+        // 5. merge and store
         const uint8_t* sm = td->sm;
         uint16_t* out = td->out;
-        const uint64_t gbase = out0 & ~15ull;  // stage index 0 <-> output gbase
-        const uint64_t ngroups = (out1 - gbase + 15) >> 4;
+        const uint64_t gbase = out0 & ~15ull;
+        const uint32_t ngroups = (align + total + 15) >> 4;
         const bool vec = td->vec_ok != 0;
-        for (uint64_t g0 = tid; g0 < ngroups; g0 += 2 * static_cast<uint64_t>(T)) {
-            uint4 s16[2];
-            bool full[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const uint64_t gi = g0 + static_cast<uint64_t>(u) * T;
-                const uint64_t G = gbase + 16 * gi;
-                full[u] = vec && gi < ngroups && G >= out0 && G + 16 <= out1;
-                if (full[u]) s16[u] = __ldg(reinterpret_cast<const uint4*>(sm + G));
-            }
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const uint64_t gi = g0 + static_cast<uint64_t>(u) * T;
-                if (gi >= ngroups) continue;
-                const uint64_t G = gbase + 16 * gi;
-                const uint32_t si = static_cast<uint32_t>(16 * gi);
-                if (full[u]) {
-                    const uint4 e16 = *reinterpret_cast<const uint4*>(s_stage + si);
-                    const uint32_t sw[4] = {s16[u].x, s16[u].y, s16[u].z, s16[u].w};
-                    const uint32_t ew[4] = {e16.x, e16.y, e16.z, e16.w};
-                    uint32_t o[8];
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const uint32_t hi = (sw[k] & 0x80808080u) | ((ew[k] >> 1) & 0x7F7F7F7Fu);
-                        const uint32_t lo = ((ew[k] << 7) & 0x80808080u) | (sw[k] & 0x7F7F7F7Fu);
-                        o[2 * k] = __byte_perm(lo, hi, 0x5140);
-                        o[2 * k + 1] = __byte_perm(lo, hi, 0x7362);
-                    }
-                    uint4* dst = reinterpret_cast<uint4*>(out + G);
-                    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-                    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
-                } else {
-                    for (uint32_t k = 0; k < 16; ++k) {
-                        const uint64_t i = G + k;
-                        if (i >= out0 && i < out1) out[i] = merge1(sm[i], s_stage[si + k]);
-                    }
+        for (uint32_t gi = tid; gi < ngroups; gi += T) {
+            const uint64_t G = gbase + 16ull * gi;
+            const uint32_t c0 = 16 * gi;
+            uint32_t t = s_owner[gi];
+            if (vec && G >= out0 && G + 16 <= out1 && c0 + 16 <= s_pos[t + 1]) {
+                const uint4 s16 = __ldg(reinterpret_cast<const uint4*>(sm + G));
+                const uint32_t a = t * cfg.region_bytes + (c0 - s_pos[t]);
+                const uint32_t* w = reinterpret_cast<const uint32_t*>(s_priv + (a & ~3u));
+                const uint32_t sh = 8 * (a & 3u);
+                const uint32_t w0 = w[0], w1 = w[1], w2 = w[2], w3 = w[3], w4 = w[4];
+                const uint32_t e0 = __funnelshift_r(w0, w1, sh), e1 = __funnelshift_r(w1, w2, sh);
+                const uint32_t e2 = __funnelshift_r(w2, w3, sh), e3 = __funnelshift_r(w3, w4, sh);
+                uint32_t o[8];
+                merge4(s16.x, e0, &o[0], &o[1]);
+                merge4(s16.y, e1, &o[2], &o[3]);
+                merge4(s16.z, e2, &o[4], &o[5]);
+                merge4(s16.w, e3, &o[6], &o[7]);
+                uint4* dst = reinterpret_cast<uint4*>(out + G);
+                dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+                dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+            } else {
+                for (uint32_t k = 0; k < 16; ++k) {
+                    const uint64_t i = G + k;
+                    if (i < out0 || i >= out1) continue;
+                    const uint32_t c = c0 + k;
+                    while (c >= s_pos[t + 1]) ++t;
+                    out[i] = merge1(sm[i], s_priv[t * cfg.region_bytes + (c - s_pos[t])]);
                 }
             }
         }
@@ -317,7 +331,7 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(Src src, LaunchCfg 
 
 struct Prepared {
     DevTensor dev;
-    uint32_t stage_need;
+    uint32_t words_per_chunk, region_bytes, max_groups;
 };
 
 uint32_t min_len_of(const uint8_t* lengths) {
@@ -329,7 +343,8 @@ uint32_t min_len_of(const uint8_t* lengths) {
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
-// Validate a descriptor and fill the device-side copy.
+// Validate a descriptor and fill the device-side copy and the shared-memory
+// needs of its blocks.
 df_status prepare(const df_tensor* t, uint16_t* out, Prepared* pr) {
     if (!t || !out) return DF_ERR_INVALID_ARG;
     const uint32_t C = t->chunk_bytes, T = t->threads_per_block;
@@ -360,19 +375,28 @@ df_status prepare(const df_tensor* t, uint16_t* out, Prepared* pr) {
     d.n_chunks = n_chunks;
     d.n_blocks = static_cast<uint32_t>(n_blocks);
     d.n_tables = t->n_tables;
+    d.chunk_bytes = C;
     d.vec_ok = aligned(t->sm, 16) && aligned(out, 16);
     pr->dev = d;
-    // a block holds at most 8CT/min_len codes, and never more than n
-    uint64_t need = minl ? (cbits * T + minl - 1) / minl : 0;
-    if (need > t->n) need = t->n;
-    need = (need + 16 + 15) & ~15ull;  // + alignment slack
-    if (need > (1u << 30)) return DF_ERR_UNSUPPORTED;
-    pr->stage_need = static_cast<uint32_t>(need);
+    pr->words_per_chunk = C / 4 + 1;  // odd: C is a multiple of 16
+    // a chunk holds at most 8C/min_len code starts; its region also takes up
+    // to 3 exponents past the last counted code and one partial word
+    const uint64_t per_chunk = (cbits + minl - 1) / (minl ? minl : 1);
+    uint64_t rb = (per_chunk + 8 + 3) & ~3ull;
+    if (((rb / 4) & 1) == 0) rb += 4;  // odd word stride: regions start in distinct banks
+    // a block holds at most 8CT/min_len codes and never more than n
+    uint64_t per_block = per_chunk * T;
+    if (per_block > t->n) per_block = t->n;
+    const uint64_t groups = (per_block + 15 + 15) / 16 + 1;
+    if (rb > (1u << 20) || groups > 0xFFFFu) return DF_ERR_UNSUPPORTED;
+    pr->region_bytes = static_cast<uint32_t>(rb);
+    pr->max_groups = static_cast<uint32_t>(groups);
     return DF_OK;
 }
 
-size_t smem_bytes(uint32_t tables, uint32_t C, uint32_t T, uint32_t stage) {
-    return static_cast<size_t>(tables) * 1024 + (static_cast<size_t>(T) * C / 4 + 4) * 4 + 32 * 4 + stage;
+size_t smem_bytes(const LaunchCfg& c, uint32_t T) {
+    return 6u * kWideN + static_cast<size_t>(T) * c.words_per_chunk * 4 + ((T + 1 + 3) & ~3u) * 4 + 32 * 4 +
+           ((c.max_groups * 2 + 15) & ~15u) + static_cast<size_t>(T) * c.region_bytes;
 }
 
 df_status device_limits(int* sms, int* max_smem) {
@@ -389,6 +413,7 @@ df_status device_limits(int* sms, int* max_smem) {
 template <class Src>
 df_status launch(const Src& src, const LaunchCfg& cfg, uint32_t T, size_t smem, uint32_t* d_err,
                  cudaStream_t stream) {
+    if (cfg.total_blocks == 0) return DF_OK;
     int sms = 0, max_smem = 0;
     df_status st = device_limits(&sms, &max_smem);
     if (st != DF_OK) return st;
@@ -396,12 +421,23 @@ df_status launch(const Src& src, const LaunchCfg& cfg, uint32_t T, size_t smem, 
     cudaError_t e = cudaFuncSetAttribute(decode_kernel<Src>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return cuda_fail(e);
-    const uint64_t grid = cfg.total_blocks < 0x7FFFFFFFull ? cfg.total_blocks : 0x7FFFFFFFull;
-    if (grid == 0) return DF_OK;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<Src>, static_cast<int>(T), smem);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (per_sm < 1) return DF_ERR_UNSUPPORTED;
+    // persistent blocks: every resident slot loops over the format blocks
+    const uint64_t slots = static_cast<uint64_t>(sms) * per_sm;
+    const uint64_t grid = cfg.total_blocks < slots ? cfg.total_blocks : slots;
     decode_kernel<Src><<<static_cast<unsigned>(grid), T, smem, stream>>>(src, cfg, d_err);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e);
     return DF_OK;
+}
+
+void widen(LaunchCfg* c, const Prepared& p) {
+    c->words_per_chunk = std::max(c->words_per_chunk, p.words_per_chunk);
+    c->region_bytes = std::max(c->region_bytes, p.region_bytes);
+    c->max_groups = std::max(c->max_groups, p.max_groups);
 }
 
 }  // namespace
@@ -419,12 +455,11 @@ df_status df_decode(const df_tensor* t, uint16_t* d_out, uint32_t* d_err, void* 
     if (st != DF_OK) return st;
     SingleSrc src{pr.dev};
     LaunchCfg cfg;
-    cfg.chunk_bytes = t->chunk_bytes;
-    cfg.smem_tables = std::min<uint32_t>(t->n_tables, kSmemTableCap);
-    cfg.stage_bytes = pr.stage_need;
+    std::memset(&cfg, 0, sizeof(cfg));
+    widen(&cfg, pr);
     cfg.total_blocks = pr.dev.n_blocks;
-    const size_t smem = smem_bytes(cfg.smem_tables, t->chunk_bytes, t->threads_per_block, cfg.stage_bytes);
-    return launch(src, cfg, t->threads_per_block, smem, d_err, static_cast<cudaStream_t>(stream));
+    return launch(src, cfg, t->threads_per_block, smem_bytes(cfg, t->threads_per_block), d_err,
+                  static_cast<cudaStream_t>(stream));
 }
 
 size_t df_decode_batch_workspace(uint32_t count) {
@@ -441,33 +476,32 @@ df_status df_decode_batch_prepare(const df_tensor* tensors, uint16_t* const* d_o
     std::vector<DevTensor> dev;
     std::vector<uint64_t> start(1, 0);
     dev.reserve(count);
-    uint32_t C = 0, T = 0, stage = 16, tables = 1;
+    uint32_t T = 0;
+    LaunchCfg cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
     for (uint32_t i = 0; i < count; ++i) {
         const df_tensor* t = tensors + i;
         if (t->n == 0) continue;
         Prepared pr;
         df_status st = prepare(t, d_outs[i], &pr);
         if (st != DF_OK) return st;
-        if (!C) {
-            C = t->chunk_bytes;
+        if (!T)
             T = t->threads_per_block;
-        } else if (C != t->chunk_bytes || T != t->threads_per_block) {
+        else if (T != t->threads_per_block)
             return DF_ERR_INVALID_ARG;
-        }
-        stage = std::max(stage, pr.stage_need);
-        tables = std::max(tables, std::min<uint32_t>(t->n_tables, kSmemTableCap));
+        widen(&cfg, pr);
         dev.push_back(pr.dev);
         start.push_back(start.back() + pr.dev.n_blocks);
     }
     plan->d_ws = d_ws;
     plan->count = static_cast<uint32_t>(dev.size());
     plan->threads_per_block = T;
-    plan->chunk_bytes = C;
-    plan->smem_tables = tables;
-    plan->stage_bytes = stage;
+    plan->words_per_chunk = cfg.words_per_chunk;
+    plan->region_bytes = cfg.region_bytes;
+    plan->max_groups = cfg.max_groups;
     plan->total_blocks = start.back();
     if (plan->count == 0) return DF_OK;
-    const size_t sm = smem_bytes(tables, C, T, stage);
+    const size_t sm = smem_bytes(cfg, T);
     int sms = 0, max_smem = 0;
     df_status st = device_limits(&sms, &max_smem);
     if (st != DF_OK) return st;
@@ -490,17 +524,16 @@ df_status df_decode_batch_run(const df_batch_plan* plan, uint32_t* d_err, void* 
     if (!plan) return DF_ERR_INVALID_ARG;
     if (plan->count == 0) return DF_OK;
     if (!plan->d_ws) return DF_ERR_INVALID_ARG;
-    // same layout as df_decode_batch_prepare writes
-    BatchSrc src;
+    BatchSrc src;  // same layout as df_decode_batch_prepare writes
     src.tensors = static_cast<const DevTensor*>(plan->d_ws);
     src.count = plan->count;
-    src.block_start = nullptr;
     const size_t table_bytes = (static_cast<size_t>(plan->count) * sizeof(DevTensor) + 255) / 256 * 256;
     src.block_start = reinterpret_cast<const uint64_t*>(static_cast<const uint8_t*>(plan->d_ws) + table_bytes);
     LaunchCfg cfg;
-    cfg.chunk_bytes = plan->chunk_bytes;
-    cfg.smem_tables = plan->smem_tables;
-    cfg.stage_bytes = plan->stage_bytes;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.words_per_chunk = plan->words_per_chunk;
+    cfg.region_bytes = plan->region_bytes;
+    cfg.max_groups = plan->max_groups;
     cfg.total_blocks = plan->total_blocks;
     return launch(src, cfg, plan->threads_per_block, plan->smem_bytes, d_err, static_cast<cudaStream_t>(stream));
 }

@@ -169,13 +169,16 @@ df_status df_build_code(const uint64_t hist[256], uint32_t max_len, df_code* out
     return df_code_from_lengths(lengths, max_len, out);
 }
 
-size_t df_lut_words(const df_code* code) { return code ? static_cast<size_t>(code->n_tables) * 256 + 64 : 0; }
+size_t df_lut_words(const df_code* code) {
+    return code ? kWideWords + static_cast<size_t>(code->n_tables) * 256 + 64 : 0;
+}
 
 df_status df_build_lut(const df_code* code, uint32_t* lut, size_t lut_words) {
     if (!code || !lut || code->n_tables < 1 || lut_words < df_lut_words(code)) return DF_ERR_INVALID_ARG;
     const size_t words = df_lut_words(code);
     std::memset(lut, 0, words * sizeof(uint32_t));
-    // single-code entries first
+
+    // 1. the 8-bit-indexed tables, one code per entry (the long-code path)
     std::vector<uint32_t> tables(static_cast<size_t>(code->n_tables) * 256, 0);
     uint32_t next_table = 1;
     for (int s = 0; s < 256; ++s) {
@@ -189,7 +192,8 @@ df_status df_build_lut(const df_code* code, uint32_t* lut, size_t lut_words) {
             uint32_t& e = tables[static_cast<size_t>(t) * 256 + idx];
             if (e == 0) {
                 if (next_table >= code->n_tables) return DF_ERR_INVALID_ARG;
-                e = next_table++;  // count 0: a link to the next level
+                e = next_table;  // count 0: a link to the next level
+                ++next_table;
             } else if ((e >> kNsymShift) & 3u) {
                 return DF_ERR_INVALID_ARG;  // a shorter code is a prefix of this one
             }
@@ -201,37 +205,39 @@ df_status df_build_lut(const df_code* code, uint32_t* lut, size_t lut_words) {
         for (uint32_t x = lo; x < hi; ++x) {
             uint32_t& e = tables[static_cast<size_t>(t) * 256 + x];
             if (e != 0) return DF_ERR_INVALID_ARG;
-            e = lut_leaf(static_cast<uint32_t>(s), 1, l);
+            e = sub_leaf(static_cast<uint32_t>(s), l);
         }
     }
-    // root entries: pack up to three whole codes inside the 8 indexed bits
-    for (uint32_t x = 0; x < 256; ++x) {
-        const uint32_t e0 = tables[x];
-        uint32_t nsym = (e0 >> kNsymShift) & 3u;
-        if (!nsym) {
-            lut[x] = e0;  // a link (count 0, table index) or an unreachable 0
-            continue;
-        }
-        const uint32_t len0 = e0 >> kNbitsShift;
-        uint32_t used = len0;
-        uint32_t syms = e0 & 0xFFu;
-        while (nsym < 3 && used < 8) {
-            const uint32_t y = (x << used) & 0xFFu;  // the unknown low bits read as 0
-            const uint32_t e = tables[y];
-            const uint32_t l = e >> kNbitsShift;
-            if (!((e >> kNsymShift) & 3u) || l > 8 - used) break;  // this code needs bits beyond x
-            syms |= (e & 0xFFu) << (8 * nsym);
+    uint32_t* hier = lut + kWideWords;
+    std::memcpy(hier, tables.data(), tables.size() * sizeof(uint32_t));
+    std::memcpy(lut + kWideWords + static_cast<size_t>(code->n_tables) * 256, code->lengths, 256);
+
+    // 2. the wide table: for every kWideBits-bit window, the codes that lie
+    // wholly inside it from its first bit on (at most kWideMaxCodes)
+    const uint32_t W = kWideBits, N = 1u << W;
+    std::vector<uint32_t> first(N, 0);  // (len << 8) | symbol of the code at bit 0, if len <= W
+    for (int s = 0; s < 256; ++s) {
+        const uint32_t l = code->lengths[s];
+        if (!l || l > W) continue;
+        const uint32_t c = code->codes[s];
+        for (uint32_t x = c << (W - l); x < ((c + 1) << (W - l)); ++x) first[x] = (l << 8) | static_cast<uint32_t>(s);
+    }
+    uint16_t* meta = reinterpret_cast<uint16_t*>(lut);
+    uint32_t* sym = lut + kWideMetaWords;
+    for (uint32_t x = 0; x < N; ++x) {
+        uint32_t used = 0, n = 0, mask = 0, syms = 0;
+        while (n < kWideMaxCodes && used < W) {
+            const uint32_t e = first[(x << used) & (N - 1)];  // the unknown low bits read as 0
+            const uint32_t l = e >> 8;
+            if (!l || l > W - used) break;  // this code needs bits beyond the window
+            mask |= 1u << used;
+            syms |= (e & 0xFFu) << (8 * n);
             used += l;
-            ++nsym;
+            ++n;
         }
-        lut[x] = root_entry(syms, nsym, used, len0);
+        meta[x] = static_cast<uint16_t>(mask | (used << kWideBits));
+        sym[x] = syms;
     }
-    // next-level entries: one code each, with its full length
-    for (size_t i = 256; i < tables.size(); ++i) {
-        const uint32_t e = tables[i];
-        lut[i] = ((e >> kNsymShift) & 3u) ? sub_leaf(e & 0xFFu, e >> kNbitsShift) : e;
-    }
-    std::memcpy(lut + static_cast<size_t>(code->n_tables) * 256, code->lengths, 256);
     return DF_OK;
 }
 

@@ -21,27 +21,28 @@ struct DevTensor {
     uint64_t n_chunks;
     uint32_t n_blocks;
     uint32_t n_tables;
-    uint32_t vec_ok;       // sm 8-byte and out 16-byte aligned
-    uint32_t pad;
+    uint32_t chunk_bytes;
+    uint32_t vec_ok;       // sm and out 16-byte aligned
 };
 
-// Decode-table entries (uint32).
-//   root table, leaf:  bits 0-23 up to three exponents (first in bits 0-7),
-//                      24-25 how many (1..3), 26-28 bits they use - 1,
-//                      29-31 length of the first code - 1
-//   next-level leaf:   bits 0-7 the exponent, 8-13 its full code length,
-//                      24-25 = 1
-//   link (any table):  bits 0-15 index of the next-level table (>= 1), 24-25 = 0
-//   unreachable:       0
+// Decode tables (the words df_build_lut writes), in order:
+//   wide table, kWideBits = 11 bits of window per entry:
+//     meta[2048] uint16: bit i (i < 11) set if a code starts at window bit i
+//                        and lies wholly inside the window (at most 4 codes,
+//                        taken from bit 0 on); bits 11-14: the bits those
+//                        codes use (0: the first code is longer than 11 bits)
+//     sym[2048]  uint32: their exponents, first in bits 0-7
+//   8-bit-indexed tables for codes of any length (root + next levels):
+//     leaf:  bits 0-7 the exponent, 8-13 its full code length, 24-25 = 1
+//     link:  bits 0-15 index of the next-level table (>= 1), 24-25 = 0
+//     unreachable: 0
+//   code lengths: 256 bytes
+constexpr uint32_t kWideBits = 11;
+constexpr uint32_t kWideMaxCodes = 4;
+constexpr uint32_t kWideMetaWords = (1u << kWideBits) / 2;
+constexpr uint32_t kWideWords = kWideMetaWords + (1u << kWideBits);
 constexpr uint32_t kNsymShift = 24;
-constexpr uint32_t kNbitsShift = 26;  // build-time single-code form: full length in bits 26-31
 
-inline __host__ __device__ uint32_t lut_leaf(uint32_t syms, uint32_t nsym, uint32_t nbits) {
-    return syms | (nsym << kNsymShift) | (nbits << kNbitsShift);
-}
-inline __host__ __device__ uint32_t root_entry(uint32_t syms, uint32_t nsym, uint32_t used, uint32_t len0) {
-    return syms | (nsym << 24) | ((used - 1) << 26) | ((len0 - 1) << 29);
-}
 inline __host__ __device__ uint32_t sub_leaf(uint32_t sym, uint32_t len) { return sym | (len << 8) | (1u << 24); }
 
 // Records the CUDA error for df_last_cuda_error and maps it to DF_ERR_CUDA.

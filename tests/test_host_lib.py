@@ -115,12 +115,18 @@ def test_plan_matches_oracle_sizes(chunk_bytes, tpb):
 # ---------------------------------------------------------------- the decode tables
 
 
+WIDE = 11  # window bits of the wide table
+
+
 def table_walk_decode(stream, total_bits, n, gaps_fields, offsets, lut, n_tables, chunk_bytes, tpb):
-    """Plain-Python model of the kernel's per-chunk table walk: every chunk is
-    decoded from its start + gap up to its end, codes taken from the root
-    entry (up to three per step while 8 bits remain before the end, else only
-    the first) or from the next-level tables; counts are checked against the
-    block offsets."""
+    """Plain-Python model of the kernel's per-chunk decode: every chunk is
+    decoded from its start + gap up to its end; a wide-table step yields the
+    codes that lie wholly inside the next 11 bits (only those starting before
+    the chunk end are counted), a code longer than 11 bits walks the 8-bit
+    tables; counts are checked against the block offsets."""
+    meta = np.frombuffer(lut[: (1 << WIDE) // 2].tobytes(), np.uint16)
+    sym = lut[(1 << WIDE) // 2: (1 << WIDE) // 2 + (1 << WIDE)]
+    hier = lut[(1 << WIDE) // 2 + (1 << WIDE):]
     bits = np.unpackbits(np.asarray(stream, np.uint8))
     cb = 8 * chunk_bytes
     n_chunks = len(gaps_fields)
@@ -140,28 +146,29 @@ def table_walk_decode(stream, total_bits, n, gaps_fields, offsets, lut, n_tables
         cnt = 0
         while p < end:
             win = window(p)
-            e = int(lut[win >> 24])
-            ns = (e >> 24) & 3
-            if ns == 0:
+            m = int(meta[win >> (32 - WIDE)])
+            used = m >> WIDE
+            if used == 0:
+                e = int(hier[win >> 24])
                 for lvl in (1, 2, 3):
-                    t = e & 0xFFFF
-                    assert t != 0, "unreachable entry"
-                    e = int(lut[t * 256 + ((win >> (24 - 8 * lvl)) & 0xFF)])
                     if (e >> 24) & 3:
                         break
+                    t = e & 0xFFFF
+                    assert t != 0, "unreachable entry"
+                    e = int(hier[t * 256 + ((win >> (24 - 8 * lvl)) & 0xFF)])
                 assert (e >> 24) & 3 == 1
                 out.append(e & 0xFF)
                 cnt += 1
                 p += (e >> 8) & 63
-            elif p + 8 <= end:
-                for k in range(ns):
-                    out.append((e >> (8 * k)) & 0xFF)
-                cnt += ns
-                p += ((e >> 26) & 7) + 1
-            else:
-                out.append(e & 0xFF)
-                cnt += 1
-                p += (e >> 29) + 1
+                continue
+            mask = m & ((1 << WIDE) - 1)
+            lim = min(end - p, WIDE)
+            starts = [i for i in range(WIDE) if (mask >> i) & 1 and i < lim]
+            sy = int(sym[win >> (32 - WIDE)])
+            for k in range(len(starts)):
+                out.append((sy >> (8 * k)) & 0xFF)
+            cnt += len(starts)
+            p += used
         counts.append(cnt)
     counts = np.array(counts)
     per_block = [int(counts[b * tpb:(b + 1) * tpb].sum()) for b in range(len(offsets) - 1)]
@@ -201,8 +208,15 @@ def test_unreachable_entries_are_zero():
     h[127] = 10  # one symbol: code '0', so every index starting with bit 1 is unreachable
     code = api.df_build_code(h)
     lut = api.df_build_lut(code)
-    assert (lut[128:256] == 0).all() and (lut[:128] != 0).all()
-    # a complete code reaches every root entry
-    code = api.df_build_code(np.arange(1, 257, dtype=np.uint64))
+    meta = np.frombuffer(lut[: (1 << WIDE) // 2].tobytes(), np.uint16)
+    half = 1 << (WIDE - 1)
+    assert (meta[half:] == 0).all() and (meta[:half] != 0).all()
+    hier = lut[(1 << WIDE) // 2 + (1 << WIDE):]
+    assert (hier[128:256] == 0).all() and (hier[:128] != 0).all()
+    # 256 equally frequent exponents: every code has 8 bits, every entry is reached
+    code = api.df_build_code(np.full(256, 7, dtype=np.uint64))
     lut = api.df_build_lut(code)
-    assert (lut[:256] != 0).all()
+    meta = np.frombuffer(lut[: (1 << WIDE) // 2].tobytes(), np.uint16)
+    assert ((meta >> WIDE) == 8).all()
+    hier = lut[(1 << WIDE) // 2 + (1 << WIDE):]
+    assert (hier[:256] != 0).all()
