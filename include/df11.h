@@ -143,21 +143,26 @@ df_status df_build_code(const uint64_t hist[256], uint32_t max_len, df_code* out
  * sum 2^-l <= 1); DF_ERR_UNSUPPORTED (max_len outside 1..32). */
 df_status df_code_from_lengths(const uint8_t lengths[256], uint32_t max_len, df_code* out);
 
-/* Number of uint32 words df_build_lut writes: 256 per table plus 64 words
- * holding the 256 code-length bytes. 0 for a NULL code. */
+/* Number of uint32 words df_build_lut writes: 1536 for the wide table, 256
+ * per 8-bit-indexed table and 64 for the code lengths. 0 for a NULL code. */
 size_t df_lut_words(const df_code* code);
 
 /* df_build_lut: derive the decode tables of a code into host memory `lut`
- * (lut_words >= df_lut_words(code)). Table 0 is indexed by the next 8 stream
- * bits; an entry holds up to three whole codes that fit in those 8 bits
- * (exponents in bits 0-23, their count in bits 24-25, the bits they use minus
- * one in bits 26-28, the first code's length minus one in bits 29-31), or,
- * for a longer code, count 0 and the index of a next-level table (bits 0-15)
- * indexed by the following 8 bits, at most four levels for 32-bit codes. A
- * next-level leaf holds one exponent (bits 0-7), its full code length (bits
- * 8-13) and count 1. Entries no code reaches are zero. The caller copies the words to the
- * device and passes them as df_tensor.lut. Source: df11pack, "What is
- * checked" (--luts=correct zero-fills unreachable table entries).
+ * (lut_words >= df_lut_words(code)); the caller copies the words to the
+ * device and passes them as df_tensor.lut. Layout, in order:
+ *   - the wide table, indexed by the next 10 stream bits: 1024 uint16 (bit i
+ *     set when a code starts at window bit i and lies wholly inside the
+ *     window, up to 4 codes from bit 0 on; bits 10-13 the bits they use, 0
+ *     when the first code is longer than 10 bits) then 1024 uint32 (their
+ *     exponents, the first in bits 0-7);
+ *   - n_tables tables of 256 uint32 indexed by 8 stream bits, for codes of
+ *     any length: a leaf holds the exponent (bits 0-7), the full code length
+ *     (bits 8-13) and a 1 in bits 24-25; a link holds the index of the
+ *     next-level table (bits 0-15, >= 1) and 0 in bits 24-25; table 0 is the
+ *     root, at most four levels for 32-bit codes;
+ *   - the 256 code lengths as bytes.
+ * Entries no code reaches are zero. Source: df11pack, "What is checked"
+ * (--luts=correct zero-fills unreachable table entries).
  * Errors: DF_ERR_INVALID_ARG (null, too small, or a code that is not prefix free).
  */
 df_status df_build_lut(const df_code* code, uint32_t* lut, size_t lut_words);
@@ -198,12 +203,12 @@ df_status df_encode(const df_code* code, const uint16_t* d_in, uint64_t n, uint6
 
 /* ---- decode (device) ---------------------------------------------------------
  * df_decode: d_out[0..t->n) = the original BF16 bit patterns (uint16, device;
- * 16-byte alignment takes the vector store path). One CUDA block per T
- * chunks: the decode tables and the block's stream slice are staged in shared
- * memory, each thread counts the codes that start in its chunk, a block scan
- * turns the counts into output positions, a second pass writes the exponents
- * to a shared-memory stage, and the block merges them with the sign|fraction
- * bytes into 16-byte stores. Source: mlx-dfloat, intro and "Status" (blockwise
+ * 16-byte alignment of d_out and t->sm takes the vector path). A CUDA block
+ * decodes T chunks at a time: the wide table and the block's stream slice
+ * are staged in shared memory, each thread decodes the codes that start in
+ * its chunk into its own shared-memory region and counts them, a block scan
+ * turns the counts into output positions, and the block merges the staged
+ * exponents with the sign|fraction bytes into 16-byte stores. Source: mlx-dfloat, intro and "Status" (blockwise
  * GPU decode back to identical bits); df11pack, "Use" (chunks).
  * Data errors set DF_EFLAG_* in d_err (nullable) and skip the affected
  * block's stores. Errors: DF_ERR_INVALID_ARG, DF_ERR_UNSUPPORTED (a layout

@@ -7,15 +7,15 @@
 //
 // One CUDA block handles one format block (T chunks of C stream bytes) at a
 // time and loops over the blocks of all tensors of the launch:
-//   1. when the tensor changes, stage its 11-bit multi-code table (codes that
-//      lie wholly inside an 11-bit window: start mask, bits used, exponents)
+//   1. when the tensor changes, stage its wide multi-code table (codes that
+//      lie wholly inside a 10-bit window: start mask, bits used, exponents)
 //      in shared memory; stage the block's stream slice, one chunk per thread,
 //      byte-swapped to big-endian words at an odd word stride (no bank
 //      conflicts between the threads' windows)
 //   2. one decode pass per thread over its chunk, from chunk start + gap to
 //      the chunk end: each table step yields up to 4 codes; their exponents
 //      go to the thread's own word-aligned shared-memory region with 32-bit
-//      stores; codes longer than 11 bits walk the 8-bit-indexed tables
+//      stores; codes longer than 10 bits walk the 8-bit-indexed tables
 //   3. block scan of the code counts (warp shuffles + one shared array): the
 //      first output position of every thread; checked against the block index
 //   4. an owner map: for every group of 16 outputs, the thread whose region
@@ -105,6 +105,17 @@ __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v, int lane) {
 __device__ __forceinline__ uint16_t merge1(uint8_t sm, uint8_t e) {
     return static_cast<uint16_t>((static_cast<uint32_t>(sm & 0x80u) << 8) | (static_cast<uint32_t>(e) << 7) |
                                  (sm & 0x7Fu));
+}
+
+// 16 bytes of shared memory from byte address a (any alignment), as 4 words.
+__device__ __forceinline__ void gather16(const uint8_t* base, uint32_t a, uint32_t e[4]) {
+    const uint32_t* w = reinterpret_cast<const uint32_t*>(base + (a & ~3u));
+    const uint32_t sh = 8 * (a & 3u);
+    const uint32_t w0 = w[0], w1 = w[1], w2 = w[2], w3 = w[3], w4 = w[4];
+    e[0] = __funnelshift_r(w0, w1, sh);
+    e[1] = __funnelshift_r(w1, w2, sh);
+    e[2] = __funnelshift_r(w2, w3, sh);
+    e[3] = __funnelshift_r(w3, w4, sh);
 }
 
 // 4 BF16 weights from 4 sign|fraction bytes and 4 exponent bytes: the high
@@ -289,29 +300,46 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_consta
         }
         __syncthreads();
 
-        // 5. merge and store
+        // 5. merge and store: a group of 16 outputs takes its exponents from the
+        // owner's region and, when it runs past the owner's last code, from
+        // the next thread's region (read from k bytes before its start, so the
+        // two 16-byte reads line up; a byte mask picks the first k from the
+        // owner); a group over three or more regions, or at the ends of the
+        // block, goes one weight at a time
         const uint8_t* sm = td->sm;
         uint16_t* out = td->out;
         const uint64_t gbase = out0 & ~15ull;
         const uint32_t ngroups = (align + total + 15) >> 4;
         const bool vec = td->vec_ok != 0;
+        const uint32_t RB = cfg.region_bytes;
         for (uint32_t gi = tid; gi < ngroups; gi += T) {
             const uint64_t G = gbase + 16ull * gi;
             const uint32_t c0 = 16 * gi;
             uint32_t t = s_owner[gi];
-            if (vec && G >= out0 && G + 16 <= out1 && c0 + 16 <= s_pos[t + 1]) {
+            const uint32_t b1 = s_pos[t + 1];
+            bool fast = vec && G >= out0 && G + 16 <= out1;
+            const bool spill = c0 + 16 > b1;  // continues in region t+1
+            if (spill) fast = fast && t + 1 < T && c0 + 16 <= s_pos[t + 2];
+            if (fast) {
                 const uint4 s16 = __ldg(reinterpret_cast<const uint4*>(sm + G));
-                const uint32_t a = t * cfg.region_bytes + (c0 - s_pos[t]);
-                const uint32_t* w = reinterpret_cast<const uint32_t*>(s_priv + (a & ~3u));
-                const uint32_t sh = 8 * (a & 3u);
-                const uint32_t w0 = w[0], w1 = w[1], w2 = w[2], w3 = w[3], w4 = w[4];
-                const uint32_t e0 = __funnelshift_r(w0, w1, sh), e1 = __funnelshift_r(w1, w2, sh);
-                const uint32_t e2 = __funnelshift_r(w2, w3, sh), e3 = __funnelshift_r(w3, w4, sh);
+                uint32_t e[4];
+                gather16(s_priv, t * RB + (c0 - s_pos[t]), e);
+                if (spill) {
+                    const uint32_t k = b1 - c0;  // 1..15 exponents from region t
+                    uint32_t y[4];
+                    gather16(s_priv, (t + 1) * RB - k, y);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int sbits = 8 * static_cast<int>(k) - 32 * i;
+                        const uint32_t m = sbits >= 32 ? 0xFFFFFFFFu : (sbits <= 0 ? 0u : (1u << sbits) - 1u);
+                        e[i] = (e[i] & m) | (y[i] & ~m);
+                    }
+                }
                 uint32_t o[8];
-                merge4(s16.x, e0, &o[0], &o[1]);
-                merge4(s16.y, e1, &o[2], &o[3]);
-                merge4(s16.z, e2, &o[4], &o[5]);
-                merge4(s16.w, e3, &o[6], &o[7]);
+                merge4(s16.x, e[0], &o[0], &o[1]);
+                merge4(s16.y, e[1], &o[2], &o[3]);
+                merge4(s16.z, e[2], &o[4], &o[5]);
+                merge4(s16.w, e[3], &o[6], &o[7]);
                 uint4* dst = reinterpret_cast<uint4*>(out + G);
                 dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
                 dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
@@ -321,7 +349,7 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_consta
                     if (i < out0 || i >= out1) continue;
                     const uint32_t c = c0 + k;
                     while (c >= s_pos[t + 1]) ++t;
-                    out[i] = merge1(sm[i], s_priv[t * cfg.region_bytes + (c - s_pos[t])]);
+                    out[i] = merge1(sm[i], s_priv[t * RB + (c - s_pos[t])]);
                 }
             }
         }

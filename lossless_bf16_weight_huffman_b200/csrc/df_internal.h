@@ -26,18 +26,18 @@ struct DevTensor {
 };
 
 // Decode tables (the words df_build_lut writes), in order:
-//   wide table, kWideBits = 11 bits of window per entry:
-//     meta[2048] uint16: bit i (i < 11) set if a code starts at window bit i
+//   wide table, kWideBits = 10 bits of window per entry:
+//     meta[1024] uint16: bit i (i < 10) set if a code starts at window bit i
 //                        and lies wholly inside the window (at most 4 codes,
-//                        taken from bit 0 on); bits 11-14: the bits those
-//                        codes use (0: the first code is longer than 11 bits)
-//     sym[2048]  uint32: their exponents, first in bits 0-7
+//                        taken from bit 0 on); bits 10-13: the bits those
+//                        codes use (0: the first code is longer than 10 bits)
+//     sym[1024]  uint32: their exponents, first in bits 0-7
 //   8-bit-indexed tables for codes of any length (root + next levels):
 //     leaf:  bits 0-7 the exponent, 8-13 its full code length, 24-25 = 1
 //     link:  bits 0-15 index of the next-level table (>= 1), 24-25 = 0
 //     unreachable: 0
 //   code lengths: 256 bytes
-constexpr uint32_t kWideBits = 11;
+constexpr uint32_t kWideBits = 10;
 constexpr uint32_t kWideMaxCodes = 4;
 constexpr uint32_t kWideMetaWords = (1u << kWideBits) / 2;
 constexpr uint32_t kWideWords = kWideMetaWords + (1u << kWideBits);

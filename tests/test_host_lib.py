@@ -115,15 +115,21 @@ def test_plan_matches_oracle_sizes(chunk_bytes, tpb):
 # ---------------------------------------------------------------- the decode tables
 
 
-WIDE = 11  # window bits of the wide table
+def wide_bits(lut, n_tables):
+    """The wide table's window width, from the table sizes (1.5 * 2^W words)."""
+    words = lut.size - 256 * n_tables - 64
+    W = int(round(np.log2(words / 1.5)))
+    assert 3 * (1 << W) // 2 == words
+    return W
 
 
 def table_walk_decode(stream, total_bits, n, gaps_fields, offsets, lut, n_tables, chunk_bytes, tpb):
     """Plain-Python model of the kernel's per-chunk decode: every chunk is
     decoded from its start + gap up to its end; a wide-table step yields the
-    codes that lie wholly inside the next 11 bits (only those starting before
-    the chunk end are counted), a code longer than 11 bits walks the 8-bit
-    tables; counts are checked against the block offsets."""
+    codes that lie wholly inside the next W bits (only those starting before
+    the chunk end are counted), a longer code walks the 8-bit tables; counts
+    are checked against the block offsets."""
+    WIDE = wide_bits(lut, n_tables)
     meta = np.frombuffer(lut[: (1 << WIDE) // 2].tobytes(), np.uint16)
     sym = lut[(1 << WIDE) // 2: (1 << WIDE) // 2 + (1 << WIDE)]
     hier = lut[(1 << WIDE) // 2 + (1 << WIDE):]
@@ -208,6 +214,7 @@ def test_unreachable_entries_are_zero():
     h[127] = 10  # one symbol: code '0', so every index starting with bit 1 is unreachable
     code = api.df_build_code(h)
     lut = api.df_build_lut(code)
+    WIDE = wide_bits(lut, code.n_tables)
     meta = np.frombuffer(lut[: (1 << WIDE) // 2].tobytes(), np.uint16)
     half = 1 << (WIDE - 1)
     assert (meta[half:] == 0).all() and (meta[:half] != 0).all()
