@@ -63,6 +63,7 @@ typedef int df_status;
 #define DF_EFLAG_BAD_CODE 1u      /* decode: a bit pattern no code starts with        */
 #define DF_EFLAG_COUNT 2u         /* decode: codes in a block != its offset difference */
 #define DF_EFLAG_OFFSETS 4u       /* decode: block offsets out of range               */
+#define DF_EFLAG_TABLES 8u        /* decode: tables not built for this descriptor      */
 #define DF_EFLAG_ENC_TOTAL 16u    /* encode: stream length != the planned total_bits   */
 #define DF_EFLAG_ENC_SYMBOL 32u   /* encode: an exponent without a code                */
 
@@ -143,24 +144,27 @@ df_status df_build_code(const uint64_t hist[256], uint32_t max_len, df_code* out
  * sum 2^-l <= 1); DF_ERR_UNSUPPORTED (max_len outside 1..32). */
 df_status df_code_from_lengths(const uint8_t lengths[256], uint32_t max_len, df_code* out);
 
-/* Number of uint32 words df_build_lut writes: 1536 for the wide table, 256
- * per 8-bit-indexed table and 64 for the code lengths. 0 for a NULL code. */
+/* Number of uint32 words df_build_lut writes: 2048 for the wide table, 256
+ * per 8-bit-indexed table, 64 for the code lengths and a 4-word header.
+ * 0 for a NULL code. */
 size_t df_lut_words(const df_code* code);
 
 /* df_build_lut: derive the decode tables of a code into host memory `lut`
  * (lut_words >= df_lut_words(code)); the caller copies the words to the
  * device and passes them as df_tensor.lut. Layout, in order:
- *   - the wide table, indexed by the next 10 stream bits: 1024 uint16 (bit i
- *     set when a code starts at window bit i and lies wholly inside the
- *     window, up to 4 codes from bit 0 on; bits 10-13 the bits they use, 0
- *     when the first code is longer than 10 bits) then 1024 uint32 (their
- *     exponents, the first in bits 0-7);
+ *   - the wide table: 1024 uint64 indexed by the next 10 stream bits; an
+ *     entry holds the exponents of the codes that lie wholly inside the
+ *     window from its first bit on (up to 4, bits 0-31, the first in bits
+ *     0-7), a mask of the window bits where they start (bits 32-41), the bits
+ *     they use (bits 42-45; 0 when the first code is longer than 10 bits) and
+ *     their count (bits 46-48);
  *   - n_tables tables of 256 uint32 indexed by 8 stream bits, for codes of
  *     any length: a leaf holds the exponent (bits 0-7), the full code length
  *     (bits 8-13) and a 1 in bits 24-25; a link holds the index of the
  *     next-level table (bits 0-15, >= 1) and 0 in bits 24-25; table 0 is the
  *     root, at most four levels for 32-bit codes;
- *   - the 256 code lengths as bytes.
+ *   - the 256 code lengths as bytes;
+ *   - a header: the shortest code length, max_len, n_tables, 0xDF11DF11.
  * Entries no code reaches are zero. Source: df11pack, "What is checked"
  * (--luts=correct zero-fills unreachable table entries).
  * Errors: DF_ERR_INVALID_ARG (null, too small, or a code that is not prefix free).

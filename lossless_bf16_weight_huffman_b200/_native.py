@@ -21,6 +21,7 @@ DF_ERR_WORKSPACE = 5
 DF_EFLAG_BAD_CODE = 1
 DF_EFLAG_COUNT = 2
 DF_EFLAG_OFFSETS = 4
+DF_EFLAG_TABLES = 8
 DF_EFLAG_ENC_TOTAL = 16
 DF_EFLAG_ENC_SYMBOL = 32
 

@@ -38,8 +38,10 @@ constexpr uint32_t kWideN = 1u << kWideBits;
 
 struct SingleSrc {
     DevTensor t;
-    __device__ __forceinline__ const DevTensor* lookup(uint64_t g, uint64_t* local) const {
-        *local = g;
+    // the tensor holding global block g, and its block range [lo, hi)
+    __device__ __forceinline__ const DevTensor* find(uint64_t g, uint64_t* lo, uint64_t* hi) const {
+        *lo = 0;
+        *hi = t.n_blocks;
         return &t;
     }
 };
@@ -48,17 +50,18 @@ struct BatchSrc {
     const DevTensor* tensors;
     const uint64_t* block_start;  // count+1 prefix sums of n_blocks
     uint32_t count;
-    __device__ __forceinline__ const DevTensor* lookup(uint64_t g, uint64_t* local) const {
-        uint32_t lo = 0, hi = count;  // block_start[lo] <= g < block_start[hi]
-        while (hi - lo > 1) {
-            const uint32_t mid = (lo + hi) >> 1;
+    __device__ __forceinline__ const DevTensor* find(uint64_t g, uint64_t* lo, uint64_t* hi) const {
+        uint32_t a = 0, z = count;  // block_start[a] <= g < block_start[z]
+        while (z - a > 1) {
+            const uint32_t mid = (a + z) >> 1;
             if (block_start[mid] <= g)
-                lo = mid;
+                a = mid;
             else
-                hi = mid;
+                z = mid;
         }
-        *local = g - block_start[lo];
-        return tensors + lo;
+        *lo = block_start[a];
+        *hi = block_start[a + 1];
+        return tensors + a;
     }
 };
 
@@ -127,7 +130,55 @@ __device__ __forceinline__ void merge4(uint32_t s, uint32_t e, uint32_t* o0, uin
     *o1 = __byte_perm(lo, hi, 0x7362);
 }
 
-template <class Src>
+// Decoder state of one thread over its chunk.
+struct DecState {
+    uint32_t p;    // bit position in the chunk
+    uint32_t end;  // codes must start before this bit
+    uint32_t cnt;  // codes counted
+    uint32_t app;  // exponents appended to the region (cnt, plus up to 3 past the end)
+    uint64_t acc;  // exponents not yet stored, app & 3 of them
+    bool bad;
+};
+
+// One wide-table step. kTail: the window may reach past the chunk end, so
+// only the codes that start before it are counted.
+template <bool kTail>
+__device__ __forceinline__ void decode_step(DecState& st, const uint32_t* words, const uint64_t* wide,
+                                            const uint32_t* hier, uint32_t* region) {
+    const uint32_t win = window(words, st.p);
+    const uint64_t e = wide[win >> (32 - kWideBits)];
+    uint32_t used = static_cast<uint32_t>(e >> kWideUsedShift) & 15u;
+    uint32_t sy, ns, counted;
+    if (used == 0) {  // a code longer than the window (or corrupt data)
+        const uint32_t l = long_code(win, hier);
+        ns = counted = (l >> kNsymShift) & 3u;
+        used = (l >> 8) & 63u;
+        sy = l & 0xFFu;
+        if (ns == 0) {
+            st.bad = true;
+            st.end = st.p;
+        }
+    } else {
+        sy = static_cast<uint32_t>(e);
+        ns = static_cast<uint32_t>(e >> kWideCountShift) & 7u;
+        counted = ns;
+        if (kTail) {
+            const uint32_t mask = static_cast<uint32_t>(e >> kWideMaskShift) & ((1u << kWideBits) - 1u);
+            counted = __popc(mask & ((1u << (st.end - st.p)) - 1u));
+        }
+    }
+    st.acc |= static_cast<uint64_t>(sy) << (8 * (st.app & 3u));
+    const uint32_t na = st.app + ns;
+    if ((na ^ st.app) & ~3u) {
+        region[st.app >> 2] = static_cast<uint32_t>(st.acc);
+        st.acc >>= 32;
+    }
+    st.app = na;
+    st.cnt += counted;
+    st.p += used;
+}
+
+template <class Src, class OwnerT>
 __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_constant__ Src src, const LaunchCfg cfg,
                                                              uint32_t* d_err) {
     extern __shared__ __align__(16) uint8_t smem[];
@@ -137,32 +188,58 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_consta
     const uint32_t nwarps = T >> 5;
 
     // shared memory carve-up (sizes in smem_bytes())
-    uint16_t* s_meta = reinterpret_cast<uint16_t*>(smem);
-    uint32_t* s_sym = reinterpret_cast<uint32_t*>(smem + 2 * kWideN);
-    uint32_t* s_words = s_sym + kWideN;
+    uint64_t* s_wide = reinterpret_cast<uint64_t*>(smem);
+    uint32_t* s_words = reinterpret_cast<uint32_t*>(smem + 8 * kWideN);
     uint32_t* s_pos = s_words + T * cfg.words_per_chunk;
     uint32_t* s_warp = s_pos + ((T + 1 + 3) & ~3u);
-    uint16_t* s_owner = reinterpret_cast<uint16_t*>(s_warp + 32);
-    uint8_t* s_priv = reinterpret_cast<uint8_t*>(s_owner) + ((cfg.max_groups * 2 + 15) & ~15u);
-    uint32_t* my_region = reinterpret_cast<uint32_t*>(s_priv + tid * cfg.region_bytes);
-    const uint32_t region_words = cfg.region_bytes / 4;
+    uint32_t* s_hdr = s_warp + 32;  // the staged table's shortest code length and check word
+    OwnerT* s_owner = reinterpret_cast<OwnerT*>(s_hdr + 4);
+    uint8_t* s_priv = reinterpret_cast<uint8_t*>(s_owner) + ((cfg.max_groups * sizeof(OwnerT) + 15) & ~15u);
+    const uint32_t RB = cfg.region_bytes;
+    uint32_t* my_region = reinterpret_cast<uint32_t*>(s_priv + tid * RB);
 
+    const DevTensor* td = nullptr;
     const DevTensor* staged = nullptr;
+    uint64_t t_lo = 0, t_hi = 0;
     for (uint64_t g = blockIdx.x; g < cfg.total_blocks; g += gridDim.x) {
-        uint64_t b;
-        const DevTensor* td = src.lookup(g, &b);
+        if (g < t_lo || g >= t_hi) td = src.find(g, &t_lo, &t_hi);
+        const uint64_t b = g - t_lo;
+        const uint32_t C = td->chunk_bytes;
         // 1. tables (when the tensor changes) and the stream slice
         if (td != staged) {
             const uint4* t4 = reinterpret_cast<const uint4*>(td->lut);
             uint4* d4 = reinterpret_cast<uint4*>(smem);
             for (uint32_t i = tid; i < kWideWords / 4; i += T) d4[i] = __ldg(t4 + i);
+            if (tid == 0) {
+                const uint32_t* hdr = td->lut + kWideWords + static_cast<size_t>(td->n_tables) * 256 + 64;
+                const uint32_t minl = __ldg(hdr);
+                const bool ok = __ldg(hdr + 3) == kLutMagic && __ldg(hdr + 2) == td->n_tables && minl >= 1 &&
+                                (8 * C + minl - 1) / minl + 12 <= RB;
+                s_hdr[0] = ok ? 1u : 0u;
+            }
             staged = td;
         }
-        const uint32_t C = td->chunk_bytes;
+        // warm L2 with this slot's next block of the same tensor
+        const uint64_t g_next = g + gridDim.x;
+        if (tid == 0 && g_next < t_hi) {
+            const uint64_t bn = g_next - t_lo;
+            const uint64_t s0 = bn * T * C;
+            const uint64_t s_bytes = min(static_cast<uint64_t>(T) * C + 16, td->n_chunks * C + 16 - s0);
+            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(td->stream + s0),
+                         "r"(static_cast<uint32_t>(s_bytes)) : "memory");
+            const uint64_t a0 = __ldg(td->offs + bn) & ~15ull;
+            const uint64_t a1 = min((__ldg(td->offs + bn + 1) + 15) & ~15ull, td->n & ~15ull);
+            if (td->vec_ok && a1 > a0 && a1 - a0 < (1ull << 24))
+                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(td->sm + a0),
+                             "r"(static_cast<uint32_t>(a1 - a0)) : "memory");
+        }
         const uint32_t wpc = C / 4 + 1;
         uint32_t* my_words = s_words + tid * wpc;
         const uint64_t chunk = b * T + tid;
-        uint32_t p = 0, end = 0;
+        DecState st;
+        st.p = st.end = st.cnt = st.app = 0;
+        st.acc = 0;
+        st.bad = false;
         if (chunk < td->n_chunks) {
             const uint4* c4 = reinterpret_cast<const uint4*>(td->stream + chunk * C);
             for (uint32_t k = 0; k < C / 16; ++k) {
@@ -179,101 +256,55 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_consta
             const uint32_t cbits = 8 * C;
             const uint64_t bit0 = chunk * cbits;
             const uint64_t rem = td->total_bits > bit0 ? td->total_bits - bit0 : 0;
-            p = (two >> (11 - (q & 7))) & 31u;
-            end = static_cast<uint32_t>(rem < cbits ? rem : cbits);
+            st.p = (two >> (11 - (q & 7))) & 31u;
+            st.end = static_cast<uint32_t>(rem < cbits ? rem : cbits);
         }
         const uint64_t out0 = td->offs[b];
         const uint64_t out1 = td->offs[b + 1];
         __syncthreads();
+        if (!s_hdr[0]) {  // tables that do not belong to this descriptor
+            if (tid == 0 && d_err) atomicOr(d_err, DF_EFLAG_TABLES);
+            __syncthreads();
+            continue;
+        }
 
         // 2. decode this thread's chunk into its region
-        uint32_t cnt = 0, nacc = 0, rw = 0;
-        uint64_t acc = 0;
-        bool bad = false;
-        const uint32_t rlim = region_words - 2;
-        for (;;) {  // whole windows before the chunk end
-            const bool act = p + kWideBits <= end && rw < rlim;
+        const uint32_t* hier = td->lut + kWideWords;
+        for (;;) {  // two whole windows per vote
+            const bool act = st.p + 2 * kWideBits <= st.end;
             if (!__any_sync(0xFFFFFFFFu, act)) break;
             if (act) {
-                const uint32_t win = window(my_words, p);
-                const uint32_t x = win >> (32 - kWideBits);
-                const uint32_t m = s_meta[x];
-                uint32_t sy = s_sym[x];
-                uint32_t used = m >> kWideBits, ns;
-                if (used == 0) {
-                    const uint32_t e = long_code(win, td->lut + kWideWords);
-                    ns = (e >> kNsymShift) & 3u;
-                    used = (e >> 8) & 63u;
-                    sy = e & 0xFFu;
-                    if (ns == 0) {
-                        bad = true;
-                        end = p;
-                    }
-                } else {
-                    ns = __popc(m & (kWideN - 1));
-                }
-                cnt += ns;
-                acc |= static_cast<uint64_t>(sy) << (8 * nacc);
-                nacc += ns;
-                if (nacc >= 4) {
-                    my_region[rw++] = static_cast<uint32_t>(acc);
-                    acc >>= 32;
-                    nacc -= 4;
-                }
-                p += used;
+                decode_step<false>(st, my_words, s_wide, hier, my_region);
+                decode_step<false>(st, my_words, s_wide, hier, my_region);
             }
         }
-        for (;;) {  // the last bits: count only the codes that start before the end
-            const bool act = p < end && rw < rlim;
+        for (;;) {  // whole windows
+            const bool act = st.p + kWideBits <= st.end;
             if (!__any_sync(0xFFFFFFFFu, act)) break;
-            if (act) {
-                const uint32_t win = window(my_words, p);
-                const uint32_t x = win >> (32 - kWideBits);
-                const uint32_t m = s_meta[x];
-                uint32_t sy = s_sym[x];
-                uint32_t used = m >> kWideBits, ns, counted;
-                if (used == 0) {
-                    const uint32_t e = long_code(win, td->lut + kWideWords);
-                    ns = counted = (e >> kNsymShift) & 3u;
-                    used = (e >> 8) & 63u;
-                    sy = e & 0xFFu;
-                    if (ns == 0) {
-                        bad = true;
-                        end = p;
-                    }
-                } else {
-                    const uint32_t lim = end - p;  // < kWideBits here
-                    ns = __popc(m & (kWideN - 1));
-                    counted = __popc(m & ((1u << lim) - 1u));
-                }
-                cnt += counted;
-                acc |= static_cast<uint64_t>(sy) << (8 * nacc);
-                nacc += ns;
-                if (nacc >= 4) {
-                    my_region[rw++] = static_cast<uint32_t>(acc);
-                    acc >>= 32;
-                    nacc -= 4;
-                }
-                p += used;
-            }
+            if (act) decode_step<false>(st, my_words, s_wide, hier, my_region);
         }
-        if (p < end) bad = true;  // the region filled up: more codes than the layout allows
-        my_region[rw] = static_cast<uint32_t>(acc);
-        my_region[rw + 1] = static_cast<uint32_t>(acc >> 32);
+        for (;;) {  // windows reaching past the end
+            const bool act = st.p < st.end;
+            if (!__any_sync(0xFFFFFFFFu, act)) break;
+            if (act) decode_step<true>(st, my_words, s_wide, hier, my_region);
+        }
+        my_region[st.app >> 2] = static_cast<uint32_t>(st.acc);
+        my_region[(st.app >> 2) + 1] = static_cast<uint32_t>(st.acc >> 32);
+        const uint32_t cnt = st.cnt;
 
-        // 3. block scan of the counts
+        // 3. block scan of the counts: warp totals (with a corrupt-data bit)
+        // in shared memory, then every warp scans them again on its own
         const uint32_t incl = warp_incl_scan(cnt, lane);
-        if (lane == 31) s_warp[warp] = incl;
+        const bool warp_bad = __any_sync(0xFFFFFFFFu, st.bad);
+        if (lane == 31) s_warp[warp] = incl | (warp_bad ? 0x80000000u : 0u);
         __syncthreads();
-        if (warp == 0) {
-            uint32_t v = lane < static_cast<int>(nwarps) ? s_warp[lane] : 0;
-            v = warp_incl_scan(v, lane);
-            if (lane < static_cast<int>(nwarps)) s_warp[lane] = v;
-        }
-        __syncthreads();
-        const uint32_t total = s_warp[nwarps - 1];
+        const uint32_t wv = lane < static_cast<int>(nwarps) ? s_warp[lane] : 0u;
+        const bool any_bad = __any_sync(0xFFFFFFFFu, wv >> 31);
+        const uint32_t wincl = warp_incl_scan(wv & 0x7FFFFFFFu, lane);
+        const uint32_t wprefix = __shfl_sync(0xFFFFFFFFu, wincl - (wv & 0x7FFFFFFFu), warp);
+        const uint32_t total = __shfl_sync(0xFFFFFFFFu, wincl, nwarps - 1);
         const uint32_t align = static_cast<uint32_t>(out0 & 15);
-        const uint32_t pos = align + incl - cnt + (warp > 0 ? s_warp[warp - 1] : 0);
+        const uint32_t pos = align + wprefix + incl - cnt;
         s_pos[tid] = pos;
         if (tid == T - 1) s_pos[T] = pos + cnt;
 
@@ -284,7 +315,7 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_consta
             flags |= DF_EFLAG_OFFSETS;
         else if (static_cast<uint64_t>(total) != out1 - out0)
             flags |= DF_EFLAG_COUNT;
-        if (__syncthreads_or(bad)) flags |= DF_EFLAG_BAD_CODE;
+        if (any_bad) flags |= DF_EFLAG_BAD_CODE;
         if (flags) {
             if (tid == 0 && d_err) atomicOr(d_err, flags);
             __syncthreads();
@@ -295,8 +326,8 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_consta
         // the thread whose range holds max(16gi, align)
         if (cnt) {
             const uint32_t hi = pos + cnt;
-            if (pos <= align && align < hi) s_owner[0] = static_cast<uint16_t>(tid);
-            for (uint32_t gi = max((pos + 15) >> 4, 1u); 16 * gi < hi; ++gi) s_owner[gi] = static_cast<uint16_t>(tid);
+            if (pos <= align && align < hi) s_owner[0] = static_cast<OwnerT>(tid);
+            for (uint32_t gi = max((pos + 15) >> 4, 1u); 16 * gi < hi; ++gi) s_owner[gi] = static_cast<OwnerT>(tid);
         }
         __syncthreads();
 
@@ -311,7 +342,6 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_consta
         const uint64_t gbase = out0 & ~15ull;
         const uint32_t ngroups = (align + total + 15) >> 4;
         const bool vec = td->vec_ok != 0;
-        const uint32_t RB = cfg.region_bytes;
         for (uint32_t gi = tid; gi < ngroups; gi += T) {
             const uint64_t G = gbase + 16ull * gi;
             const uint32_t c0 = 16 * gi;
@@ -408,9 +438,9 @@ df_status prepare(const df_tensor* t, uint16_t* out, Prepared* pr) {
     pr->dev = d;
     pr->words_per_chunk = C / 4 + 1;  // odd: C is a multiple of 16
     // a chunk holds at most 8C/min_len code starts; its region also takes up
-    // to 3 exponents past the last counted code and one partial word
+    // to 3 exponents past the last counted code and the final two-word flush
     const uint64_t per_chunk = (cbits + minl - 1) / (minl ? minl : 1);
-    uint64_t rb = (per_chunk + 8 + 3) & ~3ull;
+    uint64_t rb = (per_chunk + 12 + 3) & ~3ull;
     if (((rb / 4) & 1) == 0) rb += 4;  // odd word stride: regions start in distinct banks
     // a block holds at most 8CT/min_len codes and never more than n
     uint64_t per_block = per_chunk * T;
@@ -422,9 +452,11 @@ df_status prepare(const df_tensor* t, uint16_t* out, Prepared* pr) {
     return DF_OK;
 }
 
+size_t owner_size(uint32_t T);
+
 size_t smem_bytes(const LaunchCfg& c, uint32_t T) {
-    return 6u * kWideN + static_cast<size_t>(T) * c.words_per_chunk * 4 + ((T + 1 + 3) & ~3u) * 4 + 32 * 4 +
-           ((c.max_groups * 2 + 15) & ~15u) + static_cast<size_t>(T) * c.region_bytes;
+    return 8u * kWideN + static_cast<size_t>(T) * c.words_per_chunk * 4 + ((T + 1 + 3) & ~3u) * 4 + 32 * 4 + 16 +
+           ((c.max_groups * owner_size(T) + 15) & ~15u) + static_cast<size_t>(T) * c.region_bytes;
 }
 
 df_status device_limits(int* sms, int* max_smem) {
@@ -438,28 +470,38 @@ df_status device_limits(int* sms, int* max_smem) {
     return DF_OK;
 }
 
-template <class Src>
-df_status launch(const Src& src, const LaunchCfg& cfg, uint32_t T, size_t smem, uint32_t* d_err,
-                 cudaStream_t stream) {
-    if (cfg.total_blocks == 0) return DF_OK;
+template <class Src, class OwnerT>
+df_status launch_as(const Src& src, const LaunchCfg& cfg, uint32_t T, size_t smem, uint32_t* d_err,
+                    cudaStream_t stream) {
     int sms = 0, max_smem = 0;
     df_status st = device_limits(&sms, &max_smem);
     if (st != DF_OK) return st;
     if (smem > static_cast<size_t>(max_smem)) return DF_ERR_UNSUPPORTED;
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<Src>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    auto kern = decode_kernel<Src, OwnerT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return cuda_fail(e);
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<Src>, static_cast<int>(T), smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, static_cast<int>(T), smem);
     if (e != cudaSuccess) return cuda_fail(e);
     if (per_sm < 1) return DF_ERR_UNSUPPORTED;
     // persistent blocks: every resident slot loops over the format blocks
     const uint64_t slots = static_cast<uint64_t>(sms) * per_sm;
     const uint64_t grid = cfg.total_blocks < slots ? cfg.total_blocks : slots;
-    decode_kernel<Src><<<static_cast<unsigned>(grid), T, smem, stream>>>(src, cfg, d_err);
+    kern<<<static_cast<unsigned>(grid), T, smem, stream>>>(src, cfg, d_err);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e);
     return DF_OK;
+}
+
+// owner-map entries are bytes when a block has at most 256 threads
+size_t owner_size(uint32_t T) { return T <= 256 ? 1 : 2; }
+
+template <class Src>
+df_status launch(const Src& src, const LaunchCfg& cfg, uint32_t T, size_t smem, uint32_t* d_err,
+                 cudaStream_t stream) {
+    if (cfg.total_blocks == 0) return DF_OK;
+    return T <= 256 ? launch_as<Src, uint8_t>(src, cfg, T, smem, d_err, stream)
+                    : launch_as<Src, uint16_t>(src, cfg, T, smem, d_err, stream);
 }
 
 void widen(LaunchCfg* c, const Prepared& p) {

@@ -170,7 +170,7 @@ df_status df_build_code(const uint64_t hist[256], uint32_t max_len, df_code* out
 }
 
 size_t df_lut_words(const df_code* code) {
-    return code ? kWideWords + static_cast<size_t>(code->n_tables) * 256 + 64 : 0;
+    return code ? kWideWords + static_cast<size_t>(code->n_tables) * 256 + 64 + 4 : 0;
 }
 
 df_status df_build_lut(const df_code* code, uint32_t* lut, size_t lut_words) {
@@ -210,7 +210,15 @@ df_status df_build_lut(const df_code* code, uint32_t* lut, size_t lut_words) {
     }
     uint32_t* hier = lut + kWideWords;
     std::memcpy(hier, tables.data(), tables.size() * sizeof(uint32_t));
-    std::memcpy(lut + kWideWords + static_cast<size_t>(code->n_tables) * 256, code->lengths, 256);
+    uint32_t* tail = lut + kWideWords + static_cast<size_t>(code->n_tables) * 256;
+    std::memcpy(tail, code->lengths, 256);
+    uint32_t min_len = 0;
+    for (int s = 0; s < 256; ++s)
+        if (code->lengths[s] && (!min_len || code->lengths[s] < min_len)) min_len = code->lengths[s];
+    tail[64] = min_len;  // header: the shortest code, which bounds the codes per chunk
+    tail[65] = code->max_len;
+    tail[66] = code->n_tables;
+    tail[67] = kLutMagic;
 
     // 2. the wide table: for every kWideBits-bit window, the codes that lie
     // wholly inside it from its first bit on (at most kWideMaxCodes)
@@ -222,8 +230,7 @@ df_status df_build_lut(const df_code* code, uint32_t* lut, size_t lut_words) {
         const uint32_t c = code->codes[s];
         for (uint32_t x = c << (W - l); x < ((c + 1) << (W - l)); ++x) first[x] = (l << 8) | static_cast<uint32_t>(s);
     }
-    uint16_t* meta = reinterpret_cast<uint16_t*>(lut);
-    uint32_t* sym = lut + kWideMetaWords;
+    uint64_t* wide = reinterpret_cast<uint64_t*>(lut);
     for (uint32_t x = 0; x < N; ++x) {
         uint32_t used = 0, n = 0, mask = 0, syms = 0;
         while (n < kWideMaxCodes && used < W) {
@@ -235,8 +242,8 @@ df_status df_build_lut(const df_code* code, uint32_t* lut, size_t lut_words) {
             used += l;
             ++n;
         }
-        meta[x] = static_cast<uint16_t>(mask | (used << kWideBits));
-        sym[x] = syms;
+        wide[x] = syms | (static_cast<uint64_t>(mask) << kWideMaskShift) |
+                  (static_cast<uint64_t>(used) << kWideUsedShift) | (static_cast<uint64_t>(n) << kWideCountShift);
     }
     return DF_OK;
 }

@@ -327,3 +327,20 @@ def test_invalid_arguments_are_rejected():
         api.df_decode(bad, out)
     with pytest.raises(TypeError):
         api.df_decode(d, out.cpu())
+
+
+def test_tables_of_another_code_are_reported():
+    # descriptor of tensor A with the decode tables of tensor B (B has more
+    # tables, so every read stays inside B's table buffer)
+    wa = synth.generate(synth.single_1024x4096()[0])[:100_000]
+    wb = synth.generate(synth.heavy_tail_64m()[0])[:2_000_000]
+    ca = from_oracle(oracle.encode(wa))
+    cb = from_oracle(oracle.encode(wb))
+    assert cb.code.n_tables > ca.code.n_tables
+    d = ca.descriptor()
+    bad = type(d).from_buffer_copy(d)
+    bad.lut = cb.lut.data_ptr()
+    out = torch.empty(wa.size, dtype=torch.int16, device="cuda")
+    err = err_word()
+    api.df_decode(bad, out, err)
+    assert api.df_read_error(err) & 8

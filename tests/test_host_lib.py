@@ -116,11 +116,15 @@ def test_plan_matches_oracle_sizes(chunk_bytes, tpb):
 
 
 def wide_bits(lut, n_tables):
-    """The wide table's window width, from the table sizes (1.5 * 2^W words)."""
-    words = lut.size - 256 * n_tables - 64
-    W = int(round(np.log2(words / 1.5)))
-    assert 3 * (1 << W) // 2 == words
+    """The wide table's window width, from the table sizes (2^W uint64)."""
+    words = lut.size - 256 * n_tables - 64 - 4
+    W = int(round(np.log2(words / 2)))
+    assert 2 * (1 << W) == words
     return W
+
+
+def wide_entries(lut, W):
+    return np.frombuffer(lut[: 2 * (1 << W)].tobytes(), np.uint64)
 
 
 def table_walk_decode(stream, total_bits, n, gaps_fields, offsets, lut, n_tables, chunk_bytes, tpb):
@@ -130,9 +134,9 @@ def table_walk_decode(stream, total_bits, n, gaps_fields, offsets, lut, n_tables
     the chunk end are counted), a longer code walks the 8-bit tables; counts
     are checked against the block offsets."""
     WIDE = wide_bits(lut, n_tables)
-    meta = np.frombuffer(lut[: (1 << WIDE) // 2].tobytes(), np.uint16)
-    sym = lut[(1 << WIDE) // 2: (1 << WIDE) // 2 + (1 << WIDE)]
-    hier = lut[(1 << WIDE) // 2 + (1 << WIDE):]
+    wide = wide_entries(lut, WIDE)
+    hier = lut[2 * (1 << WIDE):]
+    assert hier[256 * n_tables + 64 + 3] == 0xDF11DF11
     bits = np.unpackbits(np.asarray(stream, np.uint8))
     cb = 8 * chunk_bytes
     n_chunks = len(gaps_fields)
@@ -152,8 +156,8 @@ def table_walk_decode(stream, total_bits, n, gaps_fields, offsets, lut, n_tables
         cnt = 0
         while p < end:
             win = window(p)
-            m = int(meta[win >> (32 - WIDE)])
-            used = m >> WIDE
+            e = int(wide[win >> (32 - WIDE)])
+            used = (e >> 42) & 15
             if used == 0:
                 e = int(hier[win >> 24])
                 for lvl in (1, 2, 3):
@@ -167,10 +171,11 @@ def table_walk_decode(stream, total_bits, n, gaps_fields, offsets, lut, n_tables
                 cnt += 1
                 p += (e >> 8) & 63
                 continue
-            mask = m & ((1 << WIDE) - 1)
+            mask = (e >> 32) & ((1 << WIDE) - 1)
+            assert bin(mask).count("1") == (e >> 46) & 7
             lim = min(end - p, WIDE)
             starts = [i for i in range(WIDE) if (mask >> i) & 1 and i < lim]
-            sy = int(sym[win >> (32 - WIDE)])
+            sy = e & 0xFFFFFFFF
             for k in range(len(starts)):
                 out.append((sy >> (8 * k)) & 0xFF)
             cnt += len(starts)
@@ -215,15 +220,16 @@ def test_unreachable_entries_are_zero():
     code = api.df_build_code(h)
     lut = api.df_build_lut(code)
     WIDE = wide_bits(lut, code.n_tables)
-    meta = np.frombuffer(lut[: (1 << WIDE) // 2].tobytes(), np.uint16)
+    wide = wide_entries(lut, WIDE)
     half = 1 << (WIDE - 1)
-    assert (meta[half:] == 0).all() and (meta[:half] != 0).all()
-    hier = lut[(1 << WIDE) // 2 + (1 << WIDE):]
+    assert (wide[half:] == 0).all() and (wide[:half] != 0).all()
+    hier = lut[2 * (1 << WIDE):]
     assert (hier[128:256] == 0).all() and (hier[:128] != 0).all()
+    assert list(hier[256 * code.n_tables + 64:]) == [1, 32, code.n_tables, 0xDF11DF11]
     # 256 equally frequent exponents: every code has 8 bits, every entry is reached
     code = api.df_build_code(np.full(256, 7, dtype=np.uint64))
     lut = api.df_build_lut(code)
-    meta = np.frombuffer(lut[: (1 << WIDE) // 2].tobytes(), np.uint16)
-    assert ((meta >> WIDE) == 8).all()
-    hier = lut[(1 << WIDE) // 2 + (1 << WIDE):]
+    wide = wide_entries(lut, WIDE)
+    assert (((wide >> np.uint64(42)) & np.uint64(15)) == 8).all()
+    hier = lut[2 * (1 << WIDE):]
     assert (hier[:256] != 0).all()
