@@ -275,7 +275,8 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_consta
             if (!__any_sync(0xFFFFFFFFu, act)) break;
             if (act) {
                 decode_step<false>(st, my_words, s_wide, hier, my_region);
-                decode_step<false>(st, my_words, s_wide, hier, my_region);
+                // a long code may have moved p past the second window
+                if (st.p + kWideBits <= st.end) decode_step<false>(st, my_words, s_wide, hier, my_region);
             }
         }
         for (;;) {  // whole windows

@@ -10,6 +10,7 @@ import torch
 import oracle
 from lossless_bf16_weight_huffman_b200 import api, codec, synth
 from lossless_bf16_weight_huffman_b200._native import DfError
+from tests.cases import long_code_tensor
 from tests.gpu_util import assert_container_equal, dev_u16, err_word, from_oracle, gpu_decode, host_u16
 
 pytestmark = pytest.mark.gpu
@@ -344,3 +345,14 @@ def test_tables_of_another_code_are_reported():
     err = err_word()
     api.df_decode(bad, out, err)
     assert api.df_read_error(err) & 8
+
+
+@pytest.mark.parametrize("chunk_bytes,tpb", [(16, 32), (32, 256), (64, 128)])
+def test_decode_many_long_codes(chunk_bytes, tpb):
+    # 30% of the codes are longer than the wide window: the long-code path at
+    # every position in a chunk, including right before its end
+    w, lengths = long_code_tensor(400_001)
+    enc = oracle.encode(w, chunk_bytes=chunk_bytes, threads_per_block=tpb, lengths=lengths)
+    c = from_oracle(enc)
+    out, flags = gpu_decode(c)
+    assert flags == 0 and (out == w).all()

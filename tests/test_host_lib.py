@@ -12,6 +12,7 @@ import pytest
 
 import oracle
 from lossless_bf16_weight_huffman_b200 import _native, api, synth
+from tests.cases import long_code_tensor
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -150,36 +151,48 @@ def table_walk_decode(stream, total_bits, n, gaps_fields, offsets, lut, n_tables
             v = (v << 1) | int(b)
         return v << (32 - len(w))
 
+    def step(p, end, tail):
+        """One table step at bit p; returns (new p, codes counted)."""
+        win = window(p)
+        e = int(wide[win >> (32 - WIDE)])
+        used = (e >> 42) & 15
+        if used == 0:  # a code longer than the window: the 8-bit tables
+            e = int(hier[win >> 24])
+            for lvl in (1, 2, 3):
+                if (e >> 24) & 3:
+                    break
+                t = e & 0xFFFF
+                assert t != 0, "unreachable entry"
+                e = int(hier[t * 256 + ((win >> (24 - 8 * lvl)) & 0xFF)])
+            assert (e >> 24) & 3 == 1
+            out.append(e & 0xFF)
+            return p + ((e >> 8) & 63), 1
+        mask = (e >> 32) & ((1 << WIDE) - 1)
+        assert bin(mask).count("1") == (e >> 46) & 7
+        lim = end - p if tail else WIDE
+        starts = [i for i in range(WIDE) if (mask >> i) & 1 and i < lim]
+        for k in range(len(starts)):
+            out.append(((e & 0xFFFFFFFF) >> (8 * k)) & 0xFF)
+        return p + used, len(starts)
+
     for j in range(n_chunks):
         p = j * cb + int(gaps_fields[j])
         end = min((j + 1) * cb, total_bits)
         cnt = 0
+        # the kernel's three phases: pairs of whole windows, whole windows,
+        # windows that reach past the chunk end
+        while p + 2 * WIDE <= end:
+            p, c = step(p, end, False)
+            cnt += c
+            if p + WIDE <= end:
+                p, c = step(p, end, False)
+                cnt += c
+        while p + WIDE <= end:
+            p, c = step(p, end, False)
+            cnt += c
         while p < end:
-            win = window(p)
-            e = int(wide[win >> (32 - WIDE)])
-            used = (e >> 42) & 15
-            if used == 0:
-                e = int(hier[win >> 24])
-                for lvl in (1, 2, 3):
-                    if (e >> 24) & 3:
-                        break
-                    t = e & 0xFFFF
-                    assert t != 0, "unreachable entry"
-                    e = int(hier[t * 256 + ((win >> (24 - 8 * lvl)) & 0xFF)])
-                assert (e >> 24) & 3 == 1
-                out.append(e & 0xFF)
-                cnt += 1
-                p += (e >> 8) & 63
-                continue
-            mask = (e >> 32) & ((1 << WIDE) - 1)
-            assert bin(mask).count("1") == (e >> 46) & 7
-            lim = min(end - p, WIDE)
-            starts = [i for i in range(WIDE) if (mask >> i) & 1 and i < lim]
-            sy = e & 0xFFFFFFFF
-            for k in range(len(starts)):
-                out.append((sy >> (8 * k)) & 0xFF)
-            cnt += len(starts)
-            p += used
+            p, c = step(p, end, True)
+            cnt += c
         counts.append(cnt)
     counts = np.array(counts)
     per_block = [int(counts[b * tpb:(b + 1) * tpb].sum()) for b in range(len(offsets) - 1)]
@@ -188,10 +201,11 @@ def table_walk_decode(stream, total_bits, n, gaps_fields, offsets, lut, n_tables
     return np.array(out, np.uint8)
 
 
-@pytest.mark.parametrize("case", ["normal", "heavy12", "single", "all256", "heavy9"])
+@pytest.mark.parametrize("case", ["normal", "heavy12", "single", "all256", "heavy9", "long_codes"])
 def test_tables_decode_oracle_streams(case):
     rng = np.random.default_rng(99)
     chunk_bytes, tpb, max_len = 16, 32, 32
+    lengths = None
     if case == "normal":
         w = synth.generate(synth.single_1024x4096()[0])[:6000]
     elif case.startswith("heavy"):
@@ -204,9 +218,11 @@ def test_tables_decode_oracle_streams(case):
         max_len = int(case[5:])
     elif case == "single":
         w = (0x3F80 | rng.integers(0, 128, size=3000)).astype(np.uint16)
+    elif case == "long_codes":
+        w, lengths = long_code_tensor(20000)
     else:
         w = ((np.arange(4096) % 256) << 7).astype(np.uint16)
-    enc = oracle.encode(w, max_len=max_len, chunk_bytes=chunk_bytes, threads_per_block=tpb)
+    enc = oracle.encode(w, max_len=max_len, chunk_bytes=chunk_bytes, threads_per_block=tpb, lengths=lengths)
     code = api.df_code_from_lengths(enc.lengths, max_len)
     lut = api.df_build_lut(code)
     exps = table_walk_decode(enc.stream, enc.total_bits, enc.n, oracle.unpack_gaps(enc.gaps, enc.sizes["n_chunks"]),
