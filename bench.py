@@ -60,6 +60,9 @@ def parse():
                    choices=["llama8b_shaped", "llama_layer", "single_1024x4096", "heavy_tail_64m", "mixed_2000"],
                    help="weight set to decode (the headline number is llama8b_shaped)")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--chunk-bytes", type=int, default=0,
+                   help="format chunk size C in bytes (0: 32, or 16 where the shortest code is 1 bit)")
+    p.add_argument("--threads-per-block", type=int, default=256, help="format block size T in chunks")
     return p.parse_args()
 
 
@@ -285,16 +288,17 @@ def run_gpu(args, world, rank, local):
         ev[1].record()
         hist = hist_d.cpu().numpy().view(np.uint64)
         code = api.df_build_code(hist, 32)
-        C = codec.auto_chunk_bytes(code)
+        C = args.chunk_bytes or codec.auto_chunk_bytes(code)
+        TPB = args.threads_per_block
         lut = torch.from_numpy(api.df_build_lut(code).view(np.int32)).to(dev)
-        z = api.df_plan(code, hist, n, C, 256).as_dict()
+        z = api.df_plan(code, hist, n, C, TPB).as_dict()
         bufs = dict(stream=torch.empty(z["stream_bytes"], dtype=torch.uint8, device=dev),
                     gaps=torch.empty(z["gap_bytes"], dtype=torch.uint8, device=dev),
                     offsets=torch.empty(z["n_blocks"] + 1, dtype=torch.int64, device=dev),
                     sm=torch.empty(n, dtype=torch.uint8, device=dev))
         ws = torch.empty(z["encode_ws_bytes"], dtype=torch.uint8, device=dev)
         ev[2].record()
-        api.df_encode(code, x, z["total_bits"], C, 256, bufs["stream"], bufs["gaps"], bufs["offsets"], bufs["sm"],
+        api.df_encode(code, x, z["total_bits"], C, TPB, bufs["stream"], bufs["gaps"], bufs["offsets"], bufs["sm"],
                       ws, err)
         ev[3].record()
         torch.cuda.synchronize()
@@ -302,7 +306,7 @@ def run_gpu(args, world, rank, local):
         enc_ms += ev[2].elapsed_time(ev[3])
         del ws
         comps.append(codec.Compressed(n=n, shape=s.shape, code=code, lut=lut, sizes=z, chunk_bytes=C,
-                                      threads_per_block=256, **bufs))
+                                      threads_per_block=TPB, **bufs))
         src.append(x)
     assert api.df_read_error(err) == 0, "encode reported an error"
     container = sum(c.container_bytes for c in comps)
@@ -463,8 +467,8 @@ def run_gpu(args, world, rank, local):
             "data": "synthetic (seeded; Box-Muller normals rounded to BF16, shapes of an 8B Llama-style model)",
             "config": {"workload": WORKLOAD if args.workload == "llama8b_shaped" else args.workload,
                        "weights": n_total, "tensors": len(specs),
-                       "chunk_bytes": "32 (16 for tensors whose shortest code is 1 bit)",
-                       "threads_per_block": 256, "max_len": 32,
+                       "chunk_bytes": args.chunk_bytes or "32 (16 for tensors whose shortest code is 1 bit)",
+                       "threads_per_block": args.threads_per_block, "max_len": 32,
                        "l2": f"inputs ({(read_bytes + bf16_bytes) / 1e9:.2f} GB) larger than L2: no flush"
                        if read_bytes + bf16_bytes > 2 * 126e6 else "L2-resident (no flush)",
                        "parallelism": f"{world} replica(s), no collective" if world > 1 else "1 GPU"},

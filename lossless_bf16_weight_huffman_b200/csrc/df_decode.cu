@@ -219,7 +219,7 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_consta
             }
             staged = td;
         }
-        // warm L2 with this slot's next block of the same tensor
+        // warm L2 with the stream slice of this slot's next block of the same tensor
         const uint64_t g_next = g + gridDim.x;
         if (tid == 0 && g_next < t_hi) {
             const uint64_t bn = g_next - t_lo;
@@ -227,11 +227,6 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_consta
             const uint64_t s_bytes = min(static_cast<uint64_t>(T) * C + 16, td->n_chunks * C + 16 - s0);
             asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(td->stream + s0),
                          "r"(static_cast<uint32_t>(s_bytes)) : "memory");
-            const uint64_t a0 = __ldg(td->offs + bn) & ~15ull;
-            const uint64_t a1 = min((__ldg(td->offs + bn + 1) + 15) & ~15ull, td->n & ~15ull);
-            if (td->vec_ok && a1 > a0 && a1 - a0 < (1ull << 24))
-                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(td->sm + a0),
-                             "r"(static_cast<uint32_t>(a1 - a0)) : "memory");
         }
         const uint32_t wpc = C / 4 + 1;
         uint32_t* my_words = s_words + tid * wpc;
@@ -375,12 +370,21 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_consta
                 dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
                 dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
             } else {
-                for (uint32_t k = 0; k < 16; ++k) {
-                    const uint64_t i = G + k;
-                    if (i < out0 || i >= out1) continue;
+                // a group at either end of the block, or over three or more
+                // regions: exponents one by one from shared memory, the
+                // sign|fraction bytes in one load where the group lies inside
+                // the tensor, stores one weight at a time
+                const uint64_t k0 = G < out0 ? out0 - G : 0;
+                const uint64_t k1 = G + 16 <= out1 ? 16 : out1 - G;
+                const bool whole = vec && G + 16 <= td->n;
+                uint4 s16 = make_uint4(0, 0, 0, 0);
+                if (whole) s16 = __ldg(reinterpret_cast<const uint4*>(sm + G));
+                for (uint32_t k = static_cast<uint32_t>(k0); k < k1; ++k) {
                     const uint32_t c = c0 + k;
                     while (c >= s_pos[t + 1]) ++t;
-                    out[i] = merge1(sm[i], s_priv[t * RB + (c - s_pos[t])]);
+                    const uint32_t word = k < 8 ? (k < 4 ? s16.x : s16.y) : (k < 12 ? s16.z : s16.w);
+                    const uint8_t sbyte = whole ? static_cast<uint8_t>(word >> (8 * (k & 3))) : sm[G + k];
+                    out[G + k] = merge1(sbyte, s_priv[t * RB + (c - s_pos[t])]);
                 }
             }
         }
