@@ -21,8 +21,10 @@ struct DevTensor {
     uint64_t n_chunks;
     uint32_t n_blocks;
     uint32_t n_tables;
-    uint32_t chunk_bytes;
+    uint32_t chunk_bytes;  // C
+    uint32_t tpb;          // T: chunks per format block
     uint32_t vec_ok;       // sm and out 16-byte aligned
+    uint32_t pad;
 };
 
 // Decode tables (the words df_build_lut writes), in order:
