@@ -110,10 +110,10 @@ typedef struct df_tensor {
 typedef struct df_batch_plan {
     void* d_ws;                /* the workspace holding the device table        */
     uint32_t count;            /* tensors with n > 0                            */
-    uint32_t threads_per_block;/* CUDA threads per block of the launch (256)    */
+    uint32_t threads_per_block;/* T, shared by all tensors (CUDA block size)    */
     uint32_t words_per_chunk;  /* shared-memory words per chunk (widest C)      */
-    uint32_t region_bytes;     /* per-lane exponent region in shared memory     */
-    uint32_t max_groups;       /* per-warp owner-map bytes (16-weight groups)   */
+    uint32_t stage_bytes;      /* exponent stage of a block in shared memory    */
+    uint32_t reserved;
     uint32_t smem_bytes;       /* dynamic shared memory per CUDA block          */
     uint64_t total_blocks;     /* format blocks over all tensors                */
 } df_batch_plan;
@@ -207,13 +207,14 @@ df_status df_encode(const df_code* code, const uint16_t* d_in, uint64_t n, uint6
 
 /* ---- decode (device) ---------------------------------------------------------
  * df_decode: d_out[0..t->n) = the original BF16 bit patterns (uint16, device;
- * 16-byte alignment of d_out and t->sm takes the vector path). A warp decodes
- * one format block (T chunks) at a time, 32 chunks per sub-round: each lane
- * decodes the codes that start in its chunk through the wide table staged in
- * shared memory into its own shared-memory region and counts them, a warp
- * scan turns the counts into output positions, and the warp merges the
- * exponents with the sign|fraction bytes into 16-byte stores. Source: mlx-dfloat, intro and "Status" (blockwise
- * GPU decode back to identical bits); df11pack, "Use" (chunks).
+ * 16-byte alignment of d_out and t->sm takes the vector path). A CUDA block
+ * of T threads decodes one format block (T chunks) at a time: the wide table
+ * and the block's stream slice are staged in shared memory, each thread
+ * counts the codes that start in its chunk, a block scan turns the counts
+ * into output positions, a second pass stores the exponents into a shared
+ * stage in output order, and the block merges them with the sign|fraction
+ * bytes into 16-byte stores. Source: mlx-dfloat, intro and "Status"
+ * (blockwise GPU decode back to identical bits); df11pack, "Use" (chunks).
  * Data errors set DF_EFLAG_* in d_err (nullable) and skip the affected
  * block's stores. Errors: DF_ERR_INVALID_ARG, DF_ERR_UNSUPPORTED (a layout
  * whose block needs more shared memory than the device has), DF_ERR_CUDA.
@@ -226,8 +227,8 @@ size_t df_decode_batch_workspace(uint32_t count);
 /* df_decode_batch_prepare: validate `count` descriptors (host array) and
  * their outputs (host array of device pointers), write the device table into
  * d_ws (asynchronously on `stream`; the host arrays may be reused on return)
- * and fill *plan. chunk_bytes and threads_per_block may differ between
- * tensors (shared memory is sized for the widest chunk).
+ * and fill *plan. All tensors must share threads_per_block; chunk_bytes may
+ * differ (shared memory is sized for the widest).
  * Errors: DF_ERR_INVALID_ARG, DF_ERR_WORKSPACE, DF_ERR_UNSUPPORTED, DF_ERR_CUDA. */
 df_status df_decode_batch_prepare(const df_tensor* tensors, uint16_t* const* d_outs, uint32_t count, void* d_ws,
                                   size_t ws_bytes, df_batch_plan* plan, void* stream);
