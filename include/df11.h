@@ -205,6 +205,26 @@ df_status df_encode(const df_code* code, const uint16_t* d_in, uint64_t n, uint6
                     uint64_t* d_block_offsets, uint8_t* d_sm, void* d_ws, size_t ws_bytes, uint32_t* d_err,
                     void* stream);
 
+/* df_encode_noalloc: df_encode without a workspace argument, for callers
+ * that cannot allocate device memory when they encode (for example a
+ * runtime that owns all device memory up front in a fixed arena, or a plug-in
+ * that may only use the buffers its host hands it). Its scratch (per-tile bit
+ * counts and bases) lives in a static device array of the library, 2 MiB per
+ * GPU that loads the library, held until the process exits; n is limited to
+ * DF_ENCODE_NOALLOC_MAX_WEIGHTS. The first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress) and caches it; make that
+ * first call before any stream capture. Every call on a device shares the
+ * array, so calls that overlap on the GPU (other streams, other host threads)
+ * race: serialize them. Allocates nothing: no cudaMalloc, cudaFree or
+ * allocating library routine. The pages have no counterpart of this entry
+ * point. Arguments, outputs and errors as df_encode, plus DF_ERR_UNSUPPORTED
+ * when n > DF_ENCODE_NOALLOC_MAX_WEIGHTS.
+ */
+#define DF_ENCODE_NOALLOC_MAX_WEIGHTS (1ull << 29) /* 536,870,912 weights */
+df_status df_encode_noalloc(const df_code* code, const uint16_t* d_in, uint64_t n, uint64_t total_bits,
+                            uint32_t chunk_bytes, uint32_t threads_per_block, uint8_t* d_stream, uint8_t* d_gaps,
+                            uint64_t* d_block_offsets, uint8_t* d_sm, uint32_t* d_err, void* stream);
+
 /* ---- decode (device) ---------------------------------------------------------
  * df_decode: d_out[0..t->n) = the original BF16 bit patterns (uint16, device;
  * 16-byte alignment of d_out and t->sm takes the vector path). A CUDA block

@@ -25,10 +25,12 @@ DF_EFLAG_TABLES = 8
 DF_EFLAG_ENC_TOTAL = 16
 DF_EFLAG_ENC_SYMBOL = 32
 
+DF_ENCODE_NOALLOC_MAX_WEIGHTS = 1 << 29
+
 # every function declared in include/df11.h
 EXPORTS = (
     "df_status_string", "df_last_cuda_error", "df_build_code", "df_code_from_lengths", "df_lut_words", "df_build_lut", "df_plan",
-    "df_histogram", "df_encode", "df_decode", "df_decode_batch_workspace", "df_decode_batch_prepare",
+    "df_histogram", "df_encode", "df_encode_noalloc", "df_decode", "df_decode_batch_workspace", "df_decode_batch_prepare",
     "df_decode_batch_run", "df_decode_batch", "df_read_error",
 )
 
@@ -131,6 +133,8 @@ def lib() -> ctypes.CDLL:
     L.df_histogram.restype = i32
     L.df_encode.argtypes = [ctypes.POINTER(DfCode), vp, u64, u64, u32, u32, vp, vp, vp, vp, vp, sz, vp, vp]
     L.df_encode.restype = i32
+    L.df_encode_noalloc.argtypes = [ctypes.POINTER(DfCode), vp, u64, u64, u32, u32, vp, vp, vp, vp, vp, vp]
+    L.df_encode_noalloc.restype = i32
     L.df_decode.argtypes = [ctypes.POINTER(DfTensor), vp, vp, vp]
     L.df_decode.restype = i32
     L.df_decode_batch_workspace.argtypes = [u32]

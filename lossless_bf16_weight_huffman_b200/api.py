@@ -93,6 +93,18 @@ def df_encode(code: DfCode, d_in: torch.Tensor, total_bits: int, chunk_bytes: in
         _dev(d_sm, "d_sm"), _dev(d_ws, "d_ws"), ws_bytes, _dev(d_err, "d_err"), _stream_ptr(stream)))
 
 
+def df_encode_noalloc(code: DfCode, d_in: torch.Tensor, total_bits: int, chunk_bytes: int, threads_per_block: int,
+                      d_stream: torch.Tensor, d_gaps: torch.Tensor, d_block_offsets: torch.Tensor,
+                      d_sm: torch.Tensor, d_err: torch.Tensor | None = None, stream=None) -> None:
+    """df_encode with the library's static scratch instead of a workspace
+    (for callers that cannot allocate device memory; calls on one GPU must not
+    overlap)."""
+    check("df_encode_noalloc", lib().df_encode_noalloc(
+        ctypes.byref(code), _dev(d_in, "d_in"), d_in.numel(), total_bits, chunk_bytes, threads_per_block,
+        _dev(d_stream, "d_stream"), _dev(d_gaps, "d_gaps"), _dev(d_block_offsets, "d_block_offsets"),
+        _dev(d_sm, "d_sm"), _dev(d_err, "d_err"), _stream_ptr(stream)))
+
+
 def df_decode(t: DfTensor, d_out: torch.Tensor, d_err: torch.Tensor | None = None, stream=None) -> None:
     check("df_decode", lib().df_decode(ctypes.byref(t), _dev(d_out, "d_out"), _dev(d_err, "d_err"),
                                        _stream_ptr(stream)))

@@ -17,6 +17,7 @@
 #include <cuda_runtime.h>
 
 #include <cstring>
+#include <mutex>
 
 #include "df_internal.h"
 
@@ -281,6 +282,33 @@ df_status sm_count(int* sms) {
     return DF_OK;
 }
 
+// Scratch of df_encode_noalloc: per-tile bit counts and bases for at most
+// DF_ENCODE_NOALLOC_MAX_WEIGHTS weights, in a file-scope device array (2 MiB
+// + 32 bytes). Host code must not use the array's name as a device address;
+// noalloc_scratch() looks the address up once per device.
+constexpr uint64_t kNoAllocTiles = DF_ENCODE_NOALLOC_MAX_WEIGHTS / kTile;
+static __device__ __align__(256) uint64_t g_noalloc_scratch[2 * (kNoAllocTiles + 2) + 32];
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_address[kMaxDevices] = {};
+
+// The device address of the static scratch on the current device.
+df_status noalloc_scratch(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev < 0 || dev >= kMaxDevices) return DF_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_address[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e);
+        g_noalloc_address[dev] = p;
+    }
+    *out = g_noalloc_address[dev];
+    return DF_OK;
+}
+
 }  // namespace
 }  // namespace df
 
@@ -365,6 +393,17 @@ df_status df_encode(const df_code* code, const uint16_t* d_in, uint64_t n, uint6
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e);
     return DF_OK;
+}
+
+df_status df_encode_noalloc(const df_code* code, const uint16_t* d_in, uint64_t n, uint64_t total_bits,
+                            uint32_t chunk_bytes, uint32_t tpb, uint8_t* d_stream, uint8_t* d_gaps,
+                            uint64_t* d_block_offsets, uint8_t* d_sm, uint32_t* d_err, void* stream) {
+    if (n > DF_ENCODE_NOALLOC_MAX_WEIGHTS) return DF_ERR_UNSUPPORTED;
+    void* ws = nullptr;
+    const df_status st = noalloc_scratch(&ws);
+    if (st != DF_OK) return st;
+    return df_encode(code, d_in, n, total_bits, chunk_bytes, tpb, d_stream, d_gaps, d_block_offsets, d_sm, ws,
+                     sizeof(g_noalloc_scratch), d_err, stream);
 }
 
 }  // extern "C"
