@@ -144,7 +144,7 @@ df_status df_build_code(const uint64_t hist[256], uint32_t max_len, df_code* out
  * sum 2^-l <= 1); DF_ERR_UNSUPPORTED (max_len outside 1..32). */
 df_status df_code_from_lengths(const uint8_t lengths[256], uint32_t max_len, df_code* out);
 
-/* Number of uint32 words df_build_lut writes: 2048 for the wide table, 256
+/* Number of uint32 words df_build_lut writes: 2560 for the wide table, 256
  * per 8-bit-indexed table, 64 for the code lengths and a 4-word header.
  * 0 for a NULL code. */
 size_t df_lut_words(const df_code* code);
@@ -155,16 +155,17 @@ size_t df_lut_words(const df_code* code);
  *   - the wide table: 1024 uint64 indexed by the next 10 stream bits; an
  *     entry holds the exponents of the codes that lie wholly inside the
  *     window from its first bit on (up to 4, bits 0-31, the first in bits
- *     0-7), a mask of the window bits where they start (bits 32-41), the bits
- *     they use (bits 42-45; 0 when the first code is longer than 10 bits) and
- *     their count (bits 46-48);
+ *     0-7) and, in bits 32-63, (bits they use << 17) | (their count), or 0
+ *     when the first code is longer than 10 bits;
+ *   - 1024 uint16: for each window, the mask of the window bits where those
+ *     codes start;
  *   - n_tables tables of 256 uint32 indexed by 8 stream bits, for codes of
  *     any length: a leaf holds the exponent (bits 0-7), the full code length
  *     (bits 8-13) and a 1 in bits 24-25; a link holds the index of the
  *     next-level table (bits 0-15, >= 1) and 0 in bits 24-25; table 0 is the
  *     root, at most four levels for 32-bit codes;
  *   - the 256 code lengths as bytes;
- *   - a header: the shortest code length, max_len, n_tables, 0xDF11DF11.
+ *   - a header: the shortest code length, max_len, n_tables, 0xDF11DF12.
  * Entries no code reaches are zero. Source: df11pack, "What is checked"
  * (--luts=correct zero-fills unreachable table entries).
  * Errors: DF_ERR_INVALID_ARG (null, too small, or a code that is not prefix free).

@@ -8,14 +8,16 @@
 // One CUDA block of T threads handles one format block (T chunks of C stream
 // bytes) at a time and loops over the blocks of all tensors of the launch:
 //   1. when the tensor changes, stage its wide table (1024 entries indexed by
-//      10 stream bits: the codes that lie wholly inside the window, their
-//      exponents, start mask, bits used and count) in shared memory; stage the
+//      10 stream bits: the exponents of the codes that lie wholly inside the
+//      window and one step word, (bits used << 17) | count, plus the codes'
+//      start masks) in shared memory; stage the
 //      block's stream slice, one chunk per thread, byte-swapped to big-endian
 //      words at an odd word stride (no bank conflicts between the threads'
 //      windows)
 //   2. count pass: each thread counts the codes that start in its chunk
 //      (from chunk start + gap up to the chunk end), up to 4 per table step;
-//      codes longer than 10 bits walk the 8-bit-indexed tables
+//      its state word (bit position << 17) | count advances by one add per
+//      step; codes longer than 10 bits walk the 8-bit-indexed tables
 //   3. block scan of the counts (warp shuffles + one shared array): each
 //      thread's first output position, checked against the block index
 //   4. write pass: each thread decodes its codes again and stores their
@@ -119,111 +121,125 @@ __device__ __forceinline__ void merge4(uint32_t s, uint32_t e, uint32_t* o0, uin
     *o1 = __byte_perm(lo, hi, 0x7362);
 }
 
-// One table step at bit p: the codes (count, exponents, bits) it yields.
-struct Step {
-    uint32_t used;  // bits consumed
-    uint32_t ns;    // codes wholly inside the window (or 1 long code; 0 if corrupt)
-    uint32_t sy;    // their exponents, first in bits 0-7
-    uint32_t mask;  // window bits where they start (wide steps)
-};
-
-__device__ __forceinline__ Step table_step(uint32_t win, const uint64_t* wide, const uint32_t* hier) {
-    Step s;
-    const uint64_t e = wide[win >> (32 - kWideBits)];
-    s.used = static_cast<uint32_t>(e >> kWideUsedShift) & 15u;
-    if (s.used == 0) {  // a code longer than the window (or corrupt data)
-        const uint32_t l = long_code(win, hier);
-        s.ns = (l >> kNsymShift) & 3u;
-        s.used = (l >> 8) & 63u;
-        s.sy = l & 0xFFu;
-        s.mask = 1;
-    } else {
-        s.sy = static_cast<uint32_t>(e);
-        s.ns = static_cast<uint32_t>(e >> kWideCountShift) & 7u;
-        s.mask = static_cast<uint32_t>(e >> kWideMaskShift);
-    }
-    return s;
+// A code longer than the wide window, as a step word ((length << 17) | 1, or
+// 0 for a bit pattern no code starts with) and its exponent.
+__device__ __forceinline__ uint32_t long_step(uint32_t win, const uint32_t* hier, uint32_t* sym) {
+    const uint32_t l = long_code(win, hier);
+    *sym = l & 0xFFu;
+    return l ? (((l >> 8) & 63u) << kStepShift) | 1u : 0u;
 }
 
-// Count the codes that start in [p, end). Sets *bad on a bit pattern no code
-// starts with.
-__device__ __forceinline__ uint32_t count_codes(const uint32_t* words, uint32_t p, uint32_t end, const uint64_t* wide,
+// Count the codes that start in [p0, end). The state word is
+// (bit position << 17) | (codes so far); a table step adds its step word.
+// Sets *bad on a bit pattern no code starts with.
+__device__ __forceinline__ uint32_t count_codes(const uint32_t* words, uint32_t p0, uint32_t end,
+                                                const uint32_t* wide32, const uint16_t* wide_mask,
                                                 const uint32_t* hier, bool* bad) {
-    uint32_t cnt = 0;
+    uint32_t st = p0 << kStepShift;
     for (;;) {  // two whole windows per vote
-        const bool act = p + 2 * kWideBits <= end;
-        if (!__any_sync(kFull, act)) break;
-        if (act) {
-            Step s = table_step(window(words, p), wide, hier);
-            if (s.ns == 0) {
-                *bad = true;
-                end = p;
-            }
-            cnt += s.ns;
-            p += s.used;
-            if (p + kWideBits <= end) {  // a long code may have moved p past the second window
-                s = table_step(window(words, p), wide, hier);
-                if (s.ns == 0) {
-                    *bad = true;
-                    end = p;
-                }
-                cnt += s.ns;
-                p += s.used;
-            }
-        }
-    }
-    for (;;) {  // windows that may reach past the end: count the codes starting before it
-        const bool act = p < end;
-        if (!__any_sync(kFull, act)) break;
-        if (act) {
-            const Step s = table_step(window(words, p), wide, hier);
-            if (s.ns == 0) {
-                *bad = true;
-                end = p;
-            }
-            const uint32_t lim = end - p;
-            cnt += lim >= kWideBits ? s.ns : __popc(s.mask & ((1u << lim) - 1u));
-            p += s.used;
-        }
-    }
-    return cnt;
-}
-
-// Store the exponents of the first `remaining` codes from bit p at stage[pos...].
-// While 4 or more codes remain, all 4 exponent slots of a step are stored
-// (slots past its codes are overwritten by the next step).
-__device__ __forceinline__ void write_codes(const uint32_t* words, uint32_t p, uint32_t remaining, uint8_t* stage,
-                                            uint32_t pos, const uint64_t* wide, const uint32_t* hier) {
-    for (;;) {  // two steps per vote
-        const bool act = remaining >= 8;
+        const bool act = (st >> kStepShift) + 2 * kWideBits <= end;
         if (!__any_sync(kFull, act)) break;
         if (act) {
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
-                const Step s = table_step(window(words, p), wide, hier);
-                stage[pos] = static_cast<uint8_t>(s.sy);
-                stage[pos + 1] = static_cast<uint8_t>(s.sy >> 8);
-                stage[pos + 2] = static_cast<uint8_t>(s.sy >> 16);
-                stage[pos + 3] = static_cast<uint8_t>(s.sy >> 24);
-                pos += s.ns;
-                remaining -= s.ns;
-                p += s.used;
+                const uint32_t win = window(words, st >> kStepShift);
+                uint32_t w = wide32[2 * (win >> (32 - kWideBits)) + 1];
+                if (w == 0) {
+                    uint32_t sym;
+                    w = long_step(win, hier, &sym);
+                    if (w == 0) {
+                        *bad = true;
+                        end = 0;
+                    }
+                }
+                st += w;
+                // a long code may have moved p past the second window
+                if (u == 0 && (st >> kStepShift) + kWideBits > end) break;
+            }
+        }
+    }
+    for (;;) {  // windows that may reach past the end: count the codes starting before it
+        const uint32_t p = st >> kStepShift;
+        const bool act = p < end;
+        if (!__any_sync(kFull, act)) break;
+        if (act) {
+            const uint32_t win = window(words, p);
+            const uint32_t x = win >> (32 - kWideBits);
+            uint32_t w = wide32[2 * x + 1];
+            if (w == 0) {
+                uint32_t sym;
+                w = long_step(win, hier, &sym);
+                if (w == 0) {
+                    *bad = true;
+                    end = 0;
+                }
+            } else if (end - p < kWideBits) {
+                const uint32_t counted = __popc(wide_mask[x] & ((1u << (end - p)) - 1u));
+                w = (w & ~kStepCountMask) | counted;
+            }
+            st += w;
+        }
+    }
+    return st & kStepCountMask;
+}
+
+__device__ __forceinline__ void put4(uint8_t* a, uint32_t sy) {
+    a[0] = static_cast<uint8_t>(sy);
+    a[1] = static_cast<uint8_t>(sy >> 8);
+    a[2] = static_cast<uint8_t>(sy >> 16);
+    a[3] = static_cast<uint8_t>(sy >> 24);
+}
+
+// Store the exponents of the first `cnt` codes from bit p0 at stage[pos0...].
+// The state word is (bit position << 17) | (stage position). While 4 or more
+// codes remain, all 4 exponent slots of a step are stored (slots past its
+// codes are overwritten by the next step).
+__device__ __forceinline__ void write_codes(const uint32_t* words, uint32_t p0, uint32_t cnt, uint8_t* stage,
+                                            uint32_t pos0, const uint64_t* wide, const uint32_t* hier) {
+    uint32_t st = (p0 << kStepShift) | pos0;
+    uint32_t pend = pos0 + cnt;
+    for (;;) {  // two steps per vote
+        const bool act = (st & kStepCountMask) + 8 <= pend;
+        if (!__any_sync(kFull, act)) break;
+        if (act) {
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const uint32_t win = window(words, st >> kStepShift);
+                const uint64_t e = wide[win >> (32 - kWideBits)];
+                uint32_t sy = static_cast<uint32_t>(e);
+                uint32_t w = static_cast<uint32_t>(e >> 32);
+                if (w == 0) {
+                    w = long_step(win, hier, &sy);
+                    if (w == 0) pend = 0;  // cannot follow a clean count pass; never loop on it
+                }
+                put4(stage + (st & kStepCountMask), sy);
+                st += w;
             }
         }
     }
     for (;;) {
-        const bool act = remaining > 0;
+        const uint32_t pos = st & kStepCountMask;
+        const bool act = pos < pend;
         if (!__any_sync(kFull, act)) break;
         if (act) {
-            const Step s = table_step(window(words, p), wide, hier);
-            const uint32_t k = min(s.ns, remaining);
-            stage[pos] = static_cast<uint8_t>(s.sy);
-            if (k > 1) stage[pos + 1] = static_cast<uint8_t>(s.sy >> 8);
-            if (k > 2) stage[pos + 2] = static_cast<uint8_t>(s.sy >> 16);
-            if (k > 3) stage[pos + 3] = static_cast<uint8_t>(s.sy >> 24);
-            pos += k;
-            remaining -= k;
-            p += s.used;
+            const uint32_t win = window(words, st >> kStepShift);
+            const uint64_t e = wide[win >> (32 - kWideBits)];
+            uint32_t sy = static_cast<uint32_t>(e);
+            uint32_t w = static_cast<uint32_t>(e >> 32);
+            if (w == 0) {
+                w = long_step(win, hier, &sy);
+                if (w == 0) {
+                    pend = 0;
+                    continue;
+                }
+            }
+            const uint32_t k = min(w & kStepCountMask, pend - pos);
+            uint8_t* a = stage + pos;
+            a[0] = static_cast<uint8_t>(sy);
+            if (k > 1) a[1] = static_cast<uint8_t>(sy >> 8);
+            if (k > 2) a[2] = static_cast<uint8_t>(sy >> 16);
+            if (k > 3) a[3] = static_cast<uint8_t>(sy >> 24);
+            st += (w & ~kStepCountMask) | k;
         }
     }
 }
@@ -239,7 +255,8 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_consta
 
     // shared memory carve-up (sizes in smem_bytes())
     const uint64_t* s_wide = reinterpret_cast<const uint64_t*>(smem);
-    uint32_t* s_words = reinterpret_cast<uint32_t*>(smem + 8 * kWideN);
+    const uint16_t* s_mask = reinterpret_cast<const uint16_t*>(smem + 8 * kWideN);
+    uint32_t* s_words = reinterpret_cast<uint32_t*>(smem + 4 * kWideWords);
     uint32_t* s_warp = s_words + ((T * cfg.words_per_chunk + 3) & ~3u);
     uint32_t* s_hdr = s_warp + 32;  // 1 when the staged tables belong to the staged tensor
     uint8_t* s_stage = reinterpret_cast<uint8_t*>(s_hdr + 4);
@@ -305,7 +322,8 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_consta
         // 2. count pass
         const uint32_t* hier = td->lut + kWideWords;
         bool bad = false;
-        const uint32_t cnt = count_codes(my_words, p0, end, s_wide, hier, &bad);
+        const uint32_t cnt = count_codes(my_words, p0, end, reinterpret_cast<const uint32_t*>(s_wide), s_mask, hier,
+                                         &bad);
 
         // 3. block scan of the counts: warp totals (with a corrupt-data bit)
         // in shared memory, then every warp scans them again on its own
@@ -386,6 +404,9 @@ df_status prepare(const df_tensor* t, uint16_t* out, Prepared* pr) {
     if (!t || !out) return DF_ERR_INVALID_ARG;
     const uint32_t C = t->chunk_bytes, T = t->threads_per_block;
     if (C < 16 || C > 4096 || C % 16 || T < 32 || T > 1024 || T % 32) return DF_ERR_INVALID_ARG;
+    // the decoder's state word keeps a bit position below 2^15 and a stage
+    // position below 2^17
+    if (C > 2048) return DF_ERR_UNSUPPORTED;
     if (t->max_len < 1 || t->max_len > 32 || t->n_tables < 1) return DF_ERR_INVALID_ARG;
     if (t->n > DF_MAX_WEIGHTS) return DF_ERR_UNSUPPORTED;
     if (!t->stream || !t->gaps || !t->block_offsets || !t->sm || !t->lut) return DF_ERR_INVALID_ARG;
@@ -423,14 +444,14 @@ df_status prepare(const df_tensor* t, uint16_t* out, Prepared* pr) {
     uint64_t per_block = (cbits * T + minl - 1) / (minl ? minl : 1);
     if (per_block > t->n) per_block = t->n;
     const uint64_t stage = (per_block + 16 + 16 + 15) & ~15ull;
-    if (stage > (1u << 24)) return DF_ERR_UNSUPPORTED;
+    if (stage > (1u << kStepShift)) return DF_ERR_UNSUPPORTED;
     pr->stage_bytes = static_cast<uint32_t>(stage);
     return DF_OK;
 }
 
 size_t smem_bytes(const LaunchCfg& c, uint32_t T) {
-    return 8u * kWideN + ((static_cast<size_t>(T) * c.words_per_chunk + 3) & ~static_cast<size_t>(3)) * 4 + 32 * 4 +
-           16 + c.stage_bytes;
+    return 4u * kWideWords + ((static_cast<size_t>(T) * c.words_per_chunk + 3) & ~static_cast<size_t>(3)) * 4 +
+           32 * 4 + 16 + c.stage_bytes;
 }
 
 df_status device_limits(int* sms, int* max_smem) {

@@ -231,6 +231,7 @@ df_status df_build_lut(const df_code* code, uint32_t* lut, size_t lut_words) {
         for (uint32_t x = c << (W - l); x < ((c + 1) << (W - l)); ++x) first[x] = (l << 8) | static_cast<uint32_t>(s);
     }
     uint64_t* wide = reinterpret_cast<uint64_t*>(lut);
+    uint16_t* wide_mask = reinterpret_cast<uint16_t*>(lut + kWideEntryWords);
     for (uint32_t x = 0; x < N; ++x) {
         uint32_t used = 0, n = 0, mask = 0, syms = 0;
         while (n < kWideMaxCodes && used < W) {
@@ -242,8 +243,9 @@ df_status df_build_lut(const df_code* code, uint32_t* lut, size_t lut_words) {
             used += l;
             ++n;
         }
-        wide[x] = syms | (static_cast<uint64_t>(mask) << kWideMaskShift) |
-                  (static_cast<uint64_t>(used) << kWideUsedShift) | (static_cast<uint64_t>(n) << kWideCountShift);
+        const uint32_t step = used ? (used << kStepShift) | n : 0u;
+        wide[x] = syms | (static_cast<uint64_t>(step) << 32);
+        wide_mask[x] = static_cast<uint16_t>(mask);
     }
     return DF_OK;
 }

@@ -31,9 +31,11 @@ struct DevTensor {
 //   wide table, 1024 uint64 indexed by the next kWideBits = 10 stream bits:
 //     bits 0-31  the exponents of the codes that lie wholly inside the window,
 //                taken from its first bit on (at most 4; first in bits 0-7)
-//     bits 32-41 bit i set when one of those codes starts at window bit i
-//     bits 42-45 the bits they use (0: the first code is longer than 10 bits)
-//     bits 46-48 how many there are
+//     bits 32-63 (bits used << 17) | (how many codes); 0 when the first code
+//                is longer than the window. A decoder whose state word is
+//                (bit position << 17) | (codes so far) advances by one add.
+//   wide start masks, 1024 uint16: bit i set when one of those codes starts
+//     at window bit i
 //   8-bit-indexed tables for codes of any length (root + next levels):
 //     leaf:  bits 0-7 the exponent, 8-13 its full code length, 24-25 = 1
 //     link:  bits 0-15 index of the next-level table (>= 1), 24-25 = 0
@@ -42,12 +44,13 @@ struct DevTensor {
 //   header, 4 words: shortest code length, max_len, n_tables, kLutMagic
 constexpr uint32_t kWideBits = 10;
 constexpr uint32_t kWideMaxCodes = 4;
-constexpr uint32_t kWideMaskShift = 32;
-constexpr uint32_t kWideUsedShift = 42;
-constexpr uint32_t kWideCountShift = 46;
-constexpr uint32_t kWideWords = 2u << kWideBits;  // uint32 words of the wide table
+constexpr uint32_t kStepShift = 17;                     // bits-used field of a step word
+constexpr uint32_t kStepCountMask = (1u << kStepShift) - 1;
+constexpr uint32_t kWideEntryWords = 2u << kWideBits;   // the uint64 entries
+constexpr uint32_t kWideMaskWords = (1u << kWideBits) / 2;
+constexpr uint32_t kWideWords = kWideEntryWords + kWideMaskWords;
 constexpr uint32_t kNsymShift = 24;
-constexpr uint32_t kLutMagic = 0xDF11DF11u;
+constexpr uint32_t kLutMagic = 0xDF11DF12u;
 
 inline __host__ __device__ uint32_t sub_leaf(uint32_t sym, uint32_t len) { return sym | (len << 8) | (1u << 24); }
 

@@ -117,15 +117,19 @@ def test_plan_matches_oracle_sizes(chunk_bytes, tpb):
 
 
 def wide_bits(lut, n_tables):
-    """The wide table's window width, from the table sizes (2^W uint64)."""
+    """The wide table's window width, from the table sizes (2^W uint64 + 2^W uint16)."""
     words = lut.size - 256 * n_tables - 64 - 4
-    W = int(round(np.log2(words / 2)))
-    assert 2 * (1 << W) == words
+    W = int(round(np.log2(words / 2.5)))
+    assert 5 * (1 << W) // 2 == words
     return W
 
 
 def wide_entries(lut, W):
     return np.frombuffer(lut[: 2 * (1 << W)].tobytes(), np.uint64)
+
+
+def wide_masks(lut, W):
+    return np.frombuffer(lut[2 * (1 << W): 2 * (1 << W) + (1 << W) // 2].tobytes(), np.uint16)
 
 
 def table_walk_decode(stream, total_bits, n, gaps_fields, offsets, lut, n_tables, chunk_bytes, tpb):
@@ -136,8 +140,9 @@ def table_walk_decode(stream, total_bits, n, gaps_fields, offsets, lut, n_tables
     are checked against the block offsets."""
     WIDE = wide_bits(lut, n_tables)
     wide = wide_entries(lut, WIDE)
-    hier = lut[2 * (1 << WIDE):]
-    assert hier[256 * n_tables + 64 + 3] == 0xDF11DF11
+    masks = wide_masks(lut, WIDE)
+    hier = lut[5 * (1 << WIDE) // 2:]
+    assert hier[256 * n_tables + 64 + 3] == 0xDF11DF12
     bits = np.unpackbits(np.asarray(stream, np.uint8))
     cb = 8 * chunk_bytes
     n_chunks = len(gaps_fields)
@@ -155,8 +160,10 @@ def table_walk_decode(stream, total_bits, n, gaps_fields, offsets, lut, n_tables
         """One table step at bit p; returns (new p, codes counted)."""
         win = window(p)
         e = int(wide[win >> (32 - WIDE)])
-        used = (e >> 42) & 15
+        step_word = e >> 32
+        used = step_word >> 17
         if used == 0:  # a code longer than the window: the 8-bit tables
+            assert step_word == 0
             e = int(hier[win >> 24])
             for lvl in (1, 2, 3):
                 if (e >> 24) & 3:
@@ -167,8 +174,8 @@ def table_walk_decode(stream, total_bits, n, gaps_fields, offsets, lut, n_tables
             assert (e >> 24) & 3 == 1
             out.append(e & 0xFF)
             return p + ((e >> 8) & 63), 1
-        mask = (e >> 32) & ((1 << WIDE) - 1)
-        assert bin(mask).count("1") == (e >> 46) & 7
+        mask = int(masks[win >> (32 - WIDE)])
+        assert bin(mask).count("1") == step_word & ((1 << 17) - 1)
         lim = end - p if tail else WIDE
         starts = [i for i in range(WIDE) if (mask >> i) & 1 and i < lim]
         for k in range(len(starts)):
@@ -239,13 +246,14 @@ def test_unreachable_entries_are_zero():
     wide = wide_entries(lut, WIDE)
     half = 1 << (WIDE - 1)
     assert (wide[half:] == 0).all() and (wide[:half] != 0).all()
-    hier = lut[2 * (1 << WIDE):]
+    assert (wide_masks(lut, WIDE)[half:] == 0).all()
+    hier = lut[5 * (1 << WIDE) // 2:]
     assert (hier[128:256] == 0).all() and (hier[:128] != 0).all()
-    assert list(hier[256 * code.n_tables + 64:]) == [1, 32, code.n_tables, 0xDF11DF11]
+    assert list(hier[256 * code.n_tables + 64:]) == [1, 32, code.n_tables, 0xDF11DF12]
     # 256 equally frequent exponents: every code has 8 bits, every entry is reached
     code = api.df_build_code(np.full(256, 7, dtype=np.uint64))
     lut = api.df_build_lut(code)
     wide = wide_entries(lut, WIDE)
-    assert (((wide >> np.uint64(42)) & np.uint64(15)) == 8).all()
-    hier = lut[2 * (1 << WIDE):]
+    assert ((wide >> np.uint64(32 + 17)) == 8).all()
+    hier = lut[5 * (1 << WIDE) // 2:]
     assert (hier[:256] != 0).all()
