@@ -9,14 +9,14 @@
 // bytes) at a time and loops over the blocks of all tensors of the launch:
 //   1. when the tensor changes, stage its wide table (1024 entries indexed by
 //      10 stream bits: the exponents of the codes that lie wholly inside the
-//      window and one step word, (bits used << 17) | count, plus the codes'
+//      window and one step word, (bits used << 18) | count, plus the codes'
 //      start masks) in shared memory; stage the
 //      block's stream slice, one chunk per thread, byte-swapped to big-endian
 //      words at an odd word stride (no bank conflicts between the threads'
 //      windows)
 //   2. count pass: each thread counts the codes that start in its chunk
 //      (from chunk start + gap up to the chunk end), up to 4 per table step;
-//      its state word (bit position << 17) | count advances by one add per
+//      its state word (bit position << 18) | count advances by one add per
 //      step; codes longer than 10 bits walk the 8-bit-indexed tables
 //   3. block scan of the counts (warp shuffles + one shared array): each
 //      thread's first output position, checked against the block index
@@ -121,7 +121,7 @@ __device__ __forceinline__ void merge4(uint32_t s, uint32_t e, uint32_t* o0, uin
     *o1 = __byte_perm(lo, hi, 0x7362);
 }
 
-// A code longer than the wide window, as a step word ((length << 17) | 1, or
+// A code longer than the wide window, as a step word ((length << 18) | 1, or
 // 0 for a bit pattern no code starts with) and its exponent.
 __device__ __forceinline__ uint32_t long_step(uint32_t win, const uint32_t* hier, uint32_t* sym) {
     const uint32_t l = long_code(win, hier);
@@ -130,7 +130,7 @@ __device__ __forceinline__ uint32_t long_step(uint32_t win, const uint32_t* hier
 }
 
 // Count the codes that start in [p0, end). The state word is
-// (bit position << 17) | (codes so far); a table step adds its step word.
+// (bit position << 18) | (codes so far); a table step adds its step word.
 // Sets *bad on a bit pattern no code starts with.
 __device__ __forceinline__ uint32_t count_codes(const uint32_t* words, uint32_t p0, uint32_t end,
                                                 const uint32_t* wide32, const uint16_t* wide_mask,
@@ -191,7 +191,7 @@ __device__ __forceinline__ void put4(uint8_t* a, uint32_t sy) {
 }
 
 // Store the exponents of the first `cnt` codes from bit p0 at stage[pos0...].
-// The state word is (bit position << 17) | (stage position). While 4 or more
+// The state word is (bit position << 18) | (stage position). While 4 or more
 // codes remain, all 4 exponent slots of a step are stored (slots past its
 // codes are overwritten by the next step).
 __device__ __forceinline__ void write_codes(const uint32_t* words, uint32_t p0, uint32_t cnt, uint8_t* stage,
@@ -404,9 +404,9 @@ df_status prepare(const df_tensor* t, uint16_t* out, Prepared* pr) {
     if (!t || !out) return DF_ERR_INVALID_ARG;
     const uint32_t C = t->chunk_bytes, T = t->threads_per_block;
     if (C < 16 || C > 4096 || C % 16 || T < 32 || T > 1024 || T % 32) return DF_ERR_INVALID_ARG;
-    // the decoder's state word keeps a bit position below 2^15 and a stage
-    // position below 2^17
-    if (C > 2048) return DF_ERR_UNSUPPORTED;
+    // the decoder's state word keeps a bit position below 2^14 and a stage
+    // position below 2^18
+    if (C > 1024) return DF_ERR_UNSUPPORTED;
     if (t->max_len < 1 || t->max_len > 32 || t->n_tables < 1) return DF_ERR_INVALID_ARG;
     if (t->n > DF_MAX_WEIGHTS) return DF_ERR_UNSUPPORTED;
     if (!t->stream || !t->gaps || !t->block_offsets || !t->sm || !t->lut) return DF_ERR_INVALID_ARG;

@@ -161,7 +161,7 @@ def table_walk_decode(stream, total_bits, n, gaps_fields, offsets, lut, n_tables
         win = window(p)
         e = int(wide[win >> (32 - WIDE)])
         step_word = e >> 32
-        used = step_word >> 17
+        used = step_word >> 18
         if used == 0:  # a code longer than the window: the 8-bit tables
             assert step_word == 0
             e = int(hier[win >> 24])
@@ -175,7 +175,7 @@ def table_walk_decode(stream, total_bits, n, gaps_fields, offsets, lut, n_tables
             out.append(e & 0xFF)
             return p + ((e >> 8) & 63), 1
         mask = int(masks[win >> (32 - WIDE)])
-        assert bin(mask).count("1") == step_word & ((1 << 17) - 1)
+        assert bin(mask).count("1") == step_word & ((1 << 18) - 1)
         lim = end - p if tail else WIDE
         starts = [i for i in range(WIDE) if (mask >> i) & 1 and i < lim]
         for k in range(len(starts)):
@@ -254,6 +254,6 @@ def test_unreachable_entries_are_zero():
     code = api.df_build_code(np.full(256, 7, dtype=np.uint64))
     lut = api.df_build_lut(code)
     wide = wide_entries(lut, WIDE)
-    assert ((wide >> np.uint64(32 + 17)) == 8).all()
+    assert ((wide >> np.uint64(32 + 18)) == 8).all()
     hier = lut[5 * (1 << WIDE) // 2:]
     assert (hier[:256] != 0).all()
