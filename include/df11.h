@@ -112,8 +112,8 @@ typedef struct df_batch_plan {
     uint32_t count;            /* tensors with n > 0                            */
     uint32_t threads_per_block;/* T, shared by all tensors (CUDA block size)    */
     uint32_t words_per_chunk;  /* shared-memory words per chunk (widest C)      */
-    uint32_t stage_bytes;      /* exponent stage of a block in shared memory    */
-    uint32_t reserved;
+    uint32_t region_bytes;     /* shared-memory exponent region of a thread     */
+    uint32_t max_groups;       /* 16-output groups a block may span             */
     uint32_t smem_bytes;       /* dynamic shared memory per CUDA block          */
     uint64_t total_blocks;     /* format blocks over all tensors                */
 } df_batch_plan;
@@ -231,10 +231,10 @@ df_status df_encode_noalloc(const df_code* code, const uint16_t* d_in, uint64_t 
  * 16-byte alignment of d_out and t->sm takes the vector path). A CUDA block
  * of T threads decodes one format block (T chunks) at a time: the wide table
  * and the block's stream slice are staged in shared memory, each thread
- * counts the codes that start in its chunk, a block scan turns the counts
- * into output positions, a second pass stores the exponents into a shared
- * stage in output order, and the block merges them with the sign|fraction
- * bytes into 16-byte stores. Source: mlx-dfloat, intro and "Status"
+ * decodes its chunk once into its own shared-memory region of exponents, a
+ * block scan turns the counts into output positions, and the block merges
+ * the exponents with the sign|fraction bytes in groups of 16 outputs
+ * (16-byte loads and stores). Chunks of up to 1024 bytes. Source: mlx-dfloat, intro and "Status"
  * (blockwise GPU decode back to identical bits); df11pack, "Use" (chunks).
  * Data errors set DF_EFLAG_* in d_err (nullable) and skip the affected
  * block's stores. Errors: DF_ERR_INVALID_ARG, DF_ERR_UNSUPPORTED (a layout

@@ -89,8 +89,8 @@ class DfBatchPlan(ctypes.Structure):
         ("count", ctypes.c_uint32),
         ("threads_per_block", ctypes.c_uint32),
         ("words_per_chunk", ctypes.c_uint32),
-        ("stage_bytes", ctypes.c_uint32),
-        ("reserved", ctypes.c_uint32),
+        ("region_bytes", ctypes.c_uint32),
+        ("max_groups", ctypes.c_uint32),
         ("smem_bytes", ctypes.c_uint32),
         ("total_blocks", ctypes.c_uint64),
     ]

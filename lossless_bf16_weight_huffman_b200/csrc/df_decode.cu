@@ -7,24 +7,25 @@
 //
 // One CUDA block of T threads handles one format block (T chunks of C stream
 // bytes) at a time and loops over the blocks of all tensors of the launch:
-//   1. when the tensor changes, stage its wide table (1024 entries indexed by
-//      10 stream bits: the exponents of the codes that lie wholly inside the
-//      window and one step word, (bits used << 18) | count, plus the codes'
-//      start masks) in shared memory; stage the
-//      block's stream slice, one chunk per thread, byte-swapped to big-endian
-//      words at an odd word stride (no bank conflicts between the threads'
-//      windows)
-//   2. count pass: each thread counts the codes that start in its chunk
-//      (from chunk start + gap up to the chunk end), up to 4 per table step;
-//      its state word (bit position << 18) | count advances by one add per
-//      step; codes longer than 10 bits walk the 8-bit-indexed tables
-//   3. block scan of the counts (warp shuffles + one shared array): each
-//      thread's first output position, checked against the block index
-//   4. write pass: each thread decodes its codes again and stores their
-//      exponents into a shared-memory stage in output order, placed so that
-//      stage index == output index mod 16
-//   5. merge: per group of 16 outputs, one 16-byte shared load of exponents,
-//      one 16-byte load of sign|fraction bytes, two 16-byte BF16 stores
+//   1. when the tensor changes, stage its wide table in shared memory (1024
+//      entries indexed by 10 stream bits: the exponents of the codes that lie
+//      wholly inside the window and one step word, (bits used << 18) | count);
+//      stage the block's stream slice, one chunk per thread, byte-swapped to
+//      big-endian words at an odd word stride (no bank conflicts between the
+//      threads' windows)
+//   2. one decode pass per thread over its chunk, from chunk start + gap to
+//      the chunk end: the state word (bit position << 18) | exponents so far
+//      advances by one add per table step (up to 4 codes); the exponents go
+//      to the thread's own word-aligned shared-memory region with 32-bit
+//      stores; codes longer than 10 bits walk the 8-bit-indexed tables
+//   3. block scan of the code counts (warp shuffles + one shared array): the
+//      first output position of every thread; checked against the block index
+//   4. an owner map: for every group of 16 outputs, the thread whose region
+//      holds its first exponent
+//   5. merge, in two loops: groups that lie in one region take their 16
+//      exponents from it; then each thread takes the one group, if any, that
+//      its range ends inside, gathering from its region and the next one(s).
+//      Per group: one 16-byte load of sign|fraction bytes, two 16-byte stores.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -71,7 +72,9 @@ struct BatchSrc {
 
 struct LaunchCfg {
     uint32_t words_per_chunk;  // shared-memory words of a chunk slot (odd)
-    uint32_t stage_bytes;      // exponent stage of a block
+    uint32_t region_bytes;     // exponent region of a thread (4 * odd)
+    uint32_t max_groups;       // owner-map entries
+    uint32_t pad;
     uint64_t total_blocks;
 };
 
@@ -112,6 +115,17 @@ __device__ __forceinline__ uint16_t merge1(uint8_t sm, uint8_t e) {
                                  (sm & 0x7Fu));
 }
 
+// 16 bytes of shared memory from byte address base + a (any alignment).
+__device__ __forceinline__ void gather16(const uint8_t* base, int a, uint32_t e[4]) {
+    const uint32_t* w = reinterpret_cast<const uint32_t*>(base + (a & ~3));
+    const uint32_t sh = 8 * (a & 3);
+    const uint32_t w0 = w[0], w1 = w[1], w2 = w[2], w3 = w[3], w4 = w[4];
+    e[0] = __funnelshift_r(w0, w1, sh);
+    e[1] = __funnelshift_r(w1, w2, sh);
+    e[2] = __funnelshift_r(w2, w3, sh);
+    e[3] = __funnelshift_r(w3, w4, sh);
+}
+
 // 4 BF16 weights from 4 sign|fraction bytes and 4 exponent bytes: the high
 // byte of weight k is s | e >> 1, the low byte (e & 1) << 7 | fraction.
 __device__ __forceinline__ void merge4(uint32_t s, uint32_t e, uint32_t* o0, uint32_t* o1) {
@@ -119,6 +133,18 @@ __device__ __forceinline__ void merge4(uint32_t s, uint32_t e, uint32_t* o0, uin
     const uint32_t lo = ((e << 7) & 0x80808080u) | (s & 0x7F7F7F7Fu);
     *o0 = __byte_perm(lo, hi, 0x5140);
     *o1 = __byte_perm(lo, hi, 0x7362);
+}
+
+// 16 outputs from their 16 sign|fraction bytes and 16 exponents: two 16-byte stores.
+__device__ __forceinline__ void merge16(const uint4 s16, const uint32_t e[4], uint16_t* __restrict__ dst16) {
+    uint32_t o[8];
+    merge4(s16.x, e[0], &o[0], &o[1]);
+    merge4(s16.y, e[1], &o[2], &o[3]);
+    merge4(s16.z, e[2], &o[4], &o[5]);
+    merge4(s16.w, e[3], &o[6], &o[7]);
+    uint4* dst = reinterpret_cast<uint4*>(dst16);
+    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
 // A code longer than the wide window, as a step word ((length << 18) | 1, or
@@ -129,122 +155,45 @@ __device__ __forceinline__ uint32_t long_step(uint32_t win, const uint32_t* hier
     return l ? (((l >> 8) & 63u) << kStepShift) | 1u : 0u;
 }
 
-// Count the codes that start in [p0, end). The state word is
-// (bit position << 18) | (codes so far); a table step adds its step word.
-// Sets *bad on a bit pattern no code starts with.
-__device__ __forceinline__ uint32_t count_codes(const uint32_t* words, uint32_t p0, uint32_t end,
-                                                const uint32_t* wide32, const uint16_t* wide_mask,
-                                                const uint32_t* hier, bool* bad) {
-    uint32_t st = p0 << kStepShift;
-    for (;;) {  // two whole windows per vote
-        const bool act = (st >> kStepShift) + 2 * kWideBits <= end;
-        if (!__any_sync(kFull, act)) break;
-        if (act) {
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const uint32_t win = window(words, st >> kStepShift);
-                uint32_t w = wide32[2 * (win >> (32 - kWideBits)) + 1];
-                if (w == 0) {
-                    uint32_t sym;
-                    w = long_step(win, hier, &sym);
-                    if (w == 0) {
-                        *bad = true;
-                        end = 0;
-                    }
-                }
-                st += w;
-                // a long code may have moved p past the second window
-                if (u == 0 && (st >> kStepShift) + kWideBits > end) break;
-            }
-        }
+// Decoder of one thread's chunk: state word (bit position << 18) | exponents
+// appended to the region; the exponents of the region word not yet stored
+// sit in acc (state & 3 of them).
+struct Lane {
+    uint32_t st;
+    uint32_t end;  // codes must start before this bit
+    uint64_t acc;
+    bool bad;
+};
+
+// Append the exponents of one step word to the region.
+__device__ __forceinline__ void append(Lane& L, uint32_t w, uint32_t sy, uint32_t* region) {
+    L.acc |= static_cast<uint64_t>(sy) << (8 * (L.st & 3u));
+    const uint32_t nst = L.st + w;
+    if ((nst ^ L.st) & (kStepCountMask & ~3u)) {  // a region word is complete
+        region[(L.st & kStepCountMask) >> 2] = static_cast<uint32_t>(L.acc);
+        L.acc >>= 32;
     }
-    for (;;) {  // windows that may reach past the end: count the codes starting before it
-        const uint32_t p = st >> kStepShift;
-        const bool act = p < end;
-        if (!__any_sync(kFull, act)) break;
-        if (act) {
-            const uint32_t win = window(words, p);
-            const uint32_t x = win >> (32 - kWideBits);
-            uint32_t w = wide32[2 * x + 1];
-            if (w == 0) {
-                uint32_t sym;
-                w = long_step(win, hier, &sym);
-                if (w == 0) {
-                    *bad = true;
-                    end = 0;
-                }
-            } else if (end - p < kWideBits) {
-                const uint32_t counted = __popc(wide_mask[x] & ((1u << (end - p)) - 1u));
-                w = (w & ~kStepCountMask) | counted;
-            }
-            st += w;
-        }
-    }
-    return st & kStepCountMask;
+    L.st = nst;
 }
 
-__device__ __forceinline__ void put4(uint8_t* a, uint32_t sy) {
-    a[0] = static_cast<uint8_t>(sy);
-    a[1] = static_cast<uint8_t>(sy >> 8);
-    a[2] = static_cast<uint8_t>(sy >> 16);
-    a[3] = static_cast<uint8_t>(sy >> 24);
-}
-
-// Store the exponents of the first `cnt` codes from bit p0 at stage[pos0...].
-// The state word is (bit position << 18) | (stage position). While 4 or more
-// codes remain, all 4 exponent slots of a step are stored (slots past its
-// codes are overwritten by the next step).
-__device__ __forceinline__ void write_codes(const uint32_t* words, uint32_t p0, uint32_t cnt, uint8_t* stage,
-                                            uint32_t pos0, const uint64_t* wide, const uint32_t* hier) {
-    uint32_t st = (p0 << kStepShift) | pos0;
-    uint32_t pend = pos0 + cnt;
-    for (;;) {  // two steps per vote
-        const bool act = (st & kStepCountMask) + 8 <= pend;
-        if (!__any_sync(kFull, act)) break;
-        if (act) {
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const uint32_t win = window(words, st >> kStepShift);
-                const uint64_t e = wide[win >> (32 - kWideBits)];
-                uint32_t sy = static_cast<uint32_t>(e);
-                uint32_t w = static_cast<uint32_t>(e >> 32);
-                if (w == 0) {
-                    w = long_step(win, hier, &sy);
-                    if (w == 0) pend = 0;  // cannot follow a clean count pass; never loop on it
-                }
-                put4(stage + (st & kStepCountMask), sy);
-                st += w;
-            }
+// One table step whose window lies before the chunk end.
+__device__ __forceinline__ void full_step(Lane& L, const uint32_t* words, const uint64_t* wide, const uint32_t* hier,
+                                          uint32_t* region) {
+    const uint32_t win = window(words, L.st >> kStepShift);
+    const uint64_t e = wide[win >> (32 - kWideBits)];
+    uint32_t sy = static_cast<uint32_t>(e);
+    uint32_t w = static_cast<uint32_t>(e >> 32);
+    if (w == 0) {
+        w = long_step(win, hier, &sy);
+        if (w == 0) {
+            L.bad = true;
+            L.end = 0;
         }
     }
-    for (;;) {
-        const uint32_t pos = st & kStepCountMask;
-        const bool act = pos < pend;
-        if (!__any_sync(kFull, act)) break;
-        if (act) {
-            const uint32_t win = window(words, st >> kStepShift);
-            const uint64_t e = wide[win >> (32 - kWideBits)];
-            uint32_t sy = static_cast<uint32_t>(e);
-            uint32_t w = static_cast<uint32_t>(e >> 32);
-            if (w == 0) {
-                w = long_step(win, hier, &sy);
-                if (w == 0) {
-                    pend = 0;
-                    continue;
-                }
-            }
-            const uint32_t k = min(w & kStepCountMask, pend - pos);
-            uint8_t* a = stage + pos;
-            a[0] = static_cast<uint8_t>(sy);
-            if (k > 1) a[1] = static_cast<uint8_t>(sy >> 8);
-            if (k > 2) a[2] = static_cast<uint8_t>(sy >> 16);
-            if (k > 3) a[3] = static_cast<uint8_t>(sy >> 24);
-            st += (w & ~kStepCountMask) | k;
-        }
-    }
+    append(L, w, sy, region);
 }
 
-template <class Src>
+template <class Src, class OwnerT>
 __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_constant__ Src src, const LaunchCfg cfg,
                                                              uint32_t* d_err) {
     extern __shared__ __align__(16) uint8_t smem[];
@@ -255,11 +204,14 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_consta
 
     // shared memory carve-up (sizes in smem_bytes())
     const uint64_t* s_wide = reinterpret_cast<const uint64_t*>(smem);
-    const uint16_t* s_mask = reinterpret_cast<const uint16_t*>(smem + 8 * kWideN);
-    uint32_t* s_words = reinterpret_cast<uint32_t*>(smem + 4 * kWideWords);
-    uint32_t* s_warp = s_words + ((T * cfg.words_per_chunk + 3) & ~3u);
+    uint32_t* s_words = reinterpret_cast<uint32_t*>(smem + 8 * kWideN);
+    uint32_t* s_pos = s_words + ((T * cfg.words_per_chunk + 3) & ~3u);
+    uint32_t* s_warp = s_pos + ((T + 1 + 3) & ~3u);
     uint32_t* s_hdr = s_warp + 32;  // 1 when the staged tables belong to the staged tensor
-    uint8_t* s_stage = reinterpret_cast<uint8_t*>(s_hdr + 4);
+    OwnerT* s_owner = reinterpret_cast<OwnerT*>(s_hdr + 4);
+    uint8_t* s_priv = reinterpret_cast<uint8_t*>(s_owner) + ((cfg.max_groups * sizeof(OwnerT) + 15) & ~15u);
+    const uint32_t RB = cfg.region_bytes;
+    uint32_t* my_region = reinterpret_cast<uint32_t*>(s_priv + tid * RB);
 
     const DevTensor* td = nullptr;
     const DevTensor* staged = nullptr;
@@ -272,10 +224,13 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_consta
         if (td != staged) {
             const uint4* t4 = reinterpret_cast<const uint4*>(td->lut);
             uint4* d4 = reinterpret_cast<uint4*>(smem);
-            for (uint32_t i = tid; i < kWideWords / 4; i += T) d4[i] = __ldg(t4 + i);
+            for (uint32_t i = tid; i < kWideEntryWords / 4; i += T) d4[i] = __ldg(t4 + i);
             if (tid == 0) {
                 const uint32_t* hdr = td->lut + kWideWords + static_cast<size_t>(td->n_tables) * 256 + 64;
-                s_hdr[0] = __ldg(hdr + 3) == kLutMagic && __ldg(hdr + 2) == td->n_tables && __ldg(hdr) >= 1;
+                const uint32_t minl = __ldg(hdr);
+                // the region must hold every code the tables can yield in one chunk
+                s_hdr[0] = __ldg(hdr + 3) == kLutMagic && __ldg(hdr + 2) == td->n_tables && minl >= 1 &&
+                           (8 * C + minl - 1) / minl + 12 <= RB;
             }
             staged = td;
         }
@@ -290,7 +245,11 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_consta
         const uint32_t wpc = C / 4 + 1;
         uint32_t* my_words = s_words + tid * wpc;
         const uint64_t chunk = b * T + tid;
-        uint32_t p0 = 0, end = 0;
+        Lane L;
+        L.st = 0;
+        L.end = 0;
+        L.acc = 0;
+        L.bad = false;
         if (chunk < td->n_chunks) {
             const uint4* c4 = reinterpret_cast<const uint4*>(td->stream + chunk * C);
             for (uint32_t k = 0; k < C / 16; ++k) {
@@ -307,11 +266,18 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_consta
             const uint32_t cbits = 8 * C;
             const uint64_t bit0 = chunk * cbits;
             const uint64_t rem = td->total_bits > bit0 ? td->total_bits - bit0 : 0;
-            p0 = (two >> (11 - (q & 7))) & 31u;
-            end = static_cast<uint32_t>(rem < cbits ? rem : cbits);
+            L.st = ((two >> (11 - (q & 7))) & 31u) << kStepShift;
+            L.end = static_cast<uint32_t>(rem < cbits ? rem : cbits);
         }
         const uint64_t out0 = td->offs[b];
         const uint64_t out1 = td->offs[b + 1];
+        if (tid == 0 && out0 <= out1 && out1 <= td->n) {  // warm L2 with the block's sign|fraction bytes
+            const uintptr_t lo = (reinterpret_cast<uintptr_t>(td->sm + out0) + 15) & ~static_cast<uintptr_t>(15);
+            const uintptr_t hi = reinterpret_cast<uintptr_t>(td->sm + out1) & ~static_cast<uintptr_t>(15);
+            if (hi > lo)
+                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(lo),
+                             "r"(static_cast<uint32_t>(hi - lo)) : "memory");
+        }
         __syncthreads();
         if (!s_hdr[0]) {  // tables that do not belong to this descriptor
             if (tid == 0 && d_err) atomicOr(d_err, DF_EFLAG_TABLES);
@@ -319,16 +285,53 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_consta
             continue;
         }
 
-        // 2. count pass
+        // 2. decode this thread's chunk into its region
         const uint32_t* hier = td->lut + kWideWords;
-        bool bad = false;
-        const uint32_t cnt = count_codes(my_words, p0, end, reinterpret_cast<const uint32_t*>(s_wide), s_mask, hier,
-                                         &bad);
+        for (;;) {  // two whole windows per vote
+            const bool act = (L.st >> kStepShift) + 2 * kWideBits <= L.end;
+            if (!__any_sync(kFull, act)) break;
+            if (act) {
+                full_step(L, my_words, s_wide, hier, my_region);
+                // a long code may have moved p past the second window
+                if ((L.st >> kStepShift) + kWideBits <= L.end) full_step(L, my_words, s_wide, hier, my_region);
+            }
+        }
+        uint32_t cnt = L.st & kStepCountMask;  // every code of a whole window starts before the end
+        for (;;) {  // windows that may reach past the end: count the codes starting before it
+            const uint32_t p = L.st >> kStepShift;
+            const bool act = p < L.end;
+            if (!__any_sync(kFull, act)) break;
+            if (act) {
+                const uint32_t win = window(my_words, p);
+                const uint32_t x = win >> (32 - kWideBits);
+                const uint64_t e = s_wide[x];
+                uint32_t sy = static_cast<uint32_t>(e);
+                uint32_t w = static_cast<uint32_t>(e >> 32);
+                uint32_t counted;
+                if (w == 0) {
+                    w = long_step(win, hier, &sy);
+                    counted = w & kStepCountMask;
+                    if (w == 0) {
+                        L.bad = true;
+                        L.end = 0;
+                    }
+                } else if (L.end - p < kWideBits) {
+                    const uint16_t* mask = reinterpret_cast<const uint16_t*>(td->lut + kWideEntryWords);
+                    counted = __popc(__ldg(mask + x) & ((1u << (L.end - p)) - 1u));
+                } else {
+                    counted = w & kStepCountMask;
+                }
+                append(L, w, sy, my_region);  // exponents past the end land in the region, uncounted
+                cnt += counted;
+            }
+        }
+        // the pending exponents (at most 3) complete the region
+        my_region[(L.st & kStepCountMask) >> 2] = static_cast<uint32_t>(L.acc);
 
         // 3. block scan of the counts: warp totals (with a corrupt-data bit)
         // in shared memory, then every warp scans them again on its own
         const uint32_t incl = warp_incl_scan(cnt, lane);
-        const bool warp_bad = __any_sync(kFull, bad);
+        const bool warp_bad = __any_sync(kFull, L.bad);
         if (lane == 31) s_warp[warp] = incl | (warp_bad ? 0x80000000u : 0u);
         __syncthreads();
         const uint32_t wv = lane < nwarps ? s_warp[lane] : 0u;
@@ -337,10 +340,13 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_consta
         const uint32_t wprefix = __shfl_sync(kFull, wincl - (wv & 0x7FFFFFFFu), warp);
         const uint32_t total = __shfl_sync(kFull, wincl, nwarps - 1);
         const uint32_t align = static_cast<uint32_t>(out0 & 15);
+        const uint32_t pos = align + wprefix + incl - cnt;
+        s_pos[tid] = pos;
+        if (tid == T - 1) s_pos[T] = pos + cnt;
 
         // consistency with the block index (uniform over the block)
         uint32_t flags = 0;
-        if (out1 < out0 || out1 > td->n || out1 - out0 + align + 16 > cfg.stage_bytes ||
+        if (out1 < out0 || out1 > td->n || (out1 - out0 + align + 15) / 16 > cfg.max_groups ||
             (b + 1 == td->n_blocks && out1 != td->n))
             flags |= DF_EFLAG_OFFSETS;
         else if (static_cast<uint64_t>(total) != out1 - out0)
@@ -352,32 +358,87 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_consta
             continue;
         }
 
-        // 4. write pass: exponents into the stage in output order
-        write_codes(my_words, p0, cnt, s_stage, align + wprefix + incl - cnt, s_wide, hier);
+        // 4. owner map: group gi (stage positions [16gi, 16gi+16)) belongs to
+        // the thread whose range holds max(16gi, align)
+        if (cnt) {
+            const uint32_t hi = pos + cnt;
+            if (pos <= align && align < hi) s_owner[0] = static_cast<OwnerT>(tid);
+            for (uint32_t gi = max((pos + 15) >> 4, 1u); 16 * gi < hi; ++gi) s_owner[gi] = static_cast<OwnerT>(tid);
+        }
         __syncthreads();
 
-        // 5. merge and store
+        // 5. merge and store; stage position c <-> output gbase + c
         const uint8_t* __restrict__ sm = td->sm;
         uint16_t* __restrict__ out = td->out;
-        const uint64_t gbase = out0 & ~15ull;  // stage index 0 <-> output gbase
-        const uint32_t ngroups = (align + total + 15) >> 4;
+        const uint64_t gbase = out0 & ~15ull;
+        const uint32_t vend = align + total;  // decoded stage positions are [align, vend)
+        const uint32_t ngroups = total ? (vend + 15) >> 4 : 0;  // a block may hold no code start
         const bool vec = td->vec_ok != 0;
-        for (uint32_t gi = tid; gi < ngroups; gi += T) {
-            const uint64_t G = gbase + 16ull * gi;
-            const uint4 e16 = *reinterpret_cast<const uint4*>(s_stage + 16 * gi);
-            if (vec && G >= out0 && G + 16 <= out1) {
-                const uint4 s16 = __ldg(reinterpret_cast<const uint4*>(sm + G));
-                uint32_t o[8];
-                merge4(s16.x, e16.x, &o[0], &o[1]);
-                merge4(s16.y, e16.y, &o[2], &o[3]);
-                merge4(s16.z, e16.z, &o[4], &o[5]);
-                merge4(s16.w, e16.w, &o[6], &o[7]);
-                uint4* dst = reinterpret_cast<uint4*>(out + G);
-                dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-                dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
-            } else {  // the groups at either end of the block, or unaligned buffers
-                const uint64_t lo = max(G, out0), hi = min(G + 16, out1);
-                for (uint64_t i = lo; i < hi; ++i) out[i] = merge1(sm[i], s_stage[i - gbase]);
+        // 5a. groups inside their owner's range; the others are left to 5b.
+        // Two groups per thread and iteration: both sign|fraction loads are
+        // in flight before the first merge.
+        for (uint32_t g0 = tid; g0 < ngroups; g0 += 2 * T) {
+            uint4 sv[2];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const uint32_t gi = g0 + k * T;
+                const uint64_t G = gbase + 16 * gi;
+                sv[k] = make_uint4(0, 0, 0, 0);
+                if (vec && gi < ngroups && G >= out0 && 16 * gi + 16 <= vend)
+                    sv[k] = __ldg(reinterpret_cast<const uint4*>(sm + G));
+            }
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const uint32_t gi = g0 + k * T;
+                if (gi >= ngroups) break;
+                const uint32_t c0 = 16 * gi;
+                const uint32_t t = s_owner[gi];
+                if (c0 + 16 > s_pos[t + 1]) continue;
+                const uint64_t G = gbase + c0;
+                uint32_t e[4];
+                gather16(s_priv, static_cast<int>(t * RB + c0) - static_cast<int>(s_pos[t]), e);
+                if (vec && G >= out0) {
+                    merge16(sv[k], e, out + G);
+                } else {  // the block's first group, or buffers without 16-byte alignment
+                    for (uint32_t q = 0; q < 16; ++q) {
+                        const uint64_t i = G + q;
+                        if (i >= out0) out[i] = merge1(sm[i], static_cast<uint8_t>(e[q >> 2] >> (8 * (q & 3))));
+                    }
+                }
+            }
+        }
+        // 5b. the group this thread's range ends inside, when it owns that
+        // group (then the group runs past the range, into later regions)
+        const uint32_t bend = pos + cnt;
+        if (cnt && (bend & 15) && s_owner[bend >> 4] == tid) {
+            const uint32_t c0 = bend & ~15u;
+            const uint64_t G = gbase + c0;
+            const uint32_t hi = min(c0 + 16, vend);
+            uint32_t e[4];
+            if (tid + 1 < T && hi <= s_pos[tid + 2]) {  // two regions: this one and the next
+                uint32_t x[4], y[4];
+                gather16(s_priv, static_cast<int>(tid * RB + c0) - static_cast<int>(pos), x);
+                gather16(s_priv, static_cast<int>((tid + 1) * RB) - static_cast<int>(bend - c0), y);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {  // bytes before bend from x, the rest from y
+                    const int sbits = 8 * static_cast<int>(bend - c0) - 32 * i;
+                    const uint32_t m = sbits >= 32 ? 0xFFFFFFFFu : (sbits <= 0 ? 0u : (1u << sbits) - 1u);
+                    e[i] = (x[i] & m) | (y[i] & ~m);
+                }
+            } else {  // three or more regions, or the last thread
+                e[0] = e[1] = e[2] = e[3] = 0;
+                uint32_t t = tid;
+                for (uint32_t c = max(c0, pos); c < hi; ++c) {
+                    while (c >= s_pos[t + 1]) ++t;
+                    e[(c - c0) >> 2] |= static_cast<uint32_t>(s_priv[t * RB + (c - s_pos[t])]) << (8 * ((c - c0) & 3));
+                }
+            }
+            const uint64_t lo_i = max(G, out0), hi_i = min(G + 16, out1);
+            if (vec && lo_i == G && hi_i == G + 16) {
+                merge16(__ldg(reinterpret_cast<const uint4*>(sm + G)), e, out + G);
+            } else {
+                for (uint64_t i = lo_i; i < hi_i; ++i)
+                    out[i] = merge1(sm[i], static_cast<uint8_t>(e[(i - G) >> 2] >> (8 * ((i - G) & 3))));
             }
         }
         __syncthreads();  // the next block overwrites shared memory
@@ -386,7 +447,7 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_consta
 
 struct Prepared {
     DevTensor dev;
-    uint32_t words_per_chunk, stage_bytes;
+    uint32_t words_per_chunk, region_bytes, max_groups;
 };
 
 uint32_t min_len_of(const uint8_t* lengths) {
@@ -403,9 +464,8 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 df_status prepare(const df_tensor* t, uint16_t* out, Prepared* pr) {
     if (!t || !out) return DF_ERR_INVALID_ARG;
     const uint32_t C = t->chunk_bytes, T = t->threads_per_block;
-    if (C < 16 || C > 4096 || C % 16 || T < 32 || T > 1024 || T % 32) return DF_ERR_INVALID_ARG;
-    // the decoder's state word keeps a bit position below 2^14 and a stage
-    // position below 2^18
+    if (C < 16 || C > 4096 || C % 16 || T < 32 || T > kMaxThreads || T % 32) return DF_ERR_INVALID_ARG;
+    // the state word keeps a bit position below 2^14 (C <= 1024 bytes)
     if (C > 1024) return DF_ERR_UNSUPPORTED;
     if (t->max_len < 1 || t->max_len > 32 || t->n_tables < 1) return DF_ERR_INVALID_ARG;
     if (t->n > DF_MAX_WEIGHTS) return DF_ERR_UNSUPPORTED;
@@ -438,20 +498,28 @@ df_status prepare(const df_tensor* t, uint16_t* out, Prepared* pr) {
     d.vec_ok = aligned(t->sm, 16) && aligned(out, 16);
     pr->dev = d;
     pr->words_per_chunk = C / 4 + 1;  // odd: C is a multiple of 16
-    // a block holds at most 8CT/min_len codes and never more than n; the
-    // stage also takes the alignment of the first output (< 16) and the
-    // 3 bytes a 4-byte exponent store may write past the last one
-    uint64_t per_block = (cbits * T + minl - 1) / (minl ? minl : 1);
+    // a chunk holds at most 8C/min_len code starts; its region also takes up
+    // to 3 exponents past the last counted code and the word they end in
+    const uint64_t per_chunk = (cbits + minl - 1) / (minl ? minl : 1);
+    uint64_t rb = (per_chunk + 12 + 3) & ~3ull;
+    if (((rb / 4) & 1) == 0) rb += 4;  // odd word stride: regions start in distinct banks
+    // a block holds at most 8CT/min_len codes and never more than n
+    uint64_t per_block = per_chunk * T;
     if (per_block > t->n) per_block = t->n;
-    const uint64_t stage = (per_block + 16 + 16 + 15) & ~15ull;
-    if (stage > (1u << kStepShift)) return DF_ERR_UNSUPPORTED;
-    pr->stage_bytes = static_cast<uint32_t>(stage);
+    const uint64_t groups = (per_block + 15 + 15) / 16 + 1;
+    if (rb > (1u << 20) || groups > 0xFFFFu) return DF_ERR_UNSUPPORTED;
+    pr->region_bytes = static_cast<uint32_t>(rb);
+    pr->max_groups = static_cast<uint32_t>(groups);
     return DF_OK;
 }
 
+// owner-map entries are bytes when a block has at most 256 threads
+size_t owner_size(uint32_t T) { return T <= 256 ? 1 : 2; }
+
 size_t smem_bytes(const LaunchCfg& c, uint32_t T) {
-    return 4u * kWideWords + ((static_cast<size_t>(T) * c.words_per_chunk + 3) & ~static_cast<size_t>(3)) * 4 +
-           32 * 4 + 16 + c.stage_bytes;
+    return 8u * kWideN + ((static_cast<size_t>(T) * c.words_per_chunk + 3) & ~static_cast<size_t>(3)) * 4 +
+           ((T + 1 + 3) & ~3u) * 4 + 32 * 4 + 16 + ((c.max_groups * owner_size(T) + 15) & ~static_cast<size_t>(15)) +
+           static_cast<size_t>(T) * c.region_bytes;
 }
 
 df_status device_limits(int* sms, int* max_smem) {
@@ -465,15 +533,14 @@ df_status device_limits(int* sms, int* max_smem) {
     return DF_OK;
 }
 
-template <class Src>
-df_status launch(const Src& src, const LaunchCfg& cfg, uint32_t T, size_t smem, uint32_t* d_err,
-                 cudaStream_t stream) {
-    if (cfg.total_blocks == 0) return DF_OK;
+template <class Src, class OwnerT>
+df_status launch_as(const Src& src, const LaunchCfg& cfg, uint32_t T, size_t smem, uint32_t* d_err,
+                    cudaStream_t stream) {
     int sms = 0, max_smem = 0;
     df_status st = device_limits(&sms, &max_smem);
     if (st != DF_OK) return st;
     if (smem > static_cast<size_t>(max_smem)) return DF_ERR_UNSUPPORTED;
-    auto kern = decode_kernel<Src>;
+    auto kern = decode_kernel<Src, OwnerT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return cuda_fail(e);
     int per_sm = 0;
@@ -489,9 +556,18 @@ df_status launch(const Src& src, const LaunchCfg& cfg, uint32_t T, size_t smem, 
     return DF_OK;
 }
 
+template <class Src>
+df_status launch(const Src& src, const LaunchCfg& cfg, uint32_t T, size_t smem, uint32_t* d_err,
+                 cudaStream_t stream) {
+    if (cfg.total_blocks == 0) return DF_OK;
+    return T <= 256 ? launch_as<Src, uint8_t>(src, cfg, T, smem, d_err, stream)
+                    : launch_as<Src, uint16_t>(src, cfg, T, smem, d_err, stream);
+}
+
 void widen(LaunchCfg* c, const Prepared& p) {
     c->words_per_chunk = std::max(c->words_per_chunk, p.words_per_chunk);
-    c->stage_bytes = std::max(c->stage_bytes, p.stage_bytes);
+    c->region_bytes = std::max(c->region_bytes, p.region_bytes);
+    c->max_groups = std::max(c->max_groups, p.max_groups);
 }
 
 }  // namespace
@@ -551,7 +627,8 @@ df_status df_decode_batch_prepare(const df_tensor* tensors, uint16_t* const* d_o
     plan->count = static_cast<uint32_t>(dev.size());
     plan->threads_per_block = T;
     plan->words_per_chunk = cfg.words_per_chunk;
-    plan->stage_bytes = cfg.stage_bytes;
+    plan->region_bytes = cfg.region_bytes;
+    plan->max_groups = cfg.max_groups;
     plan->total_blocks = start.back();
     if (plan->count == 0) return DF_OK;
     const size_t sm = smem_bytes(cfg, T);
@@ -585,7 +662,8 @@ df_status df_decode_batch_run(const df_batch_plan* plan, uint32_t* d_err, void* 
     LaunchCfg cfg;
     std::memset(&cfg, 0, sizeof(cfg));
     cfg.words_per_chunk = plan->words_per_chunk;
-    cfg.stage_bytes = plan->stage_bytes;
+    cfg.region_bytes = plan->region_bytes;
+    cfg.max_groups = plan->max_groups;
     cfg.total_blocks = plan->total_blocks;
     if (smem_bytes(cfg, plan->threads_per_block) != plan->smem_bytes) return DF_ERR_INVALID_ARG;
     return launch(src, cfg, plan->threads_per_block, plan->smem_bytes, d_err, static_cast<cudaStream_t>(stream));
