@@ -9,15 +9,16 @@
 // bytes) at a time and loops over the blocks of all tensors of the launch:
 //   1. when the tensor changes, stage its wide table in shared memory (1024
 //      entries indexed by 10 stream bits: the exponents of the codes that lie
-//      wholly inside the window and one step word, (bits used << 18) | count);
+//      wholly inside the window and one step word, (bits used << 18) |
+//      (count << 3));
 //      stage the block's stream slice, one chunk per thread, byte-swapped to
 //      big-endian words at an odd word stride (no bank conflicts between the
 //      threads' windows)
 //   2. one decode pass per thread over its chunk, from chunk start + gap to
-//      the chunk end: the state word (bit position << 18) | exponents so far
-//      advances by one add per table step (up to 4 codes); the exponents go
-//      to the thread's own word-aligned shared-memory region with 32-bit
-//      stores; codes longer than 10 bits walk the 8-bit-indexed tables
+//      the chunk end: the state word (bit position << 18) | (exponents so
+//      far << 3) advances by one add per table step (up to 4 codes); the
+//      exponents go to the thread's own word-aligned shared-memory region
+//      with 32-bit stores; codes longer than 10 bits walk the 8-bit tables
 //   3. block scan of the code counts (warp shuffles + one shared array): the
 //      first output position of every thread; checked against the block index
 //   4. an owner map: for every group of 16 outputs, the thread whose region
@@ -147,31 +148,34 @@ __device__ __forceinline__ void merge16(const uint4 s16, const uint32_t e[4], ui
     dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
-// A code longer than the wide window, as a step word ((length << 18) | 1, or
-// 0 for a bit pattern no code starts with) and its exponent.
+// A code longer than the wide window, as a step word ((length << 18) | 1 << 3,
+// or 0 for a bit pattern no code starts with) and its exponent.
 __device__ __forceinline__ uint32_t long_step(uint32_t win, const uint32_t* hier, uint32_t* sym) {
     const uint32_t l = long_code(win, hier);
     *sym = l & 0xFFu;
-    return l ? (((l >> 8) & 63u) << kStepShift) | 1u : 0u;
+    return l ? (((l >> 8) & 63u) << kStepShift) | (1u << kStepCountShift) : 0u;
 }
 
-// Decoder of one thread's chunk: state word (bit position << 18) | exponents
-// appended to the region; the exponents of the region word not yet stored
-// sit in acc (state & 3 of them).
+// Decoder of one thread's chunk: state word (bit position << 18) |
+// (exponents appended to the region << 3); the exponents of the region word
+// not yet stored sit in the low bytes of acc ((state & 24) / 8 of them).
 struct Lane {
     uint32_t st;
     uint32_t end;  // codes must start before this bit
-    uint64_t acc;
+    uint32_t acc;
     bool bad;
 };
 
 // Append the exponents of one step word to the region.
 __device__ __forceinline__ void append(Lane& L, uint32_t w, uint32_t sy, uint32_t* region) {
-    L.acc |= static_cast<uint64_t>(sy) << (8 * (L.st & 3u));
+    const uint32_t sh = L.st & 24u;
+    const uint32_t lo = L.acc | (sy << sh);
     const uint32_t nst = L.st + w;
-    if ((nst ^ L.st) & (kStepCountMask & ~3u)) {  // a region word is complete
-        region[(L.st & kStepCountMask) >> 2] = static_cast<uint32_t>(L.acc);
-        L.acc >>= 32;
+    if ((nst ^ L.st) & (kStepCountMask & ~31u)) {  // a region word is complete
+        region[(L.st & kStepCountMask) >> 5] = lo;
+        L.acc = __funnelshift_rc(sy, 0u, 32u - sh);  // the bytes past it (none when sh = 0)
+    } else {
+        L.acc = lo;
     }
     L.st = nst;
 }
@@ -296,7 +300,7 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_consta
                 if ((L.st >> kStepShift) + kWideBits <= L.end) full_step(L, my_words, s_wide, hier, my_region);
             }
         }
-        uint32_t cnt = L.st & kStepCountMask;  // every code of a whole window starts before the end
+        uint32_t cnt = (L.st & kStepCountMask) >> kStepCountShift;  // codes of whole windows start before the end
         for (;;) {  // windows that may reach past the end: count the codes starting before it
             const uint32_t p = L.st >> kStepShift;
             const bool act = p < L.end;
@@ -310,7 +314,7 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_consta
                 uint32_t counted;
                 if (w == 0) {
                     w = long_step(win, hier, &sy);
-                    counted = w & kStepCountMask;
+                    counted = (w & kStepCountMask) >> kStepCountShift;
                     if (w == 0) {
                         L.bad = true;
                         L.end = 0;
@@ -319,14 +323,14 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_consta
                     const uint16_t* mask = reinterpret_cast<const uint16_t*>(td->lut + kWideEntryWords);
                     counted = __popc(__ldg(mask + x) & ((1u << (L.end - p)) - 1u));
                 } else {
-                    counted = w & kStepCountMask;
+                    counted = (w & kStepCountMask) >> kStepCountShift;
                 }
                 append(L, w, sy, my_region);  // exponents past the end land in the region, uncounted
                 cnt += counted;
             }
         }
         // the pending exponents (at most 3) complete the region
-        my_region[(L.st & kStepCountMask) >> 2] = static_cast<uint32_t>(L.acc);
+        my_region[(L.st & kStepCountMask) >> 5] = L.acc;
 
         // 3. block scan of the counts: warp totals (with a corrupt-data bit)
         // in shared memory, then every warp scans them again on its own

@@ -243,7 +243,7 @@ df_status df_build_lut(const df_code* code, uint32_t* lut, size_t lut_words) {
             used += l;
             ++n;
         }
-        const uint32_t step = used ? (used << kStepShift) | n : 0u;
+        const uint32_t step = used ? (used << kStepShift) | (n << kStepCountShift) : 0u;
         wide[x] = syms | (static_cast<uint64_t>(step) << 32);
         wide_mask[x] = static_cast<uint16_t>(mask);
     }

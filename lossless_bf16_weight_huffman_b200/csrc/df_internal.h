@@ -31,9 +31,11 @@ struct DevTensor {
 //   wide table, 1024 uint64 indexed by the next kWideBits = 10 stream bits:
 //     bits 0-31  the exponents of the codes that lie wholly inside the window,
 //                taken from its first bit on (at most 4; first in bits 0-7)
-//     bits 32-63 (bits used << 18) | (how many codes); 0 when the first code
-//                is longer than the window. A decoder whose state word is
-//                (bit position << 18) | (codes so far) advances by one add.
+//     bits 32-63 (bits used << 18) | (how many codes << 3); 0 when the first
+//                code is longer than the window. A decoder whose state word is
+//                (bit position << 18) | (codes so far << 3) advances by one
+//                add, and (state & 24) is the byte shift of the next exponent
+//                within a 32-bit word.
 //   wide start masks, 1024 uint16: bit i set when one of those codes starts
 //     at window bit i
 //   8-bit-indexed tables for codes of any length (root + next levels):
@@ -46,6 +48,7 @@ constexpr uint32_t kWideBits = 10;
 constexpr uint32_t kWideMaxCodes = 4;
 constexpr uint32_t kStepShift = 18;                     // bits-used field of a step word
 constexpr uint32_t kStepCountMask = (1u << kStepShift) - 1;
+constexpr uint32_t kStepCountShift = 3;                 // the count field holds count << 3
 constexpr uint32_t kWideEntryWords = 2u << kWideBits;   // the uint64 entries
 constexpr uint32_t kWideMaskWords = (1u << kWideBits) / 2;
 constexpr uint32_t kWideWords = kWideEntryWords + kWideMaskWords;

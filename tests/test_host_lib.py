@@ -175,7 +175,7 @@ def table_walk_decode(stream, total_bits, n, gaps_fields, offsets, lut, n_tables
             out.append(e & 0xFF)
             return p + ((e >> 8) & 63), 1
         mask = int(masks[win >> (32 - WIDE)])
-        assert bin(mask).count("1") == step_word & ((1 << 18) - 1)
+        assert bin(mask).count("1") << 3 == step_word & ((1 << 18) - 1)
         lim = end - p if tail else WIDE
         starts = [i for i in range(WIDE) if (mask >> i) & 1 and i < lim]
         for k in range(len(starts)):
