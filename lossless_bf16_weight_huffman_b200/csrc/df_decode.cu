@@ -6,7 +6,8 @@
 // The layout of the work below is this library's own, written for sm_100a.
 //
 // One CUDA block of T threads handles one format block (T chunks of C stream
-// bytes) at a time and loops over the blocks of all tensors of the launch:
+// bytes) at a time and loops over a contiguous range of the format blocks of
+// all tensors of the launch (persistent blocks, one range each):
 //   1. when the tensor changes, stage its wide table in shared memory (1024
 //      entries indexed by 10 stream bits: the exponents of the codes that lie
 //      wholly inside the window and one step word, (bits used << 18) |
@@ -220,7 +221,12 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_consta
     const DevTensor* td = nullptr;
     const DevTensor* staged = nullptr;
     uint64_t t_lo = 0, t_hi = 0;
-    for (uint64_t g = blockIdx.x; g < cfg.total_blocks; g += gridDim.x) {
+    // each CUDA block takes a contiguous range of format blocks, so that it
+    // changes tensors (and restages tables) as rarely as possible
+    const uint64_t per = cfg.total_blocks / gridDim.x, extra = cfg.total_blocks % gridDim.x;
+    const uint64_t g_begin = blockIdx.x * per + min(static_cast<uint64_t>(blockIdx.x), extra);
+    const uint64_t g_end = g_begin + per + (blockIdx.x < extra ? 1 : 0);
+    for (uint64_t g = g_begin; g < g_end; ++g) {
         if (g < t_lo || g >= t_hi) td = src.find(g, &t_lo, &t_hi);
         const uint64_t b = g - t_lo;
         const uint32_t C = td->chunk_bytes;
@@ -238,9 +244,9 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_consta
             }
             staged = td;
         }
-        // warm L2 with the stream slice of this slot's next block of the same tensor
-        const uint64_t g_next = g + gridDim.x;
-        if (tid == 0 && g_next < t_hi) {
+        // warm L2 with the stream slice of the next block of the same tensor
+        const uint64_t g_next = g + 1;
+        if (tid == 0 && g_next < t_hi && g_next < g_end) {
             const uint64_t s0 = (g_next - t_lo) * T * C;
             const uint64_t s_bytes = min(static_cast<uint64_t>(T) * C + 16, td->n_chunks * C + 16 - s0);
             asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(td->stream + s0),
