@@ -213,13 +213,17 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_consta
     uint32_t* s_pos = s_words + ((T * cfg.words_per_chunk + 3) & ~3u);
     uint32_t* s_warp = s_pos + ((T + 1 + 3) & ~3u);
     uint32_t* s_hdr = s_warp + 32;  // 1 when the staged tables belong to the staged tensor
-    OwnerT* s_owner = reinterpret_cast<OwnerT*>(s_hdr + 4);
+    // the current tensor's descriptor: copied here on a tensor switch, because
+    // the merge's streaming loads keep evicting it from L1
+    DevTensor* s_td = reinterpret_cast<DevTensor*>(s_hdr + 4);
+    OwnerT* s_owner = reinterpret_cast<OwnerT*>(reinterpret_cast<uint8_t*>(s_td) + sizeof(DevTensor));
     uint8_t* s_priv = reinterpret_cast<uint8_t*>(s_owner) + ((cfg.max_groups * sizeof(OwnerT) + 15) & ~15u);
     const uint32_t RB = cfg.region_bytes;
     uint32_t* my_region = reinterpret_cast<uint32_t*>(s_priv + tid * RB);
 
-    const DevTensor* td = nullptr;
+    const DevTensor* tg = nullptr;      // the current tensor's descriptor in global memory
     const DevTensor* staged = nullptr;
+    const DevTensor* const td = s_td;  // read through its shared-memory copy
     uint64_t t_lo = 0, t_hi = 0;
     // each CUDA block takes a contiguous range of format blocks, so that it
     // changes tensors (and restages tables) as rarely as possible
@@ -227,11 +231,13 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_consta
     const uint64_t g_begin = blockIdx.x * per + min(static_cast<uint64_t>(blockIdx.x), extra);
     const uint64_t g_end = g_begin + per + (blockIdx.x < extra ? 1 : 0);
     for (uint64_t g = g_begin; g < g_end; ++g) {
-        if (g < t_lo || g >= t_hi) td = src.find(g, &t_lo, &t_hi);
+        if (g < t_lo || g >= t_hi) tg = src.find(g, &t_lo, &t_hi);
         const uint64_t b = g - t_lo;
-        const uint32_t C = td->chunk_bytes;
-        // 1. tables (when the tensor changes) and the stream slice
-        if (td != staged) {
+        // 1. descriptor and tables (when the tensor changes) and the stream slice
+        if (tg != staged) {
+            if (tid < sizeof(DevTensor) / 4)
+                reinterpret_cast<uint32_t*>(s_td)[tid] = reinterpret_cast<const uint32_t*>(tg)[tid];
+            __syncthreads();
             const uint4* t4 = reinterpret_cast<const uint4*>(td->lut);
             uint4* d4 = reinterpret_cast<uint4*>(smem);
             for (uint32_t i = tid; i < kWideEntryWords / 4; i += T) d4[i] = __ldg(t4 + i);
@@ -240,10 +246,11 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_consta
                 const uint32_t minl = __ldg(hdr);
                 // the region must hold every code the tables can yield in one chunk
                 s_hdr[0] = __ldg(hdr + 3) == kLutMagic && __ldg(hdr + 2) == td->n_tables && minl >= 1 &&
-                           (8 * C + minl - 1) / minl + 12 <= RB;
+                           (8 * td->chunk_bytes + minl - 1) / minl + 12 <= RB;
             }
-            staged = td;
+            staged = tg;
         }
+        const uint32_t C = td->chunk_bytes;
         // warm L2 with the stream slice of the next block of the same tensor
         const uint64_t g_next = g + 1;
         if (tid == 0 && g_next < t_hi && g_next < g_end) {
@@ -528,7 +535,7 @@ size_t owner_size(uint32_t T) { return T <= 256 ? 1 : 2; }
 
 size_t smem_bytes(const LaunchCfg& c, uint32_t T) {
     return 8u * kWideN + ((static_cast<size_t>(T) * c.words_per_chunk + 3) & ~static_cast<size_t>(3)) * 4 +
-           ((T + 1 + 3) & ~3u) * 4 + 32 * 4 + 16 + ((c.max_groups * owner_size(T) + 15) & ~static_cast<size_t>(15)) +
+           ((T + 1 + 3) & ~3u) * 4 + 32 * 4 + 16 + sizeof(DevTensor) + ((c.max_groups * owner_size(T) + 15) & ~static_cast<size_t>(15)) +
            static_cast<size_t>(T) * c.region_bytes;
 }
 

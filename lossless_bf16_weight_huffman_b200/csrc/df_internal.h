@@ -26,6 +26,7 @@ struct DevTensor {
     uint32_t vec_ok;       // sm and out 16-byte aligned
     uint32_t pad;
 };
+static_assert(sizeof(DevTensor) % 16 == 0, "descriptors are copied and placed in 16-byte units");
 
 // Decode tables (the words df_build_lut writes), in order:
 //   wide table, 1024 uint64 indexed by the next kWideBits = 10 stream bits:
