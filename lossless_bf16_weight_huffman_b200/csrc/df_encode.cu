@@ -8,12 +8,11 @@
 // bits, C-byte chunks with 5-bit start gaps, per-block output offsets) is the
 // one df11.h defines.
 //
-// Tiles of 4096 weights: 8 warps x 16 steps x 32 lanes. In a step each lane
-// holds one weight's code; a warp shuffle scan gives each code its bit
-// offset, and every 32-bit stream word the step touches is assembled with one
-// warp OR-reduction. Words inside a warp's range are written whole; the first
-// and last word of a warp's range (shared with its neighbours) are OR-ed in
-// atomically into the zeroed stream.
+// Tiles of 4096 weights, 256 threads x 16 consecutive weights: a block scan of
+// the threads' code-length sums gives every code its bit offset; the tile's
+// stream words are assembled in shared memory and stored whole, except the two
+// edge words a tile shares with its neighbours, which are OR-ed atomically into
+// the zeroed stream.
 #include <cuda_runtime.h>
 
 #include <cstring>
@@ -160,6 +159,8 @@ struct PackArgs {
     uint32_t chunk_bits;
     uint32_t threads_per_block;
     uint32_t* err;
+    uint32_t in_vec;  // input 16-byte aligned
+    uint32_t sm_vec;  // sign|fraction output 16-byte aligned
 };
 
 __device__ __forceinline__ void or_gap(uint32_t* gaps32, uint64_t j, uint32_t g) {
@@ -174,100 +175,129 @@ __device__ __forceinline__ void or_gap(uint32_t* gaps32, uint64_t j, uint32_t g)
     }
 }
 
-// This lane's bits of stream word W: the code occupies [ls, ls+l).
-__device__ __forceinline__ uint32_t word_part(uint64_t ls, uint32_t l, uint32_t code, uint64_t W) {
-    const uint64_t w0 = 32 * W;
-    if (l == 0 || ls >= w0 + 32 || ls + l <= w0) return 0;
-    const uint64_t v = static_cast<uint64_t>(code) << (64 - l);
-    if (ls >= w0) return static_cast<uint32_t>(v >> (32 + (ls - w0)));
-    return static_cast<uint32_t>((v << (w0 - ls)) >> 32);
-}
+// One tile of 4096 weights per CUDA block, 16 consecutive weights per thread.
+// A block scan of the threads' code-length sums gives every code its bit
+// offset; the codes are OR-ed into the tile's words in shared memory (shared
+// atomics: neighbouring threads may share a word), then the words go out with
+// coalesced stores, byte-swapped to MSB-first order. The first and last word
+// of a tile may hold bits of the neighbouring tiles: those are OR-ed into the
+// zeroed stream atomically. The code that crosses or ends on a chunk boundary
+// writes that chunk's gap (and, at a block boundary, the block offset).
+constexpr uint32_t kPerThread = kTile / kEncThreads;  // 16 weights
 
 __global__ void __launch_bounds__(kEncThreads) pack_kernel(PackArgs a, EncTables tab) {
     __shared__ uint32_t s_code[256];
     __shared__ uint8_t s_len[256];
-    __shared__ uint64_t s_wsum[kEncThreads / 32];
-    for (uint32_t i = threadIdx.x; i < 256; i += blockDim.x) {
+    __shared__ uint32_t s_warp[kEncThreads / 32];
+    __shared__ uint32_t s_words[kTile + 2];  // a tile holds at most 4096 codes of at most 32 bits
+    const uint32_t tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (uint32_t i = tid; i < 256; i += kEncThreads) {
         s_code[i] = tab.codes[i];
         s_len[i] = tab.lengths[i];
     }
-    __syncthreads();
-    const uint32_t lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const uint64_t wbase = static_cast<uint64_t>(blockIdx.x) * kTile + warp * (kSteps * 32);
-
-    // bits of this warp's 512 weights
-    uint32_t mine = 0;
-#pragma unroll 4
-    for (uint32_t s = 0; s < kSteps; ++s) {
-        const uint64_t i = wbase + s * 32 + lane;
-        if (i < a.n) mine += s_len[(__ldg(a.in + i) >> 7) & 0xFFu];
-    }
+    const uint64_t i0 = static_cast<uint64_t>(blockIdx.x) * kTile + tid * kPerThread;
+    // this thread's 16 weights (two pairs per 32-bit word)
+    uint32_t wv[kPerThread / 2];
+    const bool full = i0 + kPerThread <= a.n;
+    if (full && a.in_vec) {
+        const uint4* p4 = reinterpret_cast<const uint4*>(a.in + i0);
+        const uint4 v0 = __ldg(p4), v1 = __ldg(p4 + 1);
+        wv[0] = v0.x; wv[1] = v0.y; wv[2] = v0.z; wv[3] = v0.w;
+        wv[4] = v1.x; wv[5] = v1.y; wv[6] = v1.z; wv[7] = v1.w;
+    } else {
 #pragma unroll
-    for (int d = 16; d > 0; d >>= 1) mine += __shfl_xor_sync(0xFFFFFFFFu, mine, d);
-    if (lane == 0) s_wsum[warp] = mine;
-    __syncthreads();
-    uint64_t pos = a.tile_base[blockIdx.x];
-    for (uint32_t w = 0; w < warp; ++w) pos += s_wsum[w];
-    if (s_wsum[warp] == 0) return;  // nothing of this warp's range is in the tensor
-
-    const uint64_t first_word = pos >> 5;
-    uint64_t cur_word = first_word;
-    uint32_t carry = 0;
-    for (uint32_t s = 0; s < kSteps; ++s) {
-        const uint64_t i = wbase + s * 32 + lane;
-        uint32_t l = 0, code = 0;
-        if (i < a.n) {
-            const uint16_t x = __ldg(a.in + i);
-            const uint32_t e = (x >> 7) & 0xFFu;
-            l = s_len[e];
-            code = s_code[e];
-            a.sm[i] = static_cast<uint8_t>(((x >> 8) & 0x80u) | (x & 0x7Fu));
+        for (uint32_t k = 0; k < kPerThread / 2; ++k) {
+            const uint64_t i = i0 + 2 * k;
+            const uint32_t lo = i < a.n ? __ldg(a.in + i) : 0u;
+            const uint32_t hi = i + 1 < a.n ? __ldg(a.in + i + 1) : 0u;
+            wv[k] = lo | (hi << 16);
         }
-        uint32_t incl = l;
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            const uint32_t u = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-            if (lane >= static_cast<uint32_t>(d)) incl += u;
-        }
-        const uint32_t step_bits = __shfl_sync(0xFFFFFFFFu, incl, 31);
-        const uint64_t ls = pos + incl - l;
-        // chunk index: the code that crosses (or ends on) a chunk boundary owns it
-        if (l) {
-            const uint64_t le = ls + l;
-            const uint64_t j = le / a.chunk_bits;
-            if (j > ls / a.chunk_bits && j < a.n_chunks) {
-                or_gap(a.gaps32, j, static_cast<uint32_t>(le - j * a.chunk_bits));
-                if (j % a.threads_per_block == 0) a.offsets[j / a.threads_per_block] = i + 1;
-            }
-        }
-        if (step_bits) {
-            const uint64_t fw = pos >> 5, lw = (pos + step_bits - 1) >> 5;
-            for (uint64_t W = fw; W <= lw; ++W) {
-                const uint32_t word = __reduce_or_sync(0xFFFFFFFFu, word_part(ls, l, code, W));
-                if (W == cur_word) {
-                    carry |= word;
-                } else {
-                    if (lane == 0) {
-                        if (cur_word >= a.stream_words) {
-                            if (a.err) atomicOr(a.err, DF_EFLAG_ENC_TOTAL);
-                        } else if (cur_word == first_word) {
-                            atomicOr(a.stream32 + cur_word, bswap32(carry));
-                        } else {
-                            a.stream32[cur_word] = bswap32(carry);
-                        }
-                    }
-                    cur_word = W;
-                    carry = word;
-                }
-            }
-        }
-        pos += step_bits;
     }
-    if (lane == 0) {
-        if (cur_word < a.stream_words)
-            atomicOr(a.stream32 + cur_word, bswap32(carry));
-        else if (a.err)
-            atomicOr(a.err, DF_EFLAG_ENC_TOTAL);
+    const uint32_t cnt = full ? kPerThread : (i0 < a.n ? static_cast<uint32_t>(a.n - i0) : 0u);
+    // sign|fraction bytes
+    uint32_t smw[kPerThread / 4];
+#pragma unroll
+    for (uint32_t k = 0; k < kPerThread / 4; ++k) {
+        const uint32_t x = wv[2 * k], y = wv[2 * k + 1];
+        // byte j of the word: (w >> 8 & 0x80) | (w & 0x7F) of weight 4k + j
+        const uint32_t hi = __byte_perm(x, y, 0x7531) & 0x80808080u;
+        const uint32_t lo = __byte_perm(x, y, 0x6420) & 0x7F7F7F7Fu;
+        smw[k] = hi | lo;
+    }
+    if (full && a.sm_vec) {
+        *reinterpret_cast<uint4*>(a.sm + i0) = make_uint4(smw[0], smw[1], smw[2], smw[3]);
+    } else {
+        for (uint32_t k = 0; k < cnt; ++k) a.sm[i0 + k] = static_cast<uint8_t>(smw[k >> 2] >> (8 * (k & 3)));
+    }
+    __syncthreads();  // the code tables
+    uint32_t sum = 0;
+#pragma unroll
+    for (uint32_t k = 0; k < kPerThread; ++k) {
+        const uint32_t e = (wv[k >> 1] >> (16 * (k & 1) + 7)) & 0xFFu;
+        sum += k < cnt ? s_len[e] : 0u;
+    }
+    // block scan of the sums
+    uint32_t incl = sum;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const uint32_t u = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+        if (lane >= static_cast<uint32_t>(d)) incl += u;
+    }
+    if (lane == 31) s_warp[warp] = incl;
+    const uint64_t tile_bit0 = a.tile_base[blockIdx.x];
+    const uint32_t head = static_cast<uint32_t>(tile_bit0 & 31);  // bits of the first word before the tile
+    __syncthreads();
+    uint32_t wprefix = 0, total = 0;
+#pragma unroll
+    for (uint32_t w = 0; w < kEncThreads / 32; ++w) {
+        const uint32_t t = s_warp[w];
+        wprefix += w < warp ? t : 0u;
+        total += t;
+    }
+    const uint32_t nw = (head + total + 31) >> 5;  // words the tile touches
+    for (uint32_t k = tid; k < nw; k += kEncThreads) s_words[k] = 0;
+    __syncthreads();
+    // OR the codes into the tile's words (bit q of the tile -> bit 31 - q % 32 of word q / 32)
+    const uint32_t off = wprefix + incl - sum;  // this thread's first bit within the tile
+    uint32_t lp = head + off;
+    uint64_t gb = tile_bit0 + off;  // ... and in the stream
+    // the first chunk boundary after gb, and its chunk index
+    uint64_t jn = gb / a.chunk_bits + 1;
+    uint64_t nb = jn * a.chunk_bits;
+#pragma unroll
+    for (uint32_t k = 0; k < kPerThread; ++k) {
+        if (k >= cnt) break;
+        const uint32_t e = (wv[k >> 1] >> (16 * (k & 1) + 7)) & 0xFFu;
+        const uint32_t l = s_len[e];
+        if (l == 0) continue;
+        const uint32_t v = s_code[e] << (32 - l);  // the code, left-aligned
+        const uint32_t sh = lp & 31;
+        atomicOr(&s_words[lp >> 5], v >> sh);
+        if (sh + l > 32) atomicOr(&s_words[(lp >> 5) + 1], v << (32 - sh));
+        lp += l;
+        gb += l;
+        if (gb >= nb) {  // this code crosses or ends on chunk boundary nb: the next start is gb
+            if (jn < a.n_chunks) {
+                or_gap(a.gaps32, jn, static_cast<uint32_t>(gb - nb));
+                if (jn % a.threads_per_block == 0) a.offsets[jn / a.threads_per_block] = i0 + k + 1;
+            }
+            ++jn;
+            nb += a.chunk_bits;
+        }
+    }
+    __syncthreads();
+    // out: whole words inside the tile are stored, the two edge words OR-ed in
+    const uint64_t w0 = tile_bit0 >> 5;
+    for (uint32_t k = tid; k < nw; k += kEncThreads) {
+        const uint64_t W = w0 + k;
+        const uint32_t val = bswap32(s_words[k]);
+        if (W >= a.stream_words) {
+            if (a.err) atomicOr(a.err, DF_EFLAG_ENC_TOTAL);
+        } else if (k == 0 || k + 1 == nw) {
+            if (val) atomicOr(a.stream32 + W, val);
+        } else {
+            a.stream32[W] = val;
+        }
     }
 }
 
@@ -389,6 +419,8 @@ df_status df_encode(const df_code* code, const uint16_t* d_in, uint64_t n, uint6
     a.err = d_err;
     a.chunk_bits = static_cast<uint32_t>(cbits);
     a.threads_per_block = tpb;
+    a.in_vec = aligned(d_in, 16) ? 1u : 0u;
+    a.sm_vec = aligned(d_sm, 16) ? 1u : 0u;
     pack_kernel<<<static_cast<unsigned>(tiles), kEncThreads, 0, s>>>(a, tab);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e);
