@@ -25,7 +25,7 @@ namespace {
 
 constexpr uint32_t kTile = 4096;
 constexpr uint32_t kEncThreads = 256;
-constexpr uint32_t kSteps = kTile / kEncThreads;  // 16 steps of 32 weights per warp
+constexpr uint32_t kPerThread = kTile / kEncThreads;  // 16 consecutive weights per thread
 
 __device__ __forceinline__ uint32_t bswap32(uint32_t x) { return __byte_perm(x, 0, 0x0123); }
 
@@ -67,22 +67,39 @@ struct EncTables {
     uint8_t lengths[256];
 };
 
-// Sum of code lengths of each tile of 4096 weights.
+// Sum of code lengths of each tile of 4096 weights (16 consecutive weights per
+// thread, as the packer reads them).
 __global__ void __launch_bounds__(kEncThreads) tile_bits_kernel(const uint16_t* __restrict__ in, uint64_t n,
-                                                                EncTables tab, uint64_t* __restrict__ tile_bits,
-                                                                uint32_t* d_err) {
+                                                                int vec, EncTables tab,
+                                                                uint64_t* __restrict__ tile_bits, uint32_t* d_err) {
     __shared__ uint8_t s_len[256];
     __shared__ uint32_t s_red[kEncThreads / 32];
     for (uint32_t i = threadIdx.x; i < 256; i += blockDim.x) s_len[i] = tab.lengths[i];
-    __syncthreads();
-    const uint64_t base = static_cast<uint64_t>(blockIdx.x) * kTile;
+    const uint64_t i0 = static_cast<uint64_t>(blockIdx.x) * kTile + threadIdx.x * kPerThread;
+    uint32_t wv[kPerThread / 2];
+    const bool full = i0 + kPerThread <= n;
+    if (full && vec) {
+        const uint4* p4 = reinterpret_cast<const uint4*>(in + i0);
+        const uint4 v0 = __ldg(p4), v1 = __ldg(p4 + 1);
+        wv[0] = v0.x; wv[1] = v0.y; wv[2] = v0.z; wv[3] = v0.w;
+        wv[4] = v1.x; wv[5] = v1.y; wv[6] = v1.z; wv[7] = v1.w;
+    } else {
+#pragma unroll
+        for (uint32_t k = 0; k < 8; ++k) {
+            const uint64_t i = i0 + 2 * k;
+            const uint32_t lo = i < n ? __ldg(in + i) : 0u;
+            const uint32_t hi = i + 1 < n ? __ldg(in + i + 1) : 0u;
+            wv[k] = lo | (hi << 16);
+        }
+    }
+    const uint32_t cnt = full ? 16u : (i0 < n ? static_cast<uint32_t>(n - i0) : 0u);
+    __syncthreads();  // the length table
     uint32_t sum = 0;
     bool missing = false;
-#pragma unroll 4
-    for (uint32_t k = 0; k < kSteps; ++k) {
-        const uint64_t i = base + k * kEncThreads + threadIdx.x;
-        if (i < n) {
-            const uint32_t l = s_len[(__ldg(in + i) >> 7) & 0xFFu];
+#pragma unroll
+    for (uint32_t k = 0; k < 16; ++k) {
+        if (k < cnt) {
+            const uint32_t l = s_len[(wv[k >> 1] >> (16 * (k & 1) + 7)) & 0xFFu];
             missing |= (l == 0);
             sum += l;
         }
@@ -183,7 +200,6 @@ __device__ __forceinline__ void or_gap(uint32_t* gaps32, uint64_t j, uint32_t g)
 // of a tile may hold bits of the neighbouring tiles: those are OR-ed into the
 // zeroed stream atomically. The code that crosses or ends on a chunk boundary
 // writes that chunk's gap (and, at a block boundary, the block offset).
-constexpr uint32_t kPerThread = kTile / kEncThreads;  // 16 weights
 
 __global__ void __launch_bounds__(kEncThreads) pack_kernel(PackArgs a, EncTables tab) {
     __shared__ uint32_t s_code[256];
@@ -402,7 +418,8 @@ df_status df_encode(const df_code* code, const uint16_t* d_in, uint64_t n, uint6
     std::memcpy(tab.lengths, code->lengths, sizeof(tab.lengths));
     uint64_t* tile_bits = static_cast<uint64_t*>(d_ws);
     uint64_t* tile_base = tile_bits + tiles;
-    tile_bits_kernel<<<static_cast<unsigned>(tiles), kEncThreads, 0, s>>>(d_in, n, tab, tile_bits, d_err);
+    tile_bits_kernel<<<static_cast<unsigned>(tiles), kEncThreads, 0, s>>>(d_in, n, aligned(d_in, 16) ? 1 : 0, tab,
+                                                                         tile_bits, d_err);
     tile_scan_kernel<<<1, 1024, 0, s>>>(tile_bits, tiles, tile_base, total_bits, d_block_offsets, n_blocks, n,
                                          d_err);
     PackArgs a;
