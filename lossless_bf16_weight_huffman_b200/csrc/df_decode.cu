@@ -137,7 +137,9 @@ __device__ __forceinline__ void merge4(uint32_t s, uint32_t e, uint32_t* o0, uin
     *o1 = __byte_perm(lo, hi, 0x7362);
 }
 
-// 16 outputs from their 16 sign|fraction bytes and 16 exponents: two 16-byte stores.
+// 16 outputs from their 16 sign|fraction bytes and 16 exponents: two 16-byte
+// stores, marked evict-first (the outputs are not read again by this kernel and
+// should not push the prefetched stream and sign|fraction lines out of L2).
 __device__ __forceinline__ void merge16(const uint4 s16, const uint32_t e[4], uint16_t* __restrict__ dst16) {
     uint32_t o[8];
     merge4(s16.x, e[0], &o[0], &o[1]);
@@ -145,8 +147,8 @@ __device__ __forceinline__ void merge16(const uint4 s16, const uint32_t e[4], ui
     merge4(s16.z, e[2], &o[4], &o[5]);
     merge4(s16.w, e[3], &o[6], &o[7]);
     uint4* dst = reinterpret_cast<uint4*>(dst16);
-    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    __stcs(dst, make_uint4(o[0], o[1], o[2], o[3]));
+    __stcs(dst + 1, make_uint4(o[4], o[5], o[6], o[7]));
 }
 
 // A code longer than the wide window, as a step word ((length << 18) | 1 << 3,
@@ -234,7 +236,8 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_consta
         if (g < t_lo || g >= t_hi) tg = src.find(g, &t_lo, &t_hi);
         const uint64_t b = g - t_lo;
         // 1. descriptor and tables (when the tensor changes) and the stream slice
-        if (tg != staged) {
+        const bool restage = tg != staged;
+        if (restage) {
             if (tid < sizeof(DevTensor) / 4)
                 reinterpret_cast<uint32_t*>(s_td)[tid] = reinterpret_cast<const uint32_t*>(tg)[tid];
             __syncthreads();
@@ -295,7 +298,9 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_consta
                 asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(lo),
                              "r"(static_cast<uint32_t>(hi - lo)) : "memory");
         }
-        __syncthreads();
+        // only the staged tables and their check are shared here: every thread
+        // reads only its own chunk slot before the scan
+        if (restage) __syncthreads();
         if (!s_hdr[0]) {  // tables that do not belong to this descriptor
             if (tid == 0 && d_err) atomicOr(d_err, DF_EFLAG_TABLES);
             __syncthreads();
