@@ -210,6 +210,33 @@ def test_encode_variants_match_oracle(max_len, chunk_bytes, tpb):
     assert flags == 0 and (out == w).all()
 
 
+@pytest.mark.parametrize("n", [4096 * 3 + 17, 300_007])
+def test_encode_unaligned_input_and_sign_fraction_output(n):
+    """Input 2-byte aligned only and sign|fraction bytes at an odd address: the
+    per-element load and store paths of the encoder, against the oracle."""
+    w = synth.generate(synth.heavy_tail_64m()[0])[:n]
+    x = dev_u16(np.concatenate([np.zeros(1, np.uint16), w]))[1:]
+    assert x.data_ptr() % 16 != 0
+    h = torch.empty(256, dtype=torch.int64, device="cuda")
+    api.df_histogram(x, h)
+    hist = h.cpu().numpy().view(np.uint64)
+    code = api.df_build_code(hist, 32)
+    z = api.df_plan(code, hist, n, 32, 256).as_dict()
+    stream = torch.empty(z["stream_bytes"], dtype=torch.uint8, device="cuda")
+    gaps = torch.empty(z["gap_bytes"], dtype=torch.uint8, device="cuda")
+    offsets = torch.empty(z["n_blocks"] + 1, dtype=torch.int64, device="cuda")
+    sm = torch.empty(n + 1, dtype=torch.uint8, device="cuda")[1:]
+    ws = torch.empty(z["encode_ws_bytes"], dtype=torch.uint8, device="cuda")
+    err = err_word()
+    api.df_encode(code, x, z["total_bits"], 32, 256, stream, gaps, offsets, sm, ws, err)
+    assert api.df_read_error(err) == 0
+    enc = oracle.encode(w)
+    assert (stream.cpu().numpy() == enc.stream).all()
+    assert (gaps.cpu().numpy() == enc.gaps).all()
+    assert (offsets.cpu().numpy().view(np.uint64) == enc.offsets).all()
+    assert (sm.cpu().numpy() == enc.sm).all()
+
+
 @pytest.mark.parametrize("n", [0, 1, 2, 31, 33, 4095, 4096, 4097, 8193, 65537])
 def test_encode_edge_sizes(n):
     w = synth.generate(synth.single_1024x4096()[0])[:n]
