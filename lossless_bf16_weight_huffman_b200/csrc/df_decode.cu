@@ -13,8 +13,8 @@
 //      wholly inside the window and one step word, (bits used << 18) |
 //      (count << 3));
 //      stage the block's stream slice, one chunk per thread, byte-swapped to
-//      big-endian words at an odd word stride (no bank conflicts between the
-//      threads' windows)
+//      big-endian words, word i of thread t at i * T + t (the 32 lanes of a
+//      warp read 32 different banks wherever their windows are)
 //   2. one decode pass per thread over its chunk, from chunk start + gap to
 //      the chunk end: the state word (bit position << 18) | (exponents so
 //      far << 3) advances by one add per table step (up to 4 codes); the
@@ -73,7 +73,7 @@ struct BatchSrc {
 };
 
 struct LaunchCfg {
-    uint32_t words_per_chunk;  // shared-memory words of a chunk slot (odd)
+    uint32_t words_per_chunk;  // shared-memory words of a chunk (C / 4 + 1 for the widest C)
     uint32_t region_bytes;     // exponent region of a thread (4 * odd)
     uint32_t max_groups;       // owner-map entries
     uint32_t pad;
@@ -97,10 +97,13 @@ __device__ __noinline__ uint32_t long_code(uint32_t win, const uint32_t* __restr
     return ((e >> kNsymShift) & 3u) ? e : 0;
 }
 
-// The 32 stream bits from bit p of a chunk whose big-endian words start at w.
+// The 32 stream bits from bit p of a chunk whose big-endian words are at
+// w[0], w[S], w[2S], ... (S = the block size).
+template <uint32_t kT>
 __device__ __forceinline__ uint32_t window(const uint32_t* w, uint32_t p) {
-    const uint32_t i = p >> 5;
-    return __funnelshift_l(w[i + 1], w[i], p);
+    const uint32_t S = kT ? kT : blockDim.x;  // word i of the chunk at w[i * S]
+    const uint32_t* a = w + (p >> 5) * S;
+    return __funnelshift_l(a[S], a[0], p);
 }
 
 __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v, uint32_t lane) {
@@ -184,9 +187,10 @@ __device__ __forceinline__ void append(Lane& L, uint32_t w, uint32_t sy, uint32_
 }
 
 // One table step whose window lies before the chunk end.
+template <uint32_t kT>
 __device__ __forceinline__ void full_step(Lane& L, const uint32_t* words, const uint64_t* wide, const uint32_t* hier,
                                           uint32_t* region) {
-    const uint32_t win = window(words, L.st >> kStepShift);
+    const uint32_t win = window<kT>(words, L.st >> kStepShift);
     const uint64_t e = wide[win >> (32 - kWideBits)];
     uint32_t sy = static_cast<uint32_t>(e);
     uint32_t w = static_cast<uint32_t>(e >> 32);
@@ -200,11 +204,14 @@ __device__ __forceinline__ void full_step(Lane& L, const uint32_t* words, const 
     append(L, w, sy, region);
 }
 
-template <class Src, class OwnerT>
-__global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_constant__ Src src, const LaunchCfg cfg,
+// kT: the block size when fixed at compile time (256, the default format),
+// else 0 and the block size is read at run time.
+template <class Src, class OwnerT, uint32_t kT>
+__global__ void __launch_bounds__(kT ? kT : kMaxThreads, kMaxThreads / (kT ? kT : kMaxThreads))
+    decode_kernel(const __grid_constant__ Src src, const LaunchCfg cfg,
                                                              uint32_t* d_err) {
     extern __shared__ __align__(16) uint8_t smem[];
-    const uint32_t T = blockDim.x;
+    const uint32_t T = kT ? kT : blockDim.x;  // a compile-time block size folds the address arithmetic
     const uint32_t tid = threadIdx.x;
     const uint32_t lane = tid & 31, warp = tid >> 5;
     const uint32_t nwarps = T >> 5;
@@ -262,8 +269,7 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_consta
             asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(td->stream + s0),
                          "r"(static_cast<uint32_t>(s_bytes)) : "memory");
         }
-        const uint32_t wpc = C / 4 + 1;
-        uint32_t* my_words = s_words + tid * wpc;
+        uint32_t* my_words = s_words + tid;  // word i of this chunk at my_words[i * T]
         const uint64_t chunk = b * T + tid;
         Lane L;
         L.st = 0;
@@ -274,12 +280,12 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_consta
             const uint4* c4 = reinterpret_cast<const uint4*>(td->stream + chunk * C);
             for (uint32_t k = 0; k < C / 16; ++k) {
                 const uint4 v = __ldg(c4 + k);
-                my_words[4 * k + 0] = bswap32(v.x);
-                my_words[4 * k + 1] = bswap32(v.y);
-                my_words[4 * k + 2] = bswap32(v.z);
-                my_words[4 * k + 3] = bswap32(v.w);
+                my_words[(4 * k + 0) * T] = bswap32(v.x);
+                my_words[(4 * k + 1) * T] = bswap32(v.y);
+                my_words[(4 * k + 2) * T] = bswap32(v.z);
+                my_words[(4 * k + 3) * T] = bswap32(v.w);
             }
-            my_words[C / 4] = bswap32(__ldg(reinterpret_cast<const uint32_t*>(td->stream + (chunk + 1) * C)));
+            my_words[(C / 4) * T] = bswap32(__ldg(reinterpret_cast<const uint32_t*>(td->stream + (chunk + 1) * C)));
             const uint64_t q = 5 * chunk;
             const uint32_t two = (static_cast<uint32_t>(__ldg(td->gaps + (q >> 3))) << 8) |
                                  __ldg(td->gaps + (q >> 3) + 1);
@@ -313,9 +319,9 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_consta
             const bool act = (L.st >> kStepShift) + 2 * kWideBits <= L.end;
             if (!__any_sync(kFull, act)) break;
             if (act) {
-                full_step(L, my_words, s_wide, hier, my_region);
+                full_step<kT>(L, my_words, s_wide, hier, my_region);
                 // a long code may have moved p past the second window
-                if ((L.st >> kStepShift) + kWideBits <= L.end) full_step(L, my_words, s_wide, hier, my_region);
+                if ((L.st >> kStepShift) + kWideBits <= L.end) full_step<kT>(L, my_words, s_wide, hier, my_region);
             }
         }
         uint32_t cnt = (L.st & kStepCountMask) >> kStepCountShift;  // codes of whole windows start before the end
@@ -324,7 +330,7 @@ __global__ void __launch_bounds__(kMaxThreads) decode_kernel(const __grid_consta
             const bool act = p < L.end;
             if (!__any_sync(kFull, act)) break;
             if (act) {
-                const uint32_t win = window(my_words, p);
+                const uint32_t win = window<kT>(my_words, p);
                 const uint32_t x = win >> (32 - kWideBits);
                 const uint64_t e = s_wide[x];
                 uint32_t sy = static_cast<uint32_t>(e);
@@ -519,7 +525,7 @@ df_status prepare(const df_tensor* t, uint16_t* out, Prepared* pr) {
     d.tpb = T;
     d.vec_ok = aligned(t->sm, 16) && aligned(out, 16);
     pr->dev = d;
-    pr->words_per_chunk = C / 4 + 1;  // odd: C is a multiple of 16
+    pr->words_per_chunk = C / 4 + 1;  // the chunk and the next chunk's first word
     // a chunk holds at most 8C/min_len code starts; its region also takes up
     // to 3 exponents past the last counted code and the word they end in
     const uint64_t per_chunk = (cbits + minl - 1) / (minl ? minl : 1);
@@ -562,7 +568,7 @@ df_status launch_as(const Src& src, const LaunchCfg& cfg, uint32_t T, size_t sme
     df_status st = device_limits(&sms, &max_smem);
     if (st != DF_OK) return st;
     if (smem > static_cast<size_t>(max_smem)) return DF_ERR_UNSUPPORTED;
-    auto kern = decode_kernel<Src, OwnerT>;
+    auto kern = T == 256 ? decode_kernel<Src, OwnerT, 256> : decode_kernel<Src, OwnerT, 0>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return cuda_fail(e);
     int per_sm = 0;
