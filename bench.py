@@ -168,10 +168,17 @@ class ClockSampler:
 
 
 def source_digest(paths):
+    """Digest of the code in `paths` with comments and whitespace removed: a
+    comment edit keeps the digest, any change to the code changes it."""
+    import re
+
     h = hashlib.sha256()
     for p in paths:
-        with open(p, "rb") as f:
-            h.update(f.read())
+        with open(p, encoding="utf-8") as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

@@ -8,10 +8,11 @@
 // One CUDA block of T threads handles one format block (T chunks of C stream
 // bytes) at a time and loops over a contiguous range of the format blocks of
 // all tensors of the launch (persistent blocks, one range each):
-//   1. when the tensor changes, stage its wide table in shared memory (1024
-//      entries indexed by 10 stream bits: the exponents of the codes that lie
-//      wholly inside the window and one step word, (bits used << 18) |
-//      (count << 3));
+//   1. when the tensor changes, copy its descriptor and stage its wide table
+//      in shared memory (1024 entries indexed by 10 stream bits: the exponents
+//      of the codes that lie wholly inside the window and one step word,
+//      (bits used << 18) | (count << 3)); warm L2 with the next block's stream
+//      slice and this block's sign|fraction bytes (bulk prefetches);
 //      stage the block's stream slice, one chunk per thread, byte-swapped to
 //      big-endian words, word i of thread t at i * T + t (the 32 lanes of a
 //      warp read 32 different banks wherever their windows are)
