@@ -12,7 +12,7 @@
 //      in shared memory (1024 entries indexed by 10 stream bits: the exponents
 //      of the codes that lie wholly inside the window and one step word,
 //      (bits used << 18) | (count << 3)); warm L2 with the next block's stream
-//      slice and this block's sign|fraction bytes (bulk prefetches);
+//      slice (bulk prefetch);
 //      stage the block's stream slice, one chunk per thread, byte-swapped to
 //      big-endian words, word i of thread t at i * T + t (the 32 lanes of a
 //      warp read 32 different banks wherever their windows are)
@@ -21,6 +21,9 @@
 //      far << 3) advances by one add per table step (up to 4 codes); the
 //      exponents go to the thread's own word-aligned shared-memory region
 //      with 32-bit stores; codes longer than 10 bits walk the 8-bit tables
+//      then warm L2 with this block's sign|fraction bytes, and load this
+//      thread's chunk of the next block into registers (it goes into the idle
+//      slot just before the merge, so the next block starts without a load)
 //   3. block scan of the code counts (warp shuffles + one shared array): the
 //      first output position of every thread; checked against the block index
 //   4. an owner map: for every group of 16 outputs, the thread whose region
@@ -235,6 +238,8 @@ __global__ void __launch_bounds__(kT ? kT : kMaxThreads, kMaxThreads / (kT ? kT 
     const DevTensor* staged = nullptr;
     const DevTensor* const td = s_td;  // read through its shared-memory copy
     uint64_t t_lo = 0, t_hi = 0;
+    bool pre = false;      // this thread's chunk of block g is already in its slot
+    uint32_t pre_two = 0;  // and its two gap bytes
     // each CUDA block takes a contiguous range of format blocks, so that it
     // changes tensors (and restages tables) as rarely as possible
     const uint64_t per = cfg.total_blocks / gridDim.x, extra = cfg.total_blocks % gridDim.x;
@@ -278,33 +283,31 @@ __global__ void __launch_bounds__(kT ? kT : kMaxThreads, kMaxThreads / (kT ? kT 
         L.acc = 0;
         L.bad = false;
         if (chunk < td->n_chunks) {
-            const uint4* c4 = reinterpret_cast<const uint4*>(td->stream + chunk * C);
-            for (uint32_t k = 0; k < C / 16; ++k) {
-                const uint4 v = __ldg(c4 + k);
-                my_words[(4 * k + 0) * T] = bswap32(v.x);
-                my_words[(4 * k + 1) * T] = bswap32(v.y);
-                my_words[(4 * k + 2) * T] = bswap32(v.z);
-                my_words[(4 * k + 3) * T] = bswap32(v.w);
-            }
-            my_words[(C / 4) * T] = bswap32(__ldg(reinterpret_cast<const uint32_t*>(td->stream + (chunk + 1) * C)));
             const uint64_t q = 5 * chunk;
-            const uint32_t two = (static_cast<uint32_t>(__ldg(td->gaps + (q >> 3))) << 8) |
-                                 __ldg(td->gaps + (q >> 3) + 1);
+            uint32_t two;
+            if (pre) {
+                two = pre_two;
+            } else {
+                const uint4* c4 = reinterpret_cast<const uint4*>(td->stream + chunk * C);
+                for (uint32_t k = 0; k < C / 16; ++k) {
+                    const uint4 v = __ldg(c4 + k);
+                    my_words[(4 * k + 0) * T] = bswap32(v.x);
+                    my_words[(4 * k + 1) * T] = bswap32(v.y);
+                    my_words[(4 * k + 2) * T] = bswap32(v.z);
+                    my_words[(4 * k + 3) * T] = bswap32(v.w);
+                }
+                my_words[(C / 4) * T] = bswap32(__ldg(reinterpret_cast<const uint32_t*>(td->stream + (chunk + 1) * C)));
+                two = (static_cast<uint32_t>(__ldg(td->gaps + (q >> 3))) << 8) | __ldg(td->gaps + (q >> 3) + 1);
+            }
             const uint32_t cbits = 8 * C;
             const uint64_t bit0 = chunk * cbits;
             const uint64_t rem = td->total_bits > bit0 ? td->total_bits - bit0 : 0;
             L.st = ((two >> (11 - (q & 7))) & 31u) << kStepShift;
             L.end = static_cast<uint32_t>(rem < cbits ? rem : cbits);
         }
+        pre = false;
         const uint64_t out0 = td->offs[b];
         const uint64_t out1 = td->offs[b + 1];
-        if (tid == 0 && out0 <= out1 && out1 <= td->n) {  // warm L2 with the block's sign|fraction bytes
-            const uintptr_t lo = (reinterpret_cast<uintptr_t>(td->sm + out0) + 15) & ~static_cast<uintptr_t>(15);
-            const uintptr_t hi = reinterpret_cast<uintptr_t>(td->sm + out1) & ~static_cast<uintptr_t>(15);
-            if (hi > lo)
-                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(lo),
-                             "r"(static_cast<uint32_t>(hi - lo)) : "memory");
-        }
         // only the staged tables and their check are shared here: every thread
         // reads only its own chunk slot before the scan
         if (restage) __syncthreads();
@@ -356,6 +359,28 @@ __global__ void __launch_bounds__(kT ? kT : kMaxThreads, kMaxThreads / (kT ? kT 
         }
         // the pending exponents (at most 3) complete the region
         my_region[(L.st & kStepCountMask) >> 5] = L.acc;
+        // load this thread's chunk of the next block (same tensor, C <= 32) now;
+        // it goes into the (idle) slot after the owner map, before the merge
+        const uint64_t nchunk = chunk + T;
+        const bool nx = C <= 32 && g + 1 < g_end && g + 1 < t_hi && nchunk < td->n_chunks;
+        uint4 na = make_uint4(0, 0, 0, 0), nb = make_uint4(0, 0, 0, 0);
+        uint32_t ntail = 0, ntwo = 0;
+        if (nx) {
+            const uint4* c4 = reinterpret_cast<const uint4*>(td->stream + nchunk * C);
+            na = __ldg(c4);
+            if (C == 32) nb = __ldg(c4 + 1);
+            ntail = __ldg(reinterpret_cast<const uint32_t*>(td->stream + (nchunk + 1) * C));
+            const uint64_t qn = 5 * nchunk;
+            ntwo = (static_cast<uint32_t>(__ldg(td->gaps + (qn >> 3))) << 8) | __ldg(td->gaps + (qn >> 3) + 1);
+        }
+        // warm L2 with the block's sign|fraction bytes (the offsets have arrived by now)
+        if (tid == 0 && out0 <= out1 && out1 <= td->n) {
+            const uintptr_t lo = (reinterpret_cast<uintptr_t>(td->sm + out0) + 15) & ~static_cast<uintptr_t>(15);
+            const uintptr_t hi = reinterpret_cast<uintptr_t>(td->sm + out1) & ~static_cast<uintptr_t>(15);
+            if (hi > lo)
+                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(lo),
+                             "r"(static_cast<uint32_t>(hi - lo)) : "memory");
+        }
 
         // 3. block scan of the counts: warp totals (with a corrupt-data bit)
         // in shared memory, then every warp scans them again on its own
@@ -395,6 +420,21 @@ __global__ void __launch_bounds__(kT ? kT : kMaxThreads, kMaxThreads / (kT ? kT 
             for (uint32_t gi = max((pos + 15) >> 4, 1u); 16 * gi < hi; ++gi) s_owner[gi] = static_cast<OwnerT>(tid);
         }
         __syncthreads();
+        if (nx) {  // only this thread reads its slot, and not before the next block's decode
+            my_words[0 * T] = bswap32(na.x);
+            my_words[1 * T] = bswap32(na.y);
+            my_words[2 * T] = bswap32(na.z);
+            my_words[3 * T] = bswap32(na.w);
+            if (C == 32) {
+                my_words[4 * T] = bswap32(nb.x);
+                my_words[5 * T] = bswap32(nb.y);
+                my_words[6 * T] = bswap32(nb.z);
+                my_words[7 * T] = bswap32(nb.w);
+            }
+            my_words[(C / 4) * T] = bswap32(ntail);
+            pre_two = ntwo;
+            pre = true;
+        }
 
         // 5. merge and store; stage position c <-> output gbase + c
         const uint8_t* __restrict__ sm = td->sm;
