@@ -39,7 +39,8 @@
  *     errors are reported through the optional device error word `d_err`
  *     (DF_EFLAG_* bits OR-ed in; the caller zeroes it) and df_read_error;
  *   - no function keeps global mutable state except the per-thread last CUDA
- *     error returned by df_last_cuda_error.
+ *     error returned by df_last_cuda_error and df_encode_noalloc's static
+ *     device scratch (with its per-device address, looked up once).
  */
 #ifndef DF11_H
 #define DF11_H
