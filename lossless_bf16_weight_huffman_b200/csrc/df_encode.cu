@@ -67,6 +67,29 @@ struct EncTables {
     uint8_t lengths[256];
 };
 
+// The 16 consecutive weights of a thread from weight i0 on, two per 32-bit
+// word (weight i0 + k in bits 16 * (k & 1) of word k / 2); weights at or past n
+// read as 0. Returns how many of the 16 are below n.
+__device__ __forceinline__ uint32_t load16(const uint16_t* __restrict__ in, uint64_t n, uint64_t i0, bool vec,
+                                           uint32_t wv[kPerThread / 2]) {
+    const bool full = i0 + kPerThread <= n;
+    if (full && vec) {
+        const uint4* p4 = reinterpret_cast<const uint4*>(in + i0);
+        const uint4 v0 = __ldg(p4), v1 = __ldg(p4 + 1);
+        wv[0] = v0.x; wv[1] = v0.y; wv[2] = v0.z; wv[3] = v0.w;
+        wv[4] = v1.x; wv[5] = v1.y; wv[6] = v1.z; wv[7] = v1.w;
+    } else {
+#pragma unroll
+        for (uint32_t k = 0; k < kPerThread / 2; ++k) {
+            const uint64_t i = i0 + 2 * k;
+            const uint32_t lo = i < n ? __ldg(in + i) : 0u;
+            const uint32_t hi = i + 1 < n ? __ldg(in + i + 1) : 0u;
+            wv[k] = lo | (hi << 16);
+        }
+    }
+    return full ? kPerThread : (i0 < n ? static_cast<uint32_t>(n - i0) : 0u);
+}
+
 // Sum of code lengths of each tile of 4096 weights (16 consecutive weights per
 // thread, as the packer reads them).
 __global__ void __launch_bounds__(kEncThreads) tile_bits_kernel(const uint16_t* __restrict__ in, uint64_t n,
@@ -77,27 +100,12 @@ __global__ void __launch_bounds__(kEncThreads) tile_bits_kernel(const uint16_t* 
     for (uint32_t i = threadIdx.x; i < 256; i += blockDim.x) s_len[i] = tab.lengths[i];
     const uint64_t i0 = static_cast<uint64_t>(blockIdx.x) * kTile + threadIdx.x * kPerThread;
     uint32_t wv[kPerThread / 2];
-    const bool full = i0 + kPerThread <= n;
-    if (full && vec) {
-        const uint4* p4 = reinterpret_cast<const uint4*>(in + i0);
-        const uint4 v0 = __ldg(p4), v1 = __ldg(p4 + 1);
-        wv[0] = v0.x; wv[1] = v0.y; wv[2] = v0.z; wv[3] = v0.w;
-        wv[4] = v1.x; wv[5] = v1.y; wv[6] = v1.z; wv[7] = v1.w;
-    } else {
-#pragma unroll
-        for (uint32_t k = 0; k < 8; ++k) {
-            const uint64_t i = i0 + 2 * k;
-            const uint32_t lo = i < n ? __ldg(in + i) : 0u;
-            const uint32_t hi = i + 1 < n ? __ldg(in + i + 1) : 0u;
-            wv[k] = lo | (hi << 16);
-        }
-    }
-    const uint32_t cnt = full ? 16u : (i0 < n ? static_cast<uint32_t>(n - i0) : 0u);
+    const uint32_t cnt = load16(in, n, i0, vec != 0, wv);
     __syncthreads();  // the length table
     uint32_t sum = 0;
     bool missing = false;
 #pragma unroll
-    for (uint32_t k = 0; k < 16; ++k) {
+    for (uint32_t k = 0; k < kPerThread; ++k) {
         if (k < cnt) {
             const uint32_t l = s_len[(wv[k >> 1] >> (16 * (k & 1) + 7)) & 0xFFu];
             missing |= (l == 0);
@@ -212,24 +220,9 @@ __global__ void __launch_bounds__(kEncThreads) pack_kernel(PackArgs a, EncTables
         s_len[i] = tab.lengths[i];
     }
     const uint64_t i0 = static_cast<uint64_t>(blockIdx.x) * kTile + tid * kPerThread;
-    // this thread's 16 weights (two pairs per 32-bit word)
-    uint32_t wv[kPerThread / 2];
-    const bool full = i0 + kPerThread <= a.n;
-    if (full && a.in_vec) {
-        const uint4* p4 = reinterpret_cast<const uint4*>(a.in + i0);
-        const uint4 v0 = __ldg(p4), v1 = __ldg(p4 + 1);
-        wv[0] = v0.x; wv[1] = v0.y; wv[2] = v0.z; wv[3] = v0.w;
-        wv[4] = v1.x; wv[5] = v1.y; wv[6] = v1.z; wv[7] = v1.w;
-    } else {
-#pragma unroll
-        for (uint32_t k = 0; k < kPerThread / 2; ++k) {
-            const uint64_t i = i0 + 2 * k;
-            const uint32_t lo = i < a.n ? __ldg(a.in + i) : 0u;
-            const uint32_t hi = i + 1 < a.n ? __ldg(a.in + i + 1) : 0u;
-            wv[k] = lo | (hi << 16);
-        }
-    }
-    const uint32_t cnt = full ? kPerThread : (i0 < a.n ? static_cast<uint32_t>(a.n - i0) : 0u);
+    uint32_t wv[kPerThread / 2];  // this thread's 16 weights
+    const uint32_t cnt = load16(a.in, a.n, i0, a.in_vec != 0, wv);
+    const bool full = cnt == kPerThread;
     // sign|fraction bytes
     uint32_t smw[kPerThread / 4];
 #pragma unroll
