@@ -64,7 +64,10 @@ void oracle_join(const uint8_t* e, const uint8_t* sm, uint64_t n, uint16_t* w) {
     for (uint64_t i = 0; i < n; ++i) w[i] = join(e[i], sm[i]);
 }
 
-/* ---- 2. histogram -------------------------------------------------------- */
+/* ---- 2. histogram ----------------------------------------------------------
+ * Counts of each exponent value: the frequencies the codebook is built from
+ * (df11pack, GitHub page, intro and "Licence").
+ */
 
 void oracle_histogram(const uint16_t* w, uint64_t n, uint64_t hist[256]) {
     for (int s = 0; s < 256; ++s) hist[s] = 0;
@@ -168,7 +171,10 @@ int oracle_package_merge(const uint64_t hist[256], int max_len, uint8_t lengths[
 
 /* ---- 4. canonical codes ---------------------------------------------------
  * Symbols sorted by (length, symbol); the first gets code 0, each next one
- * code = (previous code + 1) << (its length - previous length).
+ * code = (previous code + 1) << (its length - previous length). The pages
+ * require a deterministic codebook (df11pack, intro and "Licence") but do not
+ * say how codes are assigned to lengths; canonical order is this library's
+ * reading.
  */
 void oracle_canonical_codes(const uint8_t lengths[256], uint32_t codes[256]) {
     int order[256], k = 0;
@@ -192,7 +198,9 @@ void oracle_canonical_codes(const uint8_t lengths[256], uint32_t codes[256]) {
 }
 
 /* ---- 9. size accounting ----------------------------------------------------
- * Container layout (this library's own; the pages do not give one):
+ * The pages give only the outcome, about 70% of the BF16 size (mlx-dfloat,
+ * PyPI page, intro; df11pack, intro). Container layout (this library's own;
+ * the pages do not give one):
  *   stream   n_chunks * C bytes of MSB-first code bits, then 16 zero bytes
  *   gaps     5 bits per chunk, MSB-first, then zero padding: at least one
  *            byte, up to a multiple of 16
@@ -228,7 +236,9 @@ uint64_t oracle_total_bits(const uint64_t hist[256], const uint8_t lengths[256])
 }
 
 /* ---- 6/7. chunk gaps and block offsets from code start positions ----------
- * A code belongs to the chunk that holds its first bit. gap[j] is the distance
+ * The pages name independently decodable chunks / units (df11pack, "Use") and
+ * a block index (df11pack, "What is checked", --index idx8) without their
+ * encoding. A code belongs to the chunk that holds its first bit. gap[j] is the distance
  * from the chunk's first bit 8Cj to the first code start at or after it; when
  * no code starts in the chunk (possible only in the last one), the end of the
  * stream, total_bits, counts as that start (this library's reading: it lets a
@@ -261,8 +271,11 @@ static void index_visit(index_walk* wk, uint64_t start, uint64_t index) {
 }
 
 /* ---- 5. encode --------------------------------------------------------------
- * For i = 0..n-1 append code[e_i] in len[e_i] bits, most significant bit
- * first; the first stream bit is bit 7 of byte 0. Buffers are sized by
+ * The exponent byte of each weight is replaced by its variable-length code and
+ * the sign|fraction byte is kept raw (mlx-dfloat, PyPI page, intro and its bit
+ * diagram). For i = 0..n-1 append code[e_i] in len[e_i] bits, most
+ * significant bit first; the first stream bit is bit 7 of byte 0 (the bit
+ * order is this library's reading). Buffers are sized by
  * oracle_sizes and are zeroed here.
  */
 int oracle_encode(const uint16_t* w, uint64_t n, const uint8_t lengths[256], const uint32_t codes[256],
@@ -292,7 +305,8 @@ int oracle_encode(const uint16_t* w, uint64_t n, const uint8_t lengths[256], con
 }
 
 /* ---- 8. bit-serial canonical decode ------------------------------------------
- * One bit at a time from bit 0: code = code << 1 | bit; at length l the code is
+ * Decoding gives back the original bits exactly (mlx-dfloat, PyPI page, intro
+ * and "Status"). One bit at a time from bit 0: code = code << 1 | bit; at length l the code is
  * complete when first[l] <= code < first[l] + count[l], and names symbol
  * sorted[base[l] + code - first[l]] (canonical decoding; no lookup tables).
  * Every code must end at or before total_bits, exactly n codes must be read
