@@ -28,6 +28,41 @@ def _dev(t: torch.Tensor | None, name: str):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _need(t: torch.Tensor, nbytes: int, name: str) -> None:
+    """The library writes nbytes through t's pointer: refuse a smaller buffer
+    before any device write can run past it."""
+    have = t.numel() * t.element_size()
+    if have < nbytes:
+        raise ValueError(f"{name} holds {have} bytes; the call writes {nbytes}")
+
+
+def _format_ok(chunk_bytes: int, threads_per_block: int) -> bool:
+    return (16 <= chunk_bytes <= 4096 and chunk_bytes % 16 == 0 and 32 <= threads_per_block <= 1024
+            and threads_per_block % 32 == 0)
+
+
+def container_layout(n: int, total_bits: int, chunk_bytes: int, threads_per_block: int) -> dict:
+    """Bytes of each buffer df_encode writes for n weights and total_bits code
+    bits (the container layout of include/df11.h; df_plan reports the same)."""
+    cbits = 8 * chunk_bytes
+    n_chunks = (total_bits + cbits - 1) // cbits if total_bits else 1
+    n_blocks = (n_chunks + threads_per_block - 1) // threads_per_block
+    return {"stream_bytes": n_chunks * chunk_bytes + 16,
+            "gap_bytes": (((5 * n_chunks + 7) // 8) + 1 + 15) & ~15,
+            "offsets_bytes": 8 * (n_blocks + 1),
+            "sm_bytes": n}
+
+
+def _check_encode_buffers(n, total_bits, chunk_bytes, threads_per_block, d_stream, d_gaps, d_block_offsets, d_sm):
+    if not _format_ok(chunk_bytes, threads_per_block):
+        return  # the library rejects the format itself
+    z = container_layout(n, total_bits, chunk_bytes, threads_per_block)
+    _need(d_stream, z["stream_bytes"], "d_stream")
+    _need(d_gaps, z["gap_bytes"], "d_gaps")
+    _need(d_block_offsets, z["offsets_bytes"], "d_block_offsets")
+    _need(d_sm, z["sm_bytes"], "d_sm")
+
+
 def _hist_array(hist) -> np.ndarray:
     h = np.ascontiguousarray(np.asarray(hist, dtype=np.uint64).reshape(-1))
     if h.size != 256:
@@ -87,6 +122,8 @@ def df_encode(code: DfCode, d_in: torch.Tensor, total_bits: int, chunk_bytes: in
               d_stream: torch.Tensor, d_gaps: torch.Tensor, d_block_offsets: torch.Tensor, d_sm: torch.Tensor,
               d_ws: torch.Tensor, d_err: torch.Tensor | None = None, stream=None) -> None:
     ws_bytes = d_ws.numel() * d_ws.element_size() if d_ws is not None else 0
+    _check_encode_buffers(d_in.numel(), total_bits, chunk_bytes, threads_per_block, d_stream, d_gaps,
+                          d_block_offsets, d_sm)
     check("df_encode", lib().df_encode(
         ctypes.byref(code), _dev(d_in, "d_in"), d_in.numel(), total_bits, chunk_bytes, threads_per_block,
         _dev(d_stream, "d_stream"), _dev(d_gaps, "d_gaps"), _dev(d_block_offsets, "d_block_offsets"),
@@ -99,6 +136,8 @@ def df_encode_noalloc(code: DfCode, d_in: torch.Tensor, total_bits: int, chunk_b
     """df_encode with the library's static scratch instead of a workspace
     (for callers that cannot allocate device memory; calls on one GPU must not
     overlap)."""
+    _check_encode_buffers(d_in.numel(), total_bits, chunk_bytes, threads_per_block, d_stream, d_gaps,
+                          d_block_offsets, d_sm)
     check("df_encode_noalloc", lib().df_encode_noalloc(
         ctypes.byref(code), _dev(d_in, "d_in"), d_in.numel(), total_bits, chunk_bytes, threads_per_block,
         _dev(d_stream, "d_stream"), _dev(d_gaps, "d_gaps"), _dev(d_block_offsets, "d_block_offsets"),
@@ -106,6 +145,8 @@ def df_encode_noalloc(code: DfCode, d_in: torch.Tensor, total_bits: int, chunk_b
 
 
 def df_decode(t: DfTensor, d_out: torch.Tensor, d_err: torch.Tensor | None = None, stream=None) -> None:
+    if isinstance(d_out, torch.Tensor):
+        _need(d_out, 2 * t.n, "d_out")
     check("df_decode", lib().df_decode(ctypes.byref(t), _dev(d_out, "d_out"), _dev(d_err, "d_err"),
                                        _stream_ptr(stream)))
 
@@ -117,6 +158,9 @@ def df_decode_batch_workspace(count: int) -> int:
 def _batch_arrays(tensors, d_outs):
     if len(tensors) != len(d_outs):
         raise ValueError("one output per tensor")
+    for i, (t, o) in enumerate(zip(tensors, d_outs)):
+        if isinstance(o, torch.Tensor):
+            _need(o, 2 * t.n, f"d_outs[{i}]")
     arr = (DfTensor * max(1, len(tensors)))(*tensors)
     outs = (ctypes.c_void_p * max(1, len(d_outs)))(*[_dev(o, "d_outs[i]").value for o in d_outs])
     return arr, outs

@@ -257,3 +257,50 @@ def test_unreachable_entries_are_zero():
     assert ((wide >> np.uint64(32 + 18)) == 8).all()
     hier = lut[5 * (1 << WIDE) // 2:]
     assert (hier[:256] != 0).all()
+
+
+# ---------------------------------------------------------------- the binding's buffer checks
+
+
+def test_binding_layout_matches_plan():
+    rng = np.random.default_rng(7)
+    for trial in range(400):
+        h = _random_hist(rng, trial % 5)
+        code = api.df_build_code(h, 32)
+        n = int(h.sum())
+        C = int(rng.choice([16, 32, 48, 64, 128, 1024, 4096]))
+        T = int(rng.choice([32, 64, 96, 256, 1024]))
+        z = api.df_plan(code, h, n, C, T).as_dict()
+        got = api.container_layout(n, z["total_bits"], C, T)
+        for key, val in got.items():
+            assert val == z[key], (trial, key)
+    z = api.df_plan(api.df_build_code(np.zeros(256, np.uint64)), np.zeros(256, np.uint64), 0, 32, 256).as_dict()
+    got = api.container_layout(0, 0, 32, 256)
+    assert all(got[k] == z[k] for k in got)
+
+
+def test_binding_refuses_short_buffers_before_the_library():
+    import torch
+
+    h = np.zeros(256, np.uint64)
+    h[120:124] = [50, 30, 15, 5]
+    code = api.df_build_code(h, 32)
+    z = api.df_plan(code, h, 100, 32, 256).as_dict()
+    x = torch.zeros(100, dtype=torch.int16)
+    bufs = dict(d_stream=torch.empty(z["stream_bytes"], dtype=torch.uint8),
+                d_gaps=torch.empty(z["gap_bytes"], dtype=torch.uint8),
+                d_block_offsets=torch.empty(z["n_blocks"] + 1, dtype=torch.int64),
+                d_sm=torch.empty(100, dtype=torch.uint8))
+    for name in bufs:
+        short = dict(bufs)
+        short[name] = bufs[name][:-1]
+        with pytest.raises(ValueError, match=name):
+            api.df_encode(code, x, z["total_bits"], 32, 256, d_ws=torch.empty(16, dtype=torch.uint8), **short)
+        with pytest.raises(ValueError, match=name):
+            api.df_encode_noalloc(code, x, z["total_bits"], 32, 256, **short)
+    d = _native.DfTensor()
+    d.n = 100
+    with pytest.raises(ValueError, match="d_out"):
+        api.df_decode(d, torch.empty(99, dtype=torch.int16))
+    with pytest.raises(ValueError, match="d_outs"):
+        api.df_decode_batch_prepare([d], [torch.empty(50, dtype=torch.int16)], torch.empty(4096, dtype=torch.uint8))
