@@ -70,8 +70,6 @@ def lib():
         L.oracle_encode.restype = i32
         L.oracle_decode.argtypes = [vp, u64, vp, u64, vp, u32, u32, vp, vp, vp]
         L.oracle_decode.restype = i32
-        L.oracle_plan.argtypes = [vp, i32, u32, u32, vp, ctypes.POINTER(Sizes)]
-        L.oracle_plan.restype = i32
         _lib = L
     return _lib
 

@@ -361,14 +361,3 @@ int oracle_decode(const uint8_t* stream, uint64_t total_bits, const uint8_t* sm,
     if (offsets) offsets[z.n_blocks] = n;
     return ORACLE_OK;
 }
-
-/* Size of the code for a histogram: the whole encode-side computation from
- * frequencies to byte counts, for size comparisons at scale. */
-int oracle_plan(const uint64_t hist[256], int max_len, uint32_t chunk_bytes, uint32_t threads_per_block,
-                uint8_t lengths[256], oracle_sizes_t* out) {
-    int rc = oracle_package_merge(hist, max_len, lengths);
-    if (rc != ORACLE_OK) return rc;
-    uint64_t n = 0;
-    for (int s = 0; s < 256; ++s) n += hist[s];
-    return oracle_sizes(n, oracle_total_bits(hist, lengths), chunk_bytes, threads_per_block, out);
-}
