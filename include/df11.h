@@ -111,19 +111,21 @@ typedef struct df_tensor {
 typedef struct df_batch_plan {
     void* d_ws;                /* the workspace holding the device table        */
     uint32_t count;            /* tensors with n > 0                            */
-    uint32_t threads_per_block;/* T, shared by all tensors (CUDA block size)    */
+    uint32_t cta_threads;      /* threads per CUDA block of the launch          */
     uint32_t words_per_chunk;  /* shared-memory words per chunk (widest C)      */
-    uint32_t region_bytes;     /* shared-memory exponent region of a thread     */
-    uint32_t max_groups;       /* 16-output groups a block may span             */
+    uint32_t region_bytes;     /* shared-memory exponent region of a lane       */
+    uint32_t max_groups;       /* 16-output groups a round of 32 chunks spans   */
     uint32_t smem_bytes;       /* dynamic shared memory per CUDA block          */
     uint64_t total_blocks;     /* format blocks over all tensors                */
 } df_batch_plan;
 
-/* Human-readable name of a status. Static string; never NULL. */
+/* Human-readable name of a status. Static string; never NULL.
+ * Source: none on the pages (an error-reporting helper of this ABI). */
 const char* df_status_string(df_status s);
 
 /* The cudaError_t of the last failing CUDA call made by this thread inside
- * the library (0 if none). */
+ * the library (0 if none). Source: none on the pages (an error-reporting
+ * helper of this ABI). */
 int df_last_cuda_error(void);
 
 /* ---- code construction (host only) ---------------------------------------
@@ -140,14 +142,17 @@ int df_last_cuda_error(void);
 df_status df_build_code(const uint64_t hist[256], uint32_t max_len, df_code* out);
 
 /* df_code_from_lengths: the canonical code for given code lengths (0 = no
- * code), e.g. the lengths stored in a container. Errors: DF_ERR_INVALID_ARG
+ * code), e.g. the lengths stored in a container. Source: df11pack, intro
+ * (the codebook is a function of the stored frequencies/lengths, so a reader
+ * rebuilds the same code). Errors: DF_ERR_INVALID_ARG
  * (null, a length above max_len, or lengths that break Kraft's inequality
  * sum 2^-l <= 1); DF_ERR_UNSUPPORTED (max_len outside 1..32). */
 df_status df_code_from_lengths(const uint8_t lengths[256], uint32_t max_len, df_code* out);
 
-/* Number of uint32 words df_build_lut writes: 2560 for the wide table, 256
- * per 8-bit-indexed table, 64 for the code lengths and a 4-word header.
- * 0 for a NULL code. */
+/* Number of uint32 words df_build_lut writes: the wide table (5 words per
+ * window value), 256 per 8-bit-indexed table, 64 for the code lengths and a
+ * 4-word header. 0 for a NULL code. Source: df11pack, "What is checked"
+ * (decode lookup tables). */
 size_t df_lut_words(const df_code* code);
 
 /* df_build_lut: derive the decode tables of a code into host memory `lut`
@@ -174,13 +179,25 @@ size_t df_lut_words(const df_code* code);
 df_status df_build_lut(const df_code* code, uint32_t* lut, size_t lut_words);
 
 /* df_plan: exact sizes of the container for n weights with exponent
- * histogram hist under `code`, and of df_encode's workspace.
+ * histogram hist under `code`, and of df_encode's workspace. Source:
+ * mlx-dfloat, intro (the container is the exponent code plus one raw byte per
+ * weight); the byte counts follow the layout at the top of this header.
  * Errors: DF_ERR_INVALID_ARG (null; hist total != n; an exponent present in
  * hist without a code; chunk_bytes not a multiple of 16 in 16..4096;
  * threads_per_block not a multiple of 32 in 32..1024); DF_ERR_UNSUPPORTED
  * (n > DF_MAX_WEIGHTS). */
 df_status df_plan(const df_code* code, const uint64_t hist[256], uint64_t n, uint32_t chunk_bytes,
                   uint32_t threads_per_block, df_sizes* out);
+
+/* df_container_sizes: the same sizes for a container whose histogram is not
+ * at hand (one read from a file, one to be filled by df_encode): n weights
+ * and total_bits code bits under chunk_bytes and threads_per_block. The
+ * buffer sizes depend on nothing else. Source: the container layout at the
+ * top of this header (the pages give none). Errors: DF_ERR_INVALID_ARG (null;
+ * the format checks of df_plan; total_bits outside [n, 32n]);
+ * DF_ERR_UNSUPPORTED (n > DF_MAX_WEIGHTS). */
+df_status df_container_sizes(uint64_t n, uint64_t total_bits, uint32_t chunk_bytes, uint32_t threads_per_block,
+                             df_sizes* out);
 
 /* ---- encode (device) ---------------------------------------------------------
  * df_histogram: d_hist256[e] = number of weights of d_in[0..n) whose exponent
@@ -213,9 +230,12 @@ df_status df_encode(const df_code* code, const uint16_t* d_in, uint64_t n, uint6
  * that may only use the buffers its host hands it). Its scratch (per-tile bit
  * counts and bases) lives in a static device array of the library, 2 MiB per
  * GPU that loads the library, held until the process exits; n is limited to
- * DF_ENCODE_NOALLOC_MAX_WEIGHTS. The first call on a device looks up the
- * array's device address (cudaGetSymbolAddress) and caches it; make that
- * first call before any stream capture. Every call on a device shares the
+ * DF_ENCODE_NOALLOC_MAX_WEIGHTS. A call looks up the array's device address
+ * (cudaGetSymbolAddress) on its device, except while `stream` is capturing,
+ * when the address found by the last call on that device is used; so make
+ * the first call on a device before any stream capture (a first call inside
+ * a capture returns DF_ERR_UNSUPPORTED), and after a device reset call it
+ * once outside a capture before capturing it again. Every call on a device shares the
  * array, so calls that overlap on the GPU (other streams, other host threads)
  * race: serialize them. Allocates nothing: no cudaMalloc, cudaFree or
  * allocating library routine. The pages have no counterpart of this entry
@@ -229,45 +249,54 @@ df_status df_encode_noalloc(const df_code* code, const uint16_t* d_in, uint64_t 
 
 /* ---- decode (device) ---------------------------------------------------------
  * df_decode: d_out[0..t->n) = the original BF16 bit patterns (uint16, device;
- * 16-byte alignment of d_out and t->sm takes the vector path). A CUDA block
- * of T threads decodes one format block (T chunks) at a time: the wide table
- * and the block's stream slice are staged in shared memory, each thread
- * decodes its chunk once into its own shared-memory region of exponents, a
- * block scan turns the counts into output positions, and the block merges
- * the exponents with the sign|fraction bytes in groups of 16 outputs
- * (16-byte loads and stores). Chunks of up to 1024 bytes. Source: mlx-dfloat, intro and "Status"
- * (blockwise GPU decode back to identical bits); df11pack, "Use" (chunks).
- * Data errors set DF_EFLAG_* in d_err (nullable) and skip the affected
- * block's stores. Errors: DF_ERR_INVALID_ARG, DF_ERR_UNSUPPORTED (a layout
- * whose block needs more shared memory than the device has), DF_ERR_CUDA.
+ * 16-byte alignment of d_out and t->sm takes the vector path). Every warp
+ * decodes whole format blocks on its own, 32 chunks at a time: each lane
+ * decodes one chunk into a shared-memory region of exponents (multi-code
+ * table lookups), a warp scan turns the counts into output positions, and
+ * the warp merges the exponents with the sign|fraction bytes in groups of 16
+ * outputs (16-byte loads and stores). Chunks of up to 1024 bytes. Source:
+ * mlx-dfloat, intro and "Status" (blockwise GPU decode back to identical
+ * bits); df11pack, "Use" (independently decodable chunks).
+ * Data errors set DF_EFLAG_* in d_err (nullable); the affected block stops
+ * at the round (32 chunks) where the error shows, so its outputs may be
+ * partly written, never outside d_out[0..n). Errors: DF_ERR_INVALID_ARG,
+ * DF_ERR_UNSUPPORTED (a layout whose warp needs more shared memory than the
+ * device has), DF_ERR_CUDA.
  */
 df_status df_decode(const df_tensor* t, uint16_t* d_out, uint32_t* d_err, void* stream);
 
-/* Device workspace bytes df_decode_batch needs for `count` tensors. */
+/* Device workspace bytes df_decode_batch needs for `count` tensors.
+ * Source: none on the pages (the grouped launch is this library's own). */
 size_t df_decode_batch_workspace(uint32_t count);
 
 /* df_decode_batch_prepare: validate `count` descriptors (host array) and
  * their outputs (host array of device pointers), write the device table into
  * d_ws (asynchronously on `stream`; the host arrays may be reused on return)
- * and fill *plan. All tensors must share threads_per_block; chunk_bytes may
- * differ (shared memory is sized for the widest).
+ * and fill *plan. chunk_bytes and threads_per_block may differ between
+ * tensors (shared memory is sized for the widest chunk). Source: none on the
+ * pages: one launch over many tensors (biases, norms, small linears) is this
+ * library's own entry point; each tensor decodes as in df_decode.
  * Errors: DF_ERR_INVALID_ARG, DF_ERR_WORKSPACE, DF_ERR_UNSUPPORTED, DF_ERR_CUDA. */
 df_status df_decode_batch_prepare(const df_tensor* tensors, uint16_t* const* d_outs, uint32_t count, void* d_ws,
                                   size_t ws_bytes, df_batch_plan* plan, void* stream);
 
 /* df_decode_batch_run: decode every tensor of a prepared table in one launch
- * (one CUDA block per format block over all tensors; block -> tensor by a
- * binary search of the prefix sum of block counts). The workspace must hold
- * the prepared table until the launch has run. Errors: DF_ERR_INVALID_ARG,
- * DF_ERR_CUDA. */
+ * (persistent CUDA blocks over the format blocks of all tensors; block ->
+ * tensor by a binary search of the prefix sum of block counts). The
+ * workspace must hold the prepared table until the launch has run.
+ * Source: none on the pages (see df_decode_batch_prepare); per tensor as
+ * df_decode. Errors: DF_ERR_INVALID_ARG, DF_ERR_CUDA. */
 df_status df_decode_batch_run(const df_batch_plan* plan, uint32_t* d_err, void* stream);
 
-/* df_decode_batch: prepare + run. */
+/* df_decode_batch: prepare + run. Source: none on the pages (see
+ * df_decode_batch_prepare). */
 df_status df_decode_batch(const df_tensor* tensors, uint16_t* const* d_outs, uint32_t count, void* d_ws,
                           size_t ws_bytes, uint32_t* d_err, void* stream);
 
 /* df_read_error: wait for `stream`, copy the device error word to *flags
  * (nullable) and return DF_ERR_CORRUPT if any bit is set, else DF_OK.
+ * Source: df11pack, "Use" (a check reports pass, mismatch or could-not-check:
+ * here DF_OK, DF_ERR_CORRUPT, or another status).
  * Errors: DF_ERR_INVALID_ARG, DF_ERR_CUDA. */
 df_status df_read_error(const uint32_t* d_err, void* stream, uint32_t* flags);
 

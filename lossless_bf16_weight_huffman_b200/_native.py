@@ -30,6 +30,7 @@ DF_ENCODE_NOALLOC_MAX_WEIGHTS = 1 << 29
 # every function declared in include/df11.h
 EXPORTS = (
     "df_status_string", "df_last_cuda_error", "df_build_code", "df_code_from_lengths", "df_lut_words", "df_build_lut", "df_plan",
+    "df_container_sizes",
     "df_histogram", "df_encode", "df_encode_noalloc", "df_decode", "df_decode_batch_workspace", "df_decode_batch_prepare",
     "df_decode_batch_run", "df_decode_batch", "df_read_error",
 )
@@ -87,7 +88,7 @@ class DfBatchPlan(ctypes.Structure):
     _fields_ = [
         ("d_ws", ctypes.c_void_p),
         ("count", ctypes.c_uint32),
-        ("threads_per_block", ctypes.c_uint32),
+        ("cta_threads", ctypes.c_uint32),
         ("words_per_chunk", ctypes.c_uint32),
         ("region_bytes", ctypes.c_uint32),
         ("max_groups", ctypes.c_uint32),
@@ -129,6 +130,8 @@ def lib() -> ctypes.CDLL:
     L.df_build_lut.restype = i32
     L.df_plan.argtypes = [ctypes.POINTER(DfCode), vp, u64, u32, u32, ctypes.POINTER(DfSizes)]
     L.df_plan.restype = i32
+    L.df_container_sizes.argtypes = [u64, u64, u32, u32, ctypes.POINTER(DfSizes)]
+    L.df_container_sizes.restype = i32
     L.df_histogram.argtypes = [vp, u64, vp, vp]
     L.df_histogram.restype = i32
     L.df_encode.argtypes = [ctypes.POINTER(DfCode), vp, u64, u64, u32, u32, vp, vp, vp, vp, vp, sz, vp, vp]

@@ -36,31 +36,29 @@ def _need(t: torch.Tensor, nbytes: int, name: str) -> None:
         raise ValueError(f"{name} holds {have} bytes; the call writes {nbytes}")
 
 
-def _format_ok(chunk_bytes: int, threads_per_block: int) -> bool:
-    return (16 <= chunk_bytes <= 4096 and chunk_bytes % 16 == 0 and 32 <= threads_per_block <= 1024
-            and threads_per_block % 32 == 0)
+def _check_encode_buffers(n, total_bits, chunk_bytes, threads_per_block, d_in, d_stream, d_gaps, d_block_offsets,
+                          d_sm, d_err):
+    _need_u16(d_in, "d_in")
+    _need_err(d_err)
+    z = DfSizes()
+    if lib().df_container_sizes(n, total_bits, chunk_bytes, threads_per_block, ctypes.byref(z)) != 0:
+        return  # the library rejects these arguments itself
+    _need(d_stream, z.stream_bytes, "d_stream")
+    _need(d_gaps, z.gap_bytes, "d_gaps")
+    _need(d_block_offsets, z.offsets_bytes, "d_block_offsets")
+    _need(d_sm, z.sm_bytes, "d_sm")
 
 
-def container_layout(n: int, total_bits: int, chunk_bytes: int, threads_per_block: int) -> dict:
-    """Bytes of each buffer df_encode writes for n weights and total_bits code
-    bits (the container layout of include/df11.h; df_plan reports the same)."""
-    cbits = 8 * chunk_bytes
-    n_chunks = (total_bits + cbits - 1) // cbits if total_bits else 1
-    n_blocks = (n_chunks + threads_per_block - 1) // threads_per_block
-    return {"stream_bytes": n_chunks * chunk_bytes + 16,
-            "gap_bytes": (((5 * n_chunks + 7) // 8) + 1 + 15) & ~15,
-            "offsets_bytes": 8 * (n_blocks + 1),
-            "sm_bytes": n}
+def _need_u16(t: torch.Tensor, name: str) -> None:
+    """The library reads 2 bytes per element of a weight buffer."""
+    if isinstance(t, torch.Tensor) and t.element_size() != 2:
+        raise TypeError(f"{name} must hold 16-bit elements (BF16 bit patterns), got {t.dtype}")
 
 
-def _check_encode_buffers(n, total_bits, chunk_bytes, threads_per_block, d_stream, d_gaps, d_block_offsets, d_sm):
-    if not _format_ok(chunk_bytes, threads_per_block):
-        return  # the library rejects the format itself
-    z = container_layout(n, total_bits, chunk_bytes, threads_per_block)
-    _need(d_stream, z["stream_bytes"], "d_stream")
-    _need(d_gaps, z["gap_bytes"], "d_gaps")
-    _need(d_block_offsets, z["offsets_bytes"], "d_block_offsets")
-    _need(d_sm, z["sm_bytes"], "d_sm")
+def _need_err(d_err: torch.Tensor | None) -> None:
+    """The error word is a 32-bit word the kernels OR flags into."""
+    if d_err is not None:
+        _need(d_err, 4, "d_err")
 
 
 def _hist_array(hist) -> np.ndarray:
@@ -105,7 +103,14 @@ def df_build_lut(code: DfCode) -> np.ndarray:
     return out
 
 
-def df_plan(code: DfCode, hist, n: int, chunk_bytes: int = 32, threads_per_block: int = 256) -> DfSizes:
+def df_container_sizes(n: int, total_bits: int, chunk_bytes: int = 32, threads_per_block: int = 32) -> DfSizes:
+    z = DfSizes()
+    check("df_container_sizes", lib().df_container_sizes(n, total_bits, chunk_bytes, threads_per_block,
+                                                         ctypes.byref(z)))
+    return z
+
+
+def df_plan(code: DfCode, hist, n: int, chunk_bytes: int = 32, threads_per_block: int = 32) -> DfSizes:
     h = _hist_array(hist)
     z = DfSizes()
     check("df_plan", lib().df_plan(ctypes.byref(code), h.ctypes.data, n, chunk_bytes, threads_per_block,
@@ -114,6 +119,8 @@ def df_plan(code: DfCode, hist, n: int, chunk_bytes: int = 32, threads_per_block
 
 
 def df_histogram(d_in: torch.Tensor, d_hist256: torch.Tensor, stream=None) -> None:
+    _need_u16(d_in, "d_in")
+    _need(d_hist256, 256 * 8, "d_hist256")
     check("df_histogram", lib().df_histogram(_dev(d_in, "d_in"), d_in.numel(), _dev(d_hist256, "d_hist256"),
                                              _stream_ptr(stream)))
 
@@ -122,8 +129,8 @@ def df_encode(code: DfCode, d_in: torch.Tensor, total_bits: int, chunk_bytes: in
               d_stream: torch.Tensor, d_gaps: torch.Tensor, d_block_offsets: torch.Tensor, d_sm: torch.Tensor,
               d_ws: torch.Tensor, d_err: torch.Tensor | None = None, stream=None) -> None:
     ws_bytes = d_ws.numel() * d_ws.element_size() if d_ws is not None else 0
-    _check_encode_buffers(d_in.numel(), total_bits, chunk_bytes, threads_per_block, d_stream, d_gaps,
-                          d_block_offsets, d_sm)
+    _check_encode_buffers(d_in.numel(), total_bits, chunk_bytes, threads_per_block, d_in, d_stream, d_gaps,
+                          d_block_offsets, d_sm, d_err)
     check("df_encode", lib().df_encode(
         ctypes.byref(code), _dev(d_in, "d_in"), d_in.numel(), total_bits, chunk_bytes, threads_per_block,
         _dev(d_stream, "d_stream"), _dev(d_gaps, "d_gaps"), _dev(d_block_offsets, "d_block_offsets"),
@@ -136,8 +143,8 @@ def df_encode_noalloc(code: DfCode, d_in: torch.Tensor, total_bits: int, chunk_b
     """df_encode with the library's static scratch instead of a workspace
     (for callers that cannot allocate device memory; calls on one GPU must not
     overlap)."""
-    _check_encode_buffers(d_in.numel(), total_bits, chunk_bytes, threads_per_block, d_stream, d_gaps,
-                          d_block_offsets, d_sm)
+    _check_encode_buffers(d_in.numel(), total_bits, chunk_bytes, threads_per_block, d_in, d_stream, d_gaps,
+                          d_block_offsets, d_sm, d_err)
     check("df_encode_noalloc", lib().df_encode_noalloc(
         ctypes.byref(code), _dev(d_in, "d_in"), d_in.numel(), total_bits, chunk_bytes, threads_per_block,
         _dev(d_stream, "d_stream"), _dev(d_gaps, "d_gaps"), _dev(d_block_offsets, "d_block_offsets"),
@@ -147,6 +154,7 @@ def df_encode_noalloc(code: DfCode, d_in: torch.Tensor, total_bits: int, chunk_b
 def df_decode(t: DfTensor, d_out: torch.Tensor, d_err: torch.Tensor | None = None, stream=None) -> None:
     if isinstance(d_out, torch.Tensor):
         _need(d_out, 2 * t.n, "d_out")
+    _need_err(d_err)
     check("df_decode", lib().df_decode(ctypes.byref(t), _dev(d_out, "d_out"), _dev(d_err, "d_err"),
                                        _stream_ptr(stream)))
 
@@ -176,12 +184,14 @@ def df_decode_batch_prepare(tensors, d_outs, d_ws: torch.Tensor, stream=None) ->
 
 
 def df_decode_batch_run(plan: DfBatchPlan, d_err: torch.Tensor | None = None, stream=None) -> None:
+    _need_err(d_err)
     check("df_decode_batch_run", lib().df_decode_batch_run(ctypes.byref(plan), _dev(d_err, "d_err"),
                                                            _stream_ptr(stream)))
 
 
 def df_decode_batch(tensors, d_outs, d_ws: torch.Tensor, d_err: torch.Tensor | None = None, stream=None) -> None:
     arr, outs = _batch_arrays(tensors, d_outs)
+    _need_err(d_err)
     ws_bytes = d_ws.numel() * d_ws.element_size()
     check("df_decode_batch", lib().df_decode_batch(arr, outs, len(tensors), _dev(d_ws, "d_ws"), ws_bytes,
                                                    _dev(d_err, "d_err"), _stream_ptr(stream)))
@@ -189,6 +199,7 @@ def df_decode_batch(tensors, d_outs, d_ws: torch.Tensor, d_err: torch.Tensor | N
 
 def df_read_error(d_err: torch.Tensor, stream=None) -> int:
     """Return the device error word (0 = clean); waits for the stream."""
+    _need_err(d_err)
     flags = ctypes.c_uint32(0)
     status = lib().df_read_error(_dev(d_err, "d_err"), _stream_ptr(stream), ctypes.byref(flags))
     if status not in (0, 3):

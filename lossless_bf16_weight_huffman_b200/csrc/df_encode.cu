@@ -322,23 +322,32 @@ df_status sm_count(int* sms) {
 }
 
 // Scratch of df_encode_noalloc: per-tile bit counts and bases for at most
-// DF_ENCODE_NOALLOC_MAX_WEIGHTS weights, in a file-scope device array (2 MiB
-// + 32 bytes). Host code must not use the array's name as a device address;
-// noalloc_scratch() looks the address up once per device.
+// DF_ENCODE_NOALLOC_MAX_WEIGHTS weights, in a file-scope device array of
+// 16 * (tiles + 2) + 256 bytes (tiles = 2^29 / 4096): 2 MiB + 288 bytes, the
+// workspace df_encode asks for at that size. Host code must not use the
+// array's name as a device address; noalloc_scratch() looks the address up.
 constexpr uint64_t kNoAllocTiles = DF_ENCODE_NOALLOC_MAX_WEIGHTS / kTile;
 static __device__ __align__(256) uint64_t g_noalloc_scratch[2 * (kNoAllocTiles + 2) + 32];
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mutex;
 void* g_noalloc_address[kMaxDevices] = {};
 
-// The device address of the static scratch on the current device.
-df_status noalloc_scratch(void** out) {
+// The device address of the static scratch on the current device. Outside a
+// stream capture it is looked up on every call, so a device reset (after
+// which the module, and the array, may load elsewhere) never leaves a stale
+// address behind; during a capture the address of the last call on this
+// device is used (a lookup is not made while the stream captures).
+df_status noalloc_scratch(cudaStream_t s, void** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e);
     if (dev < 0 || dev >= kMaxDevices) return DF_ERR_UNSUPPORTED;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    e = cudaStreamIsCapturing(s, &cs);
+    if (e != cudaSuccess) return cuda_fail(e);
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (!g_noalloc_address[dev]) {
+    if (cs == cudaStreamCaptureStatusNone || !g_noalloc_address[dev]) {
+        if (cs != cudaStreamCaptureStatusNone) return DF_ERR_UNSUPPORTED;  // first call inside a capture
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess) return cuda_fail(e);
@@ -442,7 +451,7 @@ df_status df_encode_noalloc(const df_code* code, const uint16_t* d_in, uint64_t 
                             uint64_t* d_block_offsets, uint8_t* d_sm, uint32_t* d_err, void* stream) {
     if (n > DF_ENCODE_NOALLOC_MAX_WEIGHTS) return DF_ERR_UNSUPPORTED;
     void* ws = nullptr;
-    const df_status st = noalloc_scratch(&ws);
+    const df_status st = noalloc_scratch(static_cast<cudaStream_t>(stream), &ws);
     if (st != DF_OK) return st;
     return df_encode(code, d_in, n, total_bits, chunk_bytes, tpb, d_stream, d_gaps, d_block_offsets, d_sm, ws,
                      sizeof(g_noalloc_scratch), d_err, stream);

@@ -250,22 +250,17 @@ df_status df_build_lut(const df_code* code, uint32_t* lut, size_t lut_words) {
     return DF_OK;
 }
 
-df_status df_plan(const df_code* code, const uint64_t hist[256], uint64_t n, uint32_t chunk_bytes,
-                  uint32_t tpb, df_sizes* out) {
-    if (!code || !hist || !out || !valid_format(chunk_bytes, tpb)) return DF_ERR_INVALID_ARG;
+df_status df_container_sizes(uint64_t n, uint64_t total_bits, uint32_t chunk_bytes, uint32_t tpb,
+                             df_sizes* out) {
+    if (!out || !valid_format(chunk_bytes, tpb)) return DF_ERR_INVALID_ARG;
     if (n > DF_MAX_WEIGHTS) return DF_ERR_UNSUPPORTED;
-    uint64_t total = 0, bits = 0;
-    for (int s = 0; s < 256; ++s) {
-        if (hist[s] && !code->lengths[s]) return DF_ERR_INVALID_ARG;
-        total += hist[s];
-        bits += hist[s] * code->lengths[s];
-    }
-    if (total != n) return DF_ERR_INVALID_ARG;
+    // every code is at least one bit and at most 32 bits long
+    if (total_bits > 32 * n || (n && total_bits < n)) return DF_ERR_INVALID_ARG;
     df_sizes z;
     std::memset(&z, 0, sizeof(z));
     const uint64_t cbits = 8ull * chunk_bytes;
-    z.total_bits = bits;
-    z.n_chunks = bits ? (bits + cbits - 1) / cbits : 1;
+    z.total_bits = total_bits;
+    z.n_chunks = total_bits ? (total_bits + cbits - 1) / cbits : 1;
     z.stream_bytes = z.n_chunks * chunk_bytes + 16;
     const uint64_t field_bytes = (5 * z.n_chunks + 7) / 8;
     z.gap_bytes = (field_bytes + 1 + 15) & ~15ull;
@@ -278,6 +273,20 @@ df_status df_plan(const df_code* code, const uint64_t hist[256], uint64_t n, uin
     z.encode_ws_bytes = 16 * (tiles + 2) + 256;
     *out = z;
     return DF_OK;
+}
+
+df_status df_plan(const df_code* code, const uint64_t hist[256], uint64_t n, uint32_t chunk_bytes,
+                  uint32_t tpb, df_sizes* out) {
+    if (!code || !hist || !out || !valid_format(chunk_bytes, tpb)) return DF_ERR_INVALID_ARG;
+    if (n > DF_MAX_WEIGHTS) return DF_ERR_UNSUPPORTED;
+    uint64_t total = 0, bits = 0;
+    for (int s = 0; s < 256; ++s) {
+        if (hist[s] && !code->lengths[s]) return DF_ERR_INVALID_ARG;
+        total += hist[s];
+        bits += hist[s] * code->lengths[s];
+    }
+    if (total != n) return DF_ERR_INVALID_ARG;
+    return df_container_sizes(n, bits, chunk_bytes, tpb, out);
 }
 
 }  // extern "C"

@@ -2,8 +2,10 @@
 
 Records, for the small weight sets, the SHA-256 of each generated input and of
 each part of the oracle's container (stream, gaps, offsets, sign|fraction
-bytes, lengths). The GPU tests compare the CUDA encoder's bytes with these
-digests as well as with a fresh oracle run. Run from the repository root:
+bytes, lengths). tests/test_synth.py checks the input digests on the CPU;
+test_encode_matches_stored_oracle_digests (tests/test_gpu_parity.py) checks
+every part of the CUDA encoder's container against them. Run from the
+repository root:
 
     python tests/golden/make_golden.py
 """

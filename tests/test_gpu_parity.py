@@ -3,6 +3,10 @@ containers and the CUDA encoder against the oracle's bytes, element by element,
 on seeded inputs of several tiles with ragged tails, plus the edge cases of the
 method. Bit-exact is the only bar (integer work).
 """
+import hashlib
+import json
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -198,6 +202,32 @@ def test_encode_bytes_match_oracle(name):
     assert_container_equal(c, enc)
     out, flags = gpu_decode(c)
     assert flags == 0 and (out == w).all()
+
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "oracle_digests.json")
+
+
+def _sha(a: np.ndarray) -> str:
+    return hashlib.sha256(np.ascontiguousarray(a).tobytes()).hexdigest()
+
+
+def test_encode_matches_stored_oracle_digests():
+    """Every container part the CUDA encoder writes hashes to the SHA-256 the
+    oracle recorded for it (tests/golden/make_golden.py, oracle only), on the
+    recorded tensors of the small weight sets, with the recorded format."""
+    g = json.load(open(GOLDEN))
+    for t in g["tensors"]:
+        w = synth.generate(synth.weight_set(t["set"])[t["index"]])
+        assert _sha(w) == t["input_sha256"]
+        c = encode_on_gpu(w, t["max_len"], t["chunk_bytes"], t["threads_per_block"])
+        key = (t["set"], t["index"], t["max_len"])
+        assert c.total_bits == t["total_bits"], key
+        assert c.container_bytes == t["container_bytes"], key
+        assert _sha(np.frombuffer(bytes(c.code.lengths), np.uint8)) == t["lengths_sha256"], key
+        assert _sha(c.stream.cpu().numpy()) == t["stream_sha256"], key
+        assert _sha(c.gaps.cpu().numpy()) == t["gaps_sha256"], key
+        assert _sha(c.offsets.cpu().numpy().view(np.uint64)) == t["offsets_sha256"], key
+        assert _sha(c.sm[: c.n].cpu().numpy()) == t["sm_sha256"], key
 
 
 @pytest.mark.parametrize("max_len,chunk_bytes,tpb", [(12, 32, 256), (16, 16, 32), (32, 64, 128), (9, 48, 64)])

@@ -39,6 +39,19 @@ def test_library_exports_every_declared_function():
     assert sorted(_native.EXPORTS) == names
 
 
+def test_every_declaration_names_its_source():
+    """Each function declared in the header is preceded by a comment that
+    names the page passage it follows ("Source: ...") or says that the pages
+    have none."""
+    text = open(os.path.join(ROOT, "include", "df11.h")).read()
+    for name in header_functions():
+        m = re.search(r"/\*((?:(?!\*/).)*)\*/\s*(?:#define[^\n]*\n\s*)*[A-Za-z_][A-Za-z_0-9 *]*\b" + name + r"\(",
+                      text, flags=re.S)
+        assert m, name
+        comment = m.group(1)
+        assert "Source:" in comment or "no counterpart" in comment, name
+
+
 def test_struct_sizes_match_header_layout():
     import ctypes
 
@@ -262,7 +275,9 @@ def test_unreachable_entries_are_zero():
 # ---------------------------------------------------------------- the binding's buffer checks
 
 
-def test_binding_layout_matches_plan():
+def test_container_sizes_match_plan_and_oracle():
+    """df_container_sizes (the library's layout arithmetic, used by the binding
+    to size-check buffers) equals df_plan and the oracle's own size accounting."""
     rng = np.random.default_rng(7)
     for trial in range(400):
         h = _random_hist(rng, trial % 5)
@@ -271,12 +286,44 @@ def test_binding_layout_matches_plan():
         C = int(rng.choice([16, 32, 48, 64, 128, 1024, 4096]))
         T = int(rng.choice([32, 64, 96, 256, 1024]))
         z = api.df_plan(code, h, n, C, T).as_dict()
-        got = api.container_layout(n, z["total_bits"], C, T)
-        for key, val in got.items():
-            assert val == z[key], (trial, key)
+        got = api.df_container_sizes(n, z["total_bits"], C, T).as_dict()
+        assert got == z, trial
+        ref = oracle.sizes(n, z["total_bits"], C, T)
+        for key in ("total_bits", "n_chunks", "stream_bytes", "gap_bytes", "n_blocks", "offsets_bytes", "sm_bytes",
+                    "container_bytes"):
+            assert got[key] == ref[key], (trial, key)
     z = api.df_plan(api.df_build_code(np.zeros(256, np.uint64)), np.zeros(256, np.uint64), 0, 32, 256).as_dict()
-    got = api.container_layout(0, 0, 32, 256)
-    assert all(got[k] == z[k] for k in got)
+    assert api.df_container_sizes(0, 0, 32, 256).as_dict() == z
+    for bad in ((10, 9, 32, 32), (10, 321, 32, 32), (10, 20, 24, 32), (10, 20, 32, 48)):
+        with pytest.raises(_native.DfError):
+            api.df_container_sizes(*bad)
+
+
+def test_binding_refuses_wrong_element_sizes():
+    import torch
+
+    h = np.zeros(256, np.uint64)
+    h[120:124] = [50, 30, 15, 5]
+    code = api.df_build_code(h, 32)
+    z = api.df_plan(code, h, 100, 32, 32).as_dict()
+    bufs = dict(d_stream=torch.empty(z["stream_bytes"], dtype=torch.uint8),
+                d_gaps=torch.empty(z["gap_bytes"], dtype=torch.uint8),
+                d_block_offsets=torch.empty(z["n_blocks"] + 1, dtype=torch.int64),
+                d_sm=torch.empty(100, dtype=torch.uint8))
+    with pytest.raises(TypeError, match="d_in"):
+        api.df_encode(code, torch.zeros(100, dtype=torch.uint8), z["total_bits"], 32, 32,
+                      d_ws=torch.empty(16, dtype=torch.uint8), **bufs)
+    with pytest.raises(TypeError, match="d_in"):
+        api.df_encode_noalloc(code, torch.zeros(100, dtype=torch.int32), z["total_bits"], 32, 32, **bufs)
+    with pytest.raises(TypeError, match="d_in"):
+        api.df_histogram(torch.zeros(100, dtype=torch.uint8), torch.empty(256, dtype=torch.int64))
+    with pytest.raises(ValueError, match="d_err"):
+        api.df_encode(code, torch.zeros(100, dtype=torch.int16), z["total_bits"], 32, 32,
+                      d_ws=torch.empty(16, dtype=torch.uint8), d_err=torch.zeros(1, dtype=torch.uint8), **bufs)
+    d = _native.DfTensor()
+    d.n = 100
+    with pytest.raises(ValueError, match="d_err"):
+        api.df_decode(d, torch.empty(100, dtype=torch.int16), torch.zeros(2, dtype=torch.int8))
 
 
 def test_binding_refuses_short_buffers_before_the_library():
