@@ -158,12 +158,12 @@ size_t df_lut_words(const df_code* code);
 /* df_build_lut: derive the decode tables of a code into host memory `lut`
  * (lut_words >= df_lut_words(code)); the caller copies the words to the
  * device and passes them as df_tensor.lut. Layout, in order:
- *   - the wide table: 1024 uint64 indexed by the next 10 stream bits; an
+ *   - the wide table: 4096 uint64 indexed by the next 12 stream bits; an
  *     entry holds the exponents of the codes that lie wholly inside the
  *     window from its first bit on (up to 4, bits 0-31, the first in bits
  *     0-7) and, in bits 32-63, (bits they use << 18) | (their count << 3),
- *     or 0 when the first code is longer than 10 bits;
- *   - 1024 uint16: for each window, the mask of the window bits where those
+ *     or 0 when the first code is longer than 12 bits;
+ *   - 4096 uint16: for each window, the mask of the window bits where those
  *     codes start;
  *   - n_tables tables of 256 uint32 indexed by 8 stream bits, for codes of
  *     any length: a leaf holds the exponent (bits 0-7), the full code length

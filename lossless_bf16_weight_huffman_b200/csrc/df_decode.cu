@@ -51,8 +51,9 @@ constexpr uint32_t kWideN = 1u << kWideBits;
 constexpr uint32_t kFull = 0xFFFFFFFFu;
 constexpr uint32_t kLanes = 32;
 constexpr uint32_t kMaxWarps = 32;   // CUDA blocks of up to 1024 threads
-constexpr uint32_t kPosWords = 40;   // 33 stage positions, 3 spare, the 4-word carry
+constexpr uint32_t kPosWords = 72;   // 33 stage positions, 3 spare, the 4-word carry, 32 region bases
 constexpr uint32_t kCarryWord = 36;  // the carry's first word within them
+constexpr uint32_t kBaseWord = 40;   // the first region base
 constexpr uint32_t kRegionSlack = 12;  // up to 3 uncounted exponents and the word they end in
 constexpr uint32_t kSmemSlack = 32;  // gathers may read a few bytes past the last region
 // shared memory before the per-warp areas: the wide table, the current
@@ -120,13 +121,6 @@ __device__ __noinline__ uint32_t long_code(uint32_t win, const uint32_t* __restr
     return ((e >> kNsymShift) & 3u) ? e : 0;
 }
 
-// The 32 stream bits from bit p of a lane's chunk, whose big-endian words
-// are at w[0], w[32], w[64], ...
-__device__ __forceinline__ uint32_t window(const uint32_t* w, uint32_t p) {
-    const uint32_t* a = w + (p >> 5) * kLanes;
-    return __funnelshift_l(a[kLanes], a[0], p);
-}
-
 __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v, uint32_t lane) {
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
@@ -154,9 +148,17 @@ __device__ __forceinline__ void gather16(const uint8_t* base, int a, uint32_t e[
 
 // 4 BF16 weights from 4 sign|fraction bytes and 4 exponent bytes: the high
 // byte of weight k is s | e >> 1, the low byte (e & 1) << 7 | fraction.
+// Bit select: the bits of a where m is set, the bits of b elsewhere (one
+// three-input logic instruction).
+__device__ __forceinline__ uint32_t bitsel(uint32_t a, uint32_t b, uint32_t m) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xE4;" : "=r"(d) : "r"(a), "r"(b), "r"(m));
+    return d;
+}
+
 __device__ __forceinline__ void merge4(uint32_t s, uint32_t e, uint32_t* o0, uint32_t* o1) {
-    const uint32_t hi = (s & 0x80808080u) | ((e >> 1) & 0x7F7F7F7Fu);
-    const uint32_t lo = ((e << 7) & 0x80808080u) | (s & 0x7F7F7F7Fu);
+    const uint32_t hi = bitsel(s, e >> 1, 0x80808080u);
+    const uint32_t lo = bitsel(e << 7, s, 0x80808080u);
     *o0 = __byte_perm(lo, hi, 0x5140);
     *o1 = __byte_perm(lo, hi, 0x7362);
 }
@@ -175,76 +177,119 @@ __device__ __forceinline__ void merge16(const uint4 s16, const uint32_t e[4], ui
     __stcs(dst + 1, make_uint4(o[4], o[5], o[6], o[7]));
 }
 
+// Shared-memory accesses by 32-bit shared-window address.
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ void sts32(uint32_t a, uint32_t v) {
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t shared_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// The 32 stream bits from bit p of a lane's chunk, whose big-endian words
+// start at shared address wb, one word every 32 * 4 bytes.
+__device__ __forceinline__ uint32_t window_at(uint32_t wb, uint32_t p) {
+    const uint32_t a = wb + (p >> 5) * (kLanes * 4);
+    return __funnelshift_l(lds32(a + kLanes * 4), lds32(a), p);
+}
+
 // Decoder state of one lane: st = (bit position << 18) | (exponents appended
 // to the region << 3); acc holds the region word being filled (its
-// (st & 24) / 8 low bytes are exponents).
+// (st & 24) / 8 low bytes are exponents) and wp is that word's address.
 struct Lane {
     uint32_t st;
-    uint32_t end;  // codes must start before this bit
+    uint32_t endst;  // codes must start before bit endst >> 18: st < endst
     uint32_t acc;
+    uint32_t wp;
     bool bad;
 };
 
-// One lookup at the lane's bit position: up to 4 codes from the wide table,
-// or one longer code from the 8-bit tables. The region word being filled is
-// stored on every lookup (a later store of the same word supersedes it), and
-// the exponents that spill into the next word start the new accumulator.
-// (st & 31) is the byte shift of the next exponent in its word, so the two
-// funnel shifts place the new exponents without masking the state.
-__device__ __forceinline__ void step(Lane& L, const uint32_t* words, const uint64_t* wide, const uint32_t* hier,
-                                     uint32_t* region) {
-    const uint32_t win = window(words, L.st >> kStepShift);
-    const uint64_t e = wide[win >> (32 - kWideBits)];
-    uint32_t sy = static_cast<uint32_t>(e);
-    uint32_t w = static_cast<uint32_t>(e >> 32);
+// Append the exponents of one lookup (step word w, exponents sy) to the
+// lane's region. The region word being filled is stored on every lookup (a
+// later store of the same word supersedes it), and the exponents that spill
+// into the next word start the new accumulator. (st & 31) is the byte shift
+// of the next exponent in its word, so the two funnel shifts place the new
+// exponents without masking the state.
+__device__ __forceinline__ void append(Lane& L, uint32_t w, uint32_t sy) {
+    const uint32_t lo = L.acc | __funnelshift_l(0u, sy, L.st);
+    const uint32_t hi = __funnelshift_l(sy, 0u, L.st);
+    const uint32_t nst = L.st + w;
+    sts32(L.wp, lo);
+    // bit 5 of the state flips when the count enters the next region word
+    const uint32_t d = (nst ^ L.st) & 32u;
+    L.acc = __funnelshift_rc(lo, hi, d);
+    L.wp += d >> 3;
+    L.st = nst;
+}
+
+// One lookup at the lane's bit position: up to 4 codes from the wide table
+// (at shared address tb), or one longer code from the 8-bit tables.
+__device__ __forceinline__ void step(Lane& L, uint32_t wb, uint32_t tb, const uint32_t* hier) {
+    const uint32_t win = window_at(wb, L.st >> kStepShift);
+    const uint2 e = lds64(tb + (win >> (32 - kWideBits)) * 8u);
+    uint32_t sy = e.x, w = e.y;
     if (w == 0) {
         const uint32_t l = long_code(win, hier);
         sy = l & 0xFFu;
         w = l ? (((l >> 8) & 63u) << kStepShift) | (1u << kStepCountShift) : 0u;
         if (w == 0) {  // a bit pattern no code starts with
             L.bad = true;
-            L.end = 0;
+            L.endst = 0;
         }
     }
-    const uint32_t lo = L.acc | __funnelshift_l(0u, sy, L.st);
-    const uint32_t hi = __funnelshift_l(sy, 0u, L.st);
-    const uint32_t nst = L.st + w;
-    region[(L.st & kStepCountMask) >> 5] = lo;
-    // bit 5 of the state flips when the count enters the next region word
-    L.acc = __funnelshift_rc(lo, hi, (nst ^ L.st) & 32u);
-    L.st = nst;
+    append(L, w, sy);
 }
 
-// Decode one lane's chunk into its region, appending to what the region
-// already holds; returns the region's byte count with only the codes that
-// start before the chunk end (the exponents of codes past it are in the
-// region too, after the counted ones).
-__device__ __forceinline__ uint32_t decode_chunk(Lane& L, const uint32_t* words, const uint64_t* wide,
-                                                 const uint32_t* lut, uint32_t* region) {
+// Decode one lane's chunk (words at shared address wb) into its region
+// (shared address region), appending to what the region already holds: st
+// starts at (gap << 18) | (exponents already there << 3) and acc holds the
+// bytes of the region's last, unfinished word. Returns the region's byte
+// count with only the codes that start before the chunk end (bits
+// endst >> 18; the exponents of codes past it are in the region too, after
+// the counted ones), plus 1 << 31 for a bit pattern no code starts with.
+// Kept out of line: the lookup loop then runs in a register set of its own
+// instead of sharing one with the caller's bookkeeping.
+__device__ __noinline__ uint32_t decode_chunk(uint32_t st, uint32_t endst, uint32_t acc, uint32_t wb,
+                                              uint32_t region, uint32_t tb, const uint32_t* __restrict__ lut) {
     const uint32_t* hier = lut + kWideWords;
-    const uint32_t st0 = L.st;
-    uint32_t prev = L.st;  // the state before the last lookup
-    for (;;) {             // two lookups per vote
-        const bool act = (L.st >> kStepShift) < L.end;
+    Lane L;
+    L.st = st;
+    L.endst = endst;
+    L.acc = acc;
+    L.wp = region + ((st & kStepCountMask) >> 3 & ~3u);
+    L.bad = false;
+    uint32_t prev = st;  // the state before the last lookup
+    for (;;) {  // two lookups per vote
+        const bool act = L.st < L.endst;
         if (!__any_sync(kFull, act)) break;
         if (act) {
             prev = L.st;
-            step(L, words, wide, hier, region);
-            if ((L.st >> kStepShift) < L.end) {
+            step(L, wb, tb, hier);
+            if (L.st < L.endst) {
                 prev = L.st;
-                step(L, words, wide, hier, region);
+                step(L, wb, tb, hier);
             }
         }
     }
-    region[(L.st & kStepCountMask) >> 5] = L.acc;  // the word being filled
+    sts32(L.wp, L.acc);  // the word being filled
     uint32_t cnt = (L.st & kStepCountMask) >> kStepCountShift;
-    if (L.st != st0 && !L.bad) {  // every lookup advances the bit position
+    if (L.bad) return cnt | 0x80000000u;
+    if (L.st != st) {  // every lookup advances the bit position
         // codes of the last lookup that start at or after the chunk end
         const uint32_t p = prev >> kStepShift;
-        const uint32_t rel = L.end - p;
+        const uint32_t rel = (L.endst >> kStepShift) - p;
         if (rel < kWideBits) {
-            const uint32_t x = window(words, p) >> (32 - kWideBits);
-            if (wide[x] >> 32) {  // a wide-table lookup (a long code starts at p, before the end)
+            const uint32_t x = window_at(wb, p) >> (32 - kWideBits);
+            if (lds64(tb + x * 8u).y) {  // a wide-table lookup (a long code starts at p, before the end)
                 const uint16_t* mask = reinterpret_cast<const uint16_t*>(lut + kWideEntryWords);
                 cnt -= __popc(static_cast<uint32_t>(__ldg(mask + x)) >> rel);
             }
@@ -269,6 +314,7 @@ __global__ void __launch_bounds__(kMaxWarps * kLanes, 1)
     uint32_t* s_words = reinterpret_cast<uint32_t*>(wb);
     uint32_t* s_pos = s_words + kLanes * cfg.words_per_chunk;  // 33 stage positions
     uint32_t* s_carry = s_pos + kCarryWord;                     // 16 bytes: the group a round leaves open
+    int* s_base = reinterpret_cast<int*>(s_pos + kBaseWord);    // per lane: region byte of stage position 0
     uint8_t* s_owner = reinterpret_cast<uint8_t*>(s_pos + kPosWords);
     // lane 0's region starts 16 bytes early: it holds up to 15 carried
     // exponents before its own
@@ -353,15 +399,11 @@ __global__ void __launch_bounds__(kMaxWarps * kLanes, 1)
                 // 1. lane 0 starts from the exponents the previous round left
                 // open (stage positions [0, align)); at the start of a run they
                 // are placeholders for outputs of the previous run
-                Lane L;
-                L.st = 0;
-                L.end = 0;
-                L.acc = 0;
-                L.bad = false;
+                uint32_t st = 0, endst = 0, acc = 0;
                 if (lane == 0) {
                     *reinterpret_cast<uint4*>(my_region) = *reinterpret_cast<const uint4*>(s_carry);
-                    L.acc = s_carry[align >> 2] & ((1u << (8 * (align & 3))) - 1u);
-                    L.st = align << kStepCountShift;
+                    acc = s_carry[align >> 2] & ((1u << (8 * (align & 3))) - 1u);
+                    st = align << kStepCountShift;
                 }
                 // this lane's chunk and gap
                 const uint64_t chunk = c + lane;
@@ -386,13 +428,15 @@ __global__ void __launch_bounds__(kMaxWarps * kLanes, 1)
                     const uint32_t cbits = 8 * C;
                     const uint64_t bit0 = chunk * cbits;
                     const uint64_t rem = td->total_bits > bit0 ? td->total_bits - bit0 : 0;
-                    L.st += ((two >> (11 - (q & 7))) & 31u) << kStepShift;
-                    L.end = static_cast<uint32_t>(rem < cbits ? rem : cbits);
+                    st += ((two >> (11 - (q & 7))) & 31u) << kStepShift;
+                    endst = static_cast<uint32_t>(rem < cbits ? rem : cbits) << kStepShift;
                 }
                 pre = false;
 
                 // 2. decode: ext = the exponents in this lane's region
-                const uint32_t ext = decode_chunk(L, my_words, s_wide, td->lut, my_region);
+                const uint32_t dec = decode_chunk(st, endst, acc, shared_addr(my_words), shared_addr(my_region),
+                                                  shared_addr(s_wide), td->lut);
+                const uint32_t ext = dec & 0x7FFFFFFFu;
 
                 // the chunk of the next round into registers now; it goes into
                 // the slot after the scan
@@ -413,7 +457,7 @@ __global__ void __launch_bounds__(kMaxWarps * kLanes, 1)
                 const uint32_t incl = warp_incl_scan(ext, lane);
                 const uint32_t vend = __shfl_sync(kFull, incl, 31);  // positions [0, vend) hold exponents
                 const uint32_t total = vend - align;                  // codes of this round
-                const bool any_bad = __any_sync(kFull, L.bad);
+                const bool any_bad = __any_sync(kFull, dec >> 31);
                 uint32_t flags = 0;
                 if (any_bad)
                     flags = DF_EFLAG_BAD_CODE;
@@ -427,14 +471,18 @@ __global__ void __launch_bounds__(kMaxWarps * kLanes, 1)
                     break;
                 }
                 const uint32_t pos = incl - ext;
+                const int my_base = my_off - static_cast<int>(pos);  // stage position p is byte my_base + p
                 s_pos[lane] = pos;
+                s_base[lane] = my_base;
                 if (lane == 31) s_pos[32] = vend;
 
                 // 4. owner map: group gi (stage positions [16gi, 16gi+16))
-                // belongs to the lane whose range holds 16gi
+                // belongs to the lane whose range holds 16gi; bit 7 marks a
+                // group that runs past that range (merged in 5b)
                 if (ext) {
                     const uint32_t hi = pos + ext;
-                    for (uint32_t gi = (pos + 15) >> 4; 16 * gi < hi; ++gi) s_owner[gi] = static_cast<uint8_t>(lane);
+                    for (uint32_t gi = (pos + 15) >> 4; 16 * gi < hi; ++gi)
+                        s_owner[gi] = static_cast<uint8_t>(lane | (16 * gi + 16 > hi ? 0x80u : 0u));
                 }
                 if (nx) {  // only this lane reads its slot, and its decode is done
                     my_words[0 * kLanes] = bswap32(na.x);
@@ -453,57 +501,65 @@ __global__ void __launch_bounds__(kMaxWarps * kLanes, 1)
                 }
                 __syncwarp();
 
-                // 5. merge and store; stage position p <-> output gbase + p
+                // 5. merge and store; stage position p <-> output gbase + p,
+                // group gi <-> the 16 sign|fraction bytes at smg + 16gi
                 const uint64_t gbase = outr - align;
                 const uint64_t rend = outr + total;  // this round's outputs end here
                 const uint32_t ngroups = (vend + 15) >> 4;
-                // 5a. groups inside their owner's range; the others are left to
-                // 5b. Two groups per lane and iteration: both sign|fraction loads
-                // are in flight before the first merge.
-                for (uint32_t g0 = lane; g0 < ngroups; g0 += 2 * kLanes) {
-                    uint4 sv[2];
-#pragma unroll
-                    for (int k = 0; k < 2; ++k) {
-                        const uint32_t gi = g0 + k * kLanes;
-                        const uint64_t G = gbase + 16 * gi;
-                        sv[k] = make_uint4(0, 0, 0, 0);
-                        if (vec && gi < ngroups && G >= vstart && 16 * gi + 16 <= vend)
-                            sv[k] = __ldg(reinterpret_cast<const uint4*>(sm + G));
-                    }
-#pragma unroll
-                    for (int k = 0; k < 2; ++k) {
-                        const uint32_t gi = g0 + k * kLanes;
-                        if (gi >= ngroups) break;
-                        const uint32_t c0 = 16 * gi;
-                        const uint32_t t = s_owner[gi];
-                        if (c0 + 16 > s_pos[t + 1]) continue;
-                        const uint64_t G = gbase + c0;
+                const uint32_t gv0 = gbase < vstart ? 1u : 0u;      // group 0 may start before the run
+                const uint8_t* __restrict__ smg = sm + gbase;
+                uint16_t* __restrict__ outg = out + gbase;
+                // 5a. groups inside their owner's range (bit 7 of the owner byte
+                // clear); the others are merged in 5b. Two groups per lane and
+                // iteration: both sign|fraction loads are in flight first.
+                if (vec) {
+                    for (uint32_t g0 = lane; g0 < ngroups; g0 += 2 * kLanes) {
+                        const uint32_t g1 = g0 + kLanes;
+                        const uint32_t o0 = s_owner[g0];
+                        const uint32_t o1 = g1 < ngroups ? s_owner[g1] : 0x80u;
+                        const bool v0 = !(o0 & 0x80u) && g0 >= gv0;  // a run's first group is merged below
+                        const bool v1 = !(o1 & 0x80u);
+                        uint4 s0 = make_uint4(0, 0, 0, 0), s1 = make_uint4(0, 0, 0, 0);
+                        if (v0) s0 = __ldg(reinterpret_cast<const uint4*>(smg) + g0);
+                        if (v1) s1 = __ldg(reinterpret_cast<const uint4*>(smg) + g1);
                         uint32_t e[4];
-                        gather16(s_priv, region_off(t, RB) + static_cast<int>(c0 - s_pos[t]), e);
-                        if (vec && G >= vstart) {
-                            merge16(sv[k], e, out + G);
-                        } else {  // the run's first group, or buffers without 16-byte alignment
-                            for (uint32_t q = 0; q < 16; ++q) {
-                                const uint64_t i = G + q;
-                                if (i >= vstart) out[i] = merge1(sm[i], static_cast<uint8_t>(e[q >> 2] >> (8 * (q & 3))));
-                            }
+                        if (v0) {
+                            gather16(s_priv, s_base[o0 & 31u] + static_cast<int>(16 * g0), e);
+                            merge16(s0, e, outg + 16 * g0);
+                        }
+                        if (v1) {
+                            gather16(s_priv, s_base[o1 & 31u] + static_cast<int>(16 * g1), e);
+                            merge16(s1, e, outg + 16 * g1);
                         }
                     }
+                }
+                // a run's first group (it starts before the run's outputs), and
+                // every group of buffers without 16-byte alignment: element stores
+                for (uint32_t gi = vec ? (gv0 && lane == 0 ? 0u : ngroups) : lane; gi < ngroups; gi += kLanes) {
+                    const uint32_t o = s_owner[gi];
+                    if (o & 0x80u) continue;
+                    uint32_t e[4];
+                    gather16(s_priv, s_base[o & 31u] + static_cast<int>(16 * gi), e);
+                    for (uint32_t q = 0; q < 16; ++q) {
+                        const uint64_t i = gbase + 16 * gi + q;
+                        if (i >= vstart) out[i] = merge1(sm[i], static_cast<uint8_t>(e[q >> 2] >> (8 * (q & 3))));
+                    }
+                    if (vec) break;
                 }
                 // 5b. the group this lane's range ends inside, when it owns that
                 // group: it runs past the range into later regions, or it is the
                 // round's last group (kept open for the next round of the run)
                 const uint32_t bend = pos + ext;
-                if (ext && (bend & 15) && s_owner[bend >> 4] == lane) {
+                if (ext && (bend & 15) && (s_owner[bend >> 4] & 31u) == lane) {
                     const uint32_t c0 = bend & ~15u;
                     const uint64_t G = gbase + c0;
                     const uint32_t hi = min(c0 + 16, vend);
                     uint32_t e[4];
                     if (hi <= bend) {  // the round ends in this region
-                        gather16(s_priv, my_off + static_cast<int>(c0 - pos), e);
+                        gather16(s_priv, my_base + static_cast<int>(c0), e);
                     } else if (lane + 1 < kLanes && hi <= s_pos[lane + 2]) {  // this region and the next
                         uint32_t x[4], y[4];
-                        gather16(s_priv, my_off + static_cast<int>(c0 - pos), x);
+                        gather16(s_priv, my_base + static_cast<int>(c0), x);
                         gather16(s_priv, static_cast<int>((lane + 1) * RB) - static_cast<int>(bend - c0), y);
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {  // bytes before bend from x, the rest from y
@@ -516,7 +572,7 @@ __global__ void __launch_bounds__(kMaxWarps * kLanes, 1)
                         uint32_t t = lane;
                         for (uint32_t p = c0; p < hi; ++p) {
                             while (p >= s_pos[t + 1]) ++t;
-                            e[(p - c0) >> 2] |= static_cast<uint32_t>(s_priv[region_off(t, RB) + static_cast<int>(p - s_pos[t])])
+                            e[(p - c0) >> 2] |= static_cast<uint32_t>(s_priv[s_base[t] + static_cast<int>(p)])
                                                 << (8 * ((p - c0) & 3));
                         }
                     }
@@ -634,8 +690,8 @@ df_status device_limits(int* sms, int* max_smem, int* smem_per_sm) {
 }
 
 // Warps per CUDA block: as many resident warps per SM as shared memory allows
-// (at most 32, the register file's limit at 64 registers), with the fewest
-// warps per block among equals (a tensor switch then stalls fewer warps).
+// (at most 32, the register file's limit at 64 registers), with the most
+// warps per block among equals (one copy of the wide table serves them all).
 df_status choose_warps(const LaunchCfg& c, uint32_t* warps) {
     int sms = 0, max_smem = 0, per_sm = 0;
     df_status st = device_limits(&sms, &max_smem, &per_sm);
@@ -646,7 +702,7 @@ df_status choose_warps(const LaunchCfg& c, uint32_t* warps) {
         if (s > static_cast<size_t>(max_smem)) break;
         const uint32_t ctas = static_cast<uint32_t>(per_sm / (s + 1024));  // 1 KB reserved per block
         const uint32_t resident = std::min(ctas * w, kMaxWarps);
-        if (resident > best_resident) {
+        if (resident >= best_resident && resident > 0) {
             best = w;
             best_resident = resident;
         }

@@ -29,7 +29,7 @@ struct DevTensor {
 static_assert(sizeof(DevTensor) % 16 == 0, "descriptors are copied and placed in 16-byte units");
 
 // Decode tables (the words df_build_lut writes), in order:
-//   wide table, 1024 uint64 indexed by the next kWideBits = 10 stream bits:
+//   wide table, 4096 uint64 indexed by the next kWideBits = 12 stream bits:
 //     bits 0-31  the exponents of the codes that lie wholly inside the window,
 //                taken from its first bit on (at most 4; first in bits 0-7)
 //     bits 32-63 (bits used << 18) | (how many codes << 3); 0 when the first
@@ -37,7 +37,7 @@ static_assert(sizeof(DevTensor) % 16 == 0, "descriptors are copied and placed in
 //                (bit position << 18) | (codes so far << 3) advances by one
 //                add, and (state & 24) is the byte shift of the next exponent
 //                within a 32-bit word.
-//   wide start masks, 1024 uint16: bit i set when one of those codes starts
+//   wide start masks, 4096 uint16: bit i set when one of those codes starts
 //     at window bit i
 //   8-bit-indexed tables for codes of any length (root + next levels):
 //     leaf:  bits 0-7 the exponent, 8-13 its full code length, 24-25 = 1
@@ -45,7 +45,7 @@ static_assert(sizeof(DevTensor) % 16 == 0, "descriptors are copied and placed in
 //     unreachable: 0
 //   code lengths: 256 bytes
 //   header, 4 words: shortest code length, max_len, n_tables, kLutMagic
-constexpr uint32_t kWideBits = 10;
+constexpr uint32_t kWideBits = 12;
 constexpr uint32_t kWideMaxCodes = 4;
 constexpr uint32_t kStepShift = 18;                     // bits-used field of a step word
 constexpr uint32_t kStepCountMask = (1u << kStepShift) - 1;

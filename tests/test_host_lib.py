@@ -147,10 +147,12 @@ def wide_masks(lut, W):
 
 def table_walk_decode(stream, total_bits, n, gaps_fields, offsets, lut, n_tables, chunk_bytes, tpb):
     """Plain-Python model of the kernel's per-chunk decode: every chunk is
-    decoded from its start + gap up to its end; a wide-table step yields the
-    codes that lie wholly inside the next W bits (only those starting before
-    the chunk end are counted), a longer code walks the 8-bit tables; counts
-    are checked against the block offsets."""
+    decoded from its start + gap while the bit position is before its end; a
+    wide-table lookup yields every code that lies wholly inside the next W
+    bits, a longer code walks the 8-bit tables; the codes of a lookup that
+    start at or after the chunk end belong to the next chunk and are dropped
+    (the start mask gives their positions); counts are checked against the
+    block offsets."""
     WIDE = wide_bits(lut, n_tables)
     wide = wide_entries(lut, WIDE)
     masks = wide_masks(lut, WIDE)
@@ -169,8 +171,8 @@ def table_walk_decode(stream, total_bits, n, gaps_fields, offsets, lut, n_tables
             v = (v << 1) | int(b)
         return v << (32 - len(w))
 
-    def step(p, end, tail):
-        """One table step at bit p; returns (new p, codes counted)."""
+    def lookup(p):
+        """One table lookup at bit p: (bits used, [(start offset, exponent), ...])."""
         win = window(p)
         e = int(wide[win >> (32 - WIDE)])
         step_word = e >> 32
@@ -185,34 +187,23 @@ def table_walk_decode(stream, total_bits, n, gaps_fields, offsets, lut, n_tables
                 assert t != 0, "unreachable entry"
                 e = int(hier[t * 256 + ((win >> (24 - 8 * lvl)) & 0xFF)])
             assert (e >> 24) & 3 == 1
-            out.append(e & 0xFF)
-            return p + ((e >> 8) & 63), 1
+            return (e >> 8) & 63, [(0, e & 0xFF)]
         mask = int(masks[win >> (32 - WIDE)])
         assert bin(mask).count("1") << 3 == step_word & ((1 << 18) - 1)
-        lim = end - p if tail else WIDE
-        starts = [i for i in range(WIDE) if (mask >> i) & 1 and i < lim]
-        for k in range(len(starts)):
-            out.append(((e & 0xFFFFFFFF) >> (8 * k)) & 0xFF)
-        return p + used, len(starts)
+        starts = [i for i in range(WIDE) if (mask >> i) & 1]
+        return used, [(i, ((e & 0xFFFFFFFF) >> (8 * k)) & 0xFF) for k, i in enumerate(starts)]
 
     for j in range(n_chunks):
         p = j * cb + int(gaps_fields[j])
         end = min((j + 1) * cb, total_bits)
         cnt = 0
-        # the kernel's three phases: pairs of whole windows, whole windows,
-        # windows that reach past the chunk end
-        while p + 2 * WIDE <= end:
-            p, c = step(p, end, False)
-            cnt += c
-            if p + WIDE <= end:
-                p, c = step(p, end, False)
-                cnt += c
-        while p + WIDE <= end:
-            p, c = step(p, end, False)
-            cnt += c
         while p < end:
-            p, c = step(p, end, True)
-            cnt += c
+            used, codes = lookup(p)
+            for off, sym in codes:
+                if p + off < end:
+                    out.append(sym)
+                    cnt += 1
+            p += used
         counts.append(cnt)
     counts = np.array(counts)
     per_block = [int(counts[b * tpb:(b + 1) * tpb].sum()) for b in range(len(offsets) - 1)]
