@@ -10,16 +10,27 @@ weights, 16.06 GB) by ONE grouped launch (df_decode_batch_run) from the
 compressed containers resident in HBM into 16.06 GB of BF16 outputs. The inputs
 are far larger than L2, so no L2 flush is needed between steps.
 
-Also reported on the same line: the layer-by-layer decode into one reused
-buffer (34 grouped launches per pass), the GPU encode throughput, the
-end-to-end number through the public API from pinned host memory (compressed
-bytes host->device, decode, BF16 host<-device every step), the roofline of the
-decode kernel against the measured HBM copy bandwidth, the CPU oracle timed on
-a bounded sample, and the SM clocks sampled during the timed region.
+Also reported on the same line (N = 1 unless said otherwise):
+  configs         decode GB/s, weights/s, roofline fraction and compressed % of
+                  every weight set (single_1024x4096, llama_layer,
+                  heavy_tail_64m, llama8b_shaped, mixed_2000); sets that fit in
+                  L2 get an L2 flush before every timed step
+  layer_by_layer  the 8B-shaped set decoded layer by layer into reused buffers
+  jit_layer       per-step overhead of decoding each layer just in time, one or
+                  two layers ahead of a GEMM consumer, against BF16-resident
+                  weights
+  encode          device time of the GPU encoder, per call summed
+  e2e             through the public API from pinned host memory: containers
+                  copied in and BF16 copied out every step, overlapped with the
+                  decode layer by layer (every N)
+  roofline        the decode kernel against the measured HBM copy bandwidth
+  cpu_baseline    the oracle on the host cores, on a bounded sample
+  clocks          SM clocks sampled during the timed region
 
-With N > 1 (torchrun), every rank decodes its own copy of the weight set
-(weak scaling, no data-path collective); `value` = all ranks' bytes over the
-slowest rank's time.
+With N > 1 (torchrun), the tensors are partitioned over the ranks (balanced
+by the bytes each decode moves; no data-path collective, since tensors decode
+independently): every rank decodes its own share from its own HBM, `value` =
+all ranks' BF16 bytes over the slowest rank's time (strong scaling).
 
 --impl reference times the CPU oracle (the plain single-threaded decoder) on
 the host cores on a bounded sample of the same workload, same metric and unit.
@@ -30,6 +41,7 @@ import argparse
 import hashlib
 import json
 import os
+import platform
 import statistics
 import subprocess
 import sys
@@ -47,6 +59,8 @@ WORKLOAD = ("llama8b_shaped: 32 Llama-style decoder layers (q/o 4096x4096, k/v 1
             "down 4096x14336, 2 RMSNorm 4096) + embedding and lm_head 128256x4096; 8,030,257,152 BF16 weights "
             "(16.06 GB); decoded whole by one grouped launch")
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0
+SMALL_SETS = ("single_1024x4096", "heavy_tail_64m", "mixed_2000")
 
 
 def log(*a):
@@ -56,17 +70,21 @@ def log(*a):
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--steps", type=int, default=50)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--e2e-steps", type=int, default=2)
     p.add_argument("--workload", default="llama8b_shaped",
                    choices=["llama8b_shaped", "llama_layer", "single_1024x4096", "heavy_tail_64m", "mixed_2000"],
-                   help="weight set to decode (the headline number is llama8b_shaped)")
+                   help="weight set of the headline number (llama8b_shaped by default)")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-extras", action="store_true",
+                   help="headline only: skip the per-set records, layer-by-layer and jit_layer")
+    p.add_argument("--jit-tokens", type=int, default=4096, help="activation rows of the jit_layer GEMM consumer")
+    p.add_argument("--jit-layers", type=int, default=32, help="decoder layers in the jit_layer measurement")
     p.add_argument("--chunk-bytes", type=int, default=0,
                    help="format chunk size C in bytes (0: 32, or 16 where the shortest code is 1 bit)")
-    p.add_argument("--threads-per-block", type=int, default=256, help="format block size T in chunks")
+    p.add_argument("--threads-per-block", type=int, default=32, help="format block size T in chunks")
     return p.parse_args()
 
 
@@ -90,15 +108,23 @@ def _cuda_ok():
     return torch.cuda.is_available()
 
 
-def max_over_ranks(x: float, world: int, device=None) -> float:
+def _reduce(x: float, world: int, device, op: str) -> float:
     if world <= 1:
         return x
     import torch
     import torch.distributed as dist
 
     t = torch.tensor([x], dtype=torch.float64, device=device)
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
     return float(t.item())
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    return _reduce(x, world, device, "max")
+
+
+def sum_over_ranks(x: float, world: int, device=None) -> float:
+    return _reduce(x, world, device, "sum")
 
 
 def barrier(world: int):
@@ -191,8 +217,8 @@ def source_digest(paths):
 
 
 def decode_traffic_record():
-    """ncu DRAM bytes per weight for the decode kernel, if captured for the
-    current kernel source (profiles/decode_traffic.json)."""
+    """ncu DRAM bytes of one decode launch, if captured for the current kernel
+    source (profiles/decode_traffic.json), with the workload it was taken on."""
     path = os.path.join(ROOT, "profiles", "decode_traffic.json")
     src = os.path.join(ROOT, "lossless_bf16_weight_huffman_b200", "csrc", "df_decode.cu")
     try:
@@ -205,6 +231,8 @@ def decode_traffic_record():
 
 
 # ---------------------------------------------------------------------------------------------
+# the oracle on the host cores (reference arm and cpu_baseline); test infrastructure, never on
+# the GPU path
 
 
 def run_reference(args, world, rank):
@@ -231,7 +259,7 @@ def run_reference(args, world, rank):
     line = {
         "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(1e3 * total / args.steps, 3), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "u8", "data": "synthetic", "impl": "reference",
+        "scaling": "strong", "vs_baseline": None, "dtype": "u8", "data": "synthetic", "impl": "reference",
         "config": {"workload": WORKLOAD, "sample": "layers.0.q_proj (16,777,216 weights) per step",
                    "parallelism": "host, single thread"},
         "compressed_pct": round(100.0 * enc.container_bytes / (2 * w.size), 3),
@@ -242,54 +270,92 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
-def cpu_baseline_sample(specs):
-    """The oracle decoder (single thread) on layer 0 of the weight set."""
+def _oracle_job(job):
+    """One tensor through the oracle in a worker process: (weights, encode s, decode s)."""
+    set_name, index = job
     import oracle
     from lossless_bf16_weight_huffman_b200 import synth
 
-    layer0 = [s for s in specs if s.name.startswith("layers.0.")]
-    if not layer0:  # another weight set: its first tensors, up to ~2e8 weights
-        layer0, tot = [], 0
-        for s in specs:
-            if tot >= 200_000_000:
-                break
-            layer0.append(s)
-            tot += s.numel
-    encs = []
-    for s in layer0:
-        w = synth.generate(s)
-        encs.append((w, oracle.encode(w)))
-    n = sum(w.size for w, _ in encs)
+    w = synth.generate(synth.weight_set(set_name)[index])
     t0 = time.perf_counter()
-    for w, e in encs:
-        out = oracle.decode_encoded(e)
-        assert (out == w).all()
-    dt = time.perf_counter() - t0
-    return {"value": round(2 * n / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"{'layer 0' if layer0[0].name.startswith('layers.0.') else 'first tensors'} of the "
-                      f"weight set ({n:,} weights), bit-serial decode, one host thread, "
-                      f"{dt:.1f} s"}
+    enc = oracle.encode(w)
+    t1 = time.perf_counter()
+    out = oracle.decode_encoded(enc)
+    t2 = time.perf_counter()
+    if not (out == w).all():
+        raise RuntimeError(f"oracle round trip failed on {set_name}[{index}]")
+    return int(w.size), t1 - t0, t2 - t1
 
 
-def run_gpu(args, world, rank, local):
+def _cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return platform.processor() or "unknown"
+
+
+def cpu_baseline(pool, ncores):
+    """The oracle encoder and decoder on bounded samples of every weight set,
+    one process (one host thread) per tensor across all host cores; a
+    worker's own times give the one-thread rates. The 8B-shaped set is
+    extrapolated from a decoder layer (same shapes and distributions) by
+    weight count."""
+    from lossless_bf16_weight_huffman_b200 import synth
+
+    samples = {
+        "single_1024x4096": [("single_1024x4096", 0)],
+        "llama_layer": [("llama_layer", i) for i in range(len(synth.llama_layer()))],
+        "heavy_tail_64m": [("heavy_tail_64m", 0)],
+        "mixed_2000": [("mixed_2000", i) for i in range(0, 2000, 8)],  # every 8th tensor
+    }
+    per = {}
+    for name, jobs in samples.items():
+        t0 = time.perf_counter()
+        multi = pool.map(_oracle_job, jobs)
+        wall = time.perf_counter() - t0
+        n = sum(m[0] for m in multi)
+        rec = {"weights": n, "all_cores_wall_s": round(wall, 3),
+               "all_cores_gbs_roundtrip": round(2 * n / wall / 1e9, 4)}
+        # every worker is one host thread: the sum of its times is the
+        # one-thread time
+        enc_s = sum(m[1] for m in multi)
+        dec_s = sum(m[2] for m in multi)
+        rec.update({"one_thread_encode_gbs": round(2 * n / enc_s / 1e9, 4),
+                    "one_thread_decode_gbs": round(2 * n / dec_s / 1e9, 4),
+                    "one_thread_weights_per_s": round(n / dec_s, 1)})
+        if name == "mixed_2000":
+            rec["sample"] = "every 8th tensor (250 of 2000)"
+        per[name] = rec
+    layer = per["llama_layer"]
+    return {
+        "value": layer["one_thread_decode_gbs"], "unit": "GB/s", "cores": 1, "kind": "oracle",
+        "sample": "decoder layer (218,112,000 weights of the 8B shapes), bit-serial decode, one host thread; "
+                  "8B-shaped set extrapolated by weight count",
+        "host": {"nproc": ncores, "cpu_model": _cpu_model()},
+        "all_cores": {"value": layer["all_cores_gbs_roundtrip"], "unit": "GB/s (encode + decode round trip)",
+                      "cores": min(ncores, len(synth.llama_layer())),
+                      "how": "one process per tensor (spawned before the first GPU call)"},
+        "per_set": per,
+    }
+
+
+# ---------------------------------------------------------------------------------------------
+# GPU side
+
+
+def encode_set(specs, dev, args, staging):
+    """Generate each tensor on the host, copy it to HBM and encode it there.
+    Returns (source tensors, containers, histogram device ms, encode device ms):
+    the device times are CUDA events around every df_histogram / df_encode call,
+    summed (host work between calls is not counted)."""
     import numpy as np
     import torch
 
-    from lossless_bf16_weight_huffman_b200 import api, build, codec, synth
+    from lossless_bf16_weight_huffman_b200 import api, codec, synth
 
-    build.build_all()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    stream = torch.cuda.current_stream()
-    specs = synth.weight_set(args.workload)
-    n_total = sum(s.numel for s in specs)
-    max_n = max(s.numel for s in specs)
-
-    # ---- generate on the host, copy to HBM, encode on the GPU. The histograms of all
-    # tensors run back to back (one timed region), then the host builds every code, then
-    # all encodes run back to back (another timed region).
-    t_setup = time.time()
-    staging = torch.empty(max_n, dtype=torch.int16, pin_memory=True)
     src = []
     for s in specs:
         n = s.numel
@@ -299,199 +365,339 @@ def run_gpu(args, world, rank, local):
         torch.cuda.synchronize()  # the staging buffer is refilled next
         src.append(x)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
     hist_d = torch.empty((len(specs), 256), dtype=torch.int64, device=dev)
-    ev[0].record()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in specs]
     for i, x in enumerate(src):
+        ev[i][0].record()
         api.df_histogram(x, hist_d[i])
-    ev[1].record()
+        ev[i][1].record()
     hists = hist_d.cpu().numpy().view(np.uint64)
+    hist_ms = sum(a.elapsed_time(b) for a, b in ev)
     plans = []
-    for i, (s, x) in enumerate(zip(specs, src)):
+    for i, s in enumerate(specs):
         code = api.df_build_code(hists[i], 32)
         C = args.chunk_bytes or codec.auto_chunk_bytes(code)
-        TPB = args.threads_per_block
+        T = args.threads_per_block
         lut = torch.from_numpy(api.df_build_lut(code).view(np.int32)).to(dev)
-        z = api.df_plan(code, hists[i], s.numel, C, TPB).as_dict()
+        z = api.df_plan(code, hists[i], s.numel, C, T).as_dict()
         bufs = dict(stream=torch.empty(z["stream_bytes"], dtype=torch.uint8, device=dev),
                     gaps=torch.empty(z["gap_bytes"], dtype=torch.uint8, device=dev),
                     offsets=torch.empty(z["n_blocks"] + 1, dtype=torch.int64, device=dev),
-                    sm=torch.empty(s.numel, dtype=torch.uint8, device=dev))
-        plans.append((code, C, TPB, lut, z, bufs))
+                    sm=torch.empty(max(s.numel, 16), dtype=torch.uint8, device=dev))
+        plans.append((code, C, T, lut, z, bufs))
     ws = torch.empty(max(p[4]["encode_ws_bytes"] for p in plans), dtype=torch.uint8, device=dev)
     torch.cuda.synchronize()
-    ev[2].record()
-    for x, (code, C, TPB, lut, z, bufs) in zip(src, plans):
-        api.df_encode(code, x, z["total_bits"], C, TPB, bufs["stream"], bufs["gaps"], bufs["offsets"], bufs["sm"],
+    for i, (x, (code, C, T, lut, z, bufs)) in enumerate(zip(src, plans)):
+        ev[i][0].record()
+        api.df_encode(code, x, z["total_bits"], C, T, bufs["stream"], bufs["gaps"], bufs["offsets"], bufs["sm"],
                       ws, err)
-    ev[3].record()
+        ev[i][1].record()
     torch.cuda.synchronize()
-    hist_ms = ev[0].elapsed_time(ev[1])
-    enc_ms = ev[2].elapsed_time(ev[3])
-    del ws
-    comps = [codec.Compressed(n=s.numel, shape=s.shape, code=code, lut=lut, sizes=z, chunk_bytes=C,
-                              threads_per_block=TPB, **bufs)
-             for s, (code, C, TPB, lut, z, bufs) in zip(specs, plans)]
+    enc_ms = sum(a.elapsed_time(b) for a, b in ev)
     assert api.df_read_error(err) == 0, "encode reported an error"
+    comps = [codec.Compressed(n=s.numel, shape=s.shape, code=code, lut=lut, sizes=z, chunk_bytes=C,
+                              threads_per_block=T, **bufs)
+             for s, (code, C, T, lut, z, bufs) in zip(specs, plans)]
+    return src, comps, hist_ms, enc_ms
+
+
+def time_launches(run, steps, warmup, stream, flush=None):
+    """Per-step device ms of run() (CUDA events on `stream`). With `flush`, a
+    write larger than L2 precedes every step, outside its events."""
+    import torch
+
+    for _ in range(max(warmup, 1)):
+        run()
+    torch.cuda.synchronize()
+    if flush is None:
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+        evs[0].record(stream)
+        for k in range(steps):
+            run()
+            evs[k + 1].record(stream)
+        torch.cuda.synchronize()
+        return [evs[k].elapsed_time(evs[k + 1]) for k in range(steps)]
+    pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in pairs:
+        flush.zero_()
+        a.record(stream)
+        run()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in pairs]
+
+
+def verify(src, outs, names):
+    import torch
+
+    for x, o, name in zip(src, outs, names):
+        if not torch.equal(x, o.view(torch.int16).reshape(-1)):
+            raise SystemExit(f"decode mismatch on {name}")
+
+
+def decode_record(comps, outs, args, stream, err, peak, flush):
+    """Decode timing of one grouped launch over `comps`: GB/s of BF16 out,
+    weights/s, roofline fraction of the algorithmic bytes."""
+    from lossless_bf16_weight_huffman_b200 import api, codec
+
+    dec = codec.BatchDecoder(comps, outs)
+    n = sum(c.n for c in comps)
+    read = sum(c.read_bytes() for c in comps)
+    use_flush = flush is not None and read + 2 * n <= L2_FLUSH_BELOW
+    ms = time_launches(lambda: dec.run(err, stream), args.steps, args.warmup, stream, flush if use_flush else None)
+    assert api.df_read_error(err) == 0
+    med = statistics.median(ms)
+    algo = read + 2 * n
+    return {"gbs": round(2 * n / med / 1e6, 2), "weights_per_s": round(n / med * 1e3, 1),
+            "ms": round(med, 4), "roofline_frac": round(algo / med / 1e6 / peak, 4),
+            "compressed_pct": round(100.0 * sum(c.container_bytes for c in comps) / (2 * n), 4),
+            "weights": n, "tensors": len(comps),
+            "l2": "flushed before every step" if use_flush else "inputs larger than L2: no flush"}
+
+
+def layer_groups(specs, idx):
+    """Indices (into idx) grouped by decoder layer; every other tensor alone."""
+    groups = []
+    for j, i in enumerate(idx):
+        parts = specs[i].name.split(".")
+        key = ".".join(parts[:2]) if parts[0] == "layers" else None
+        if key is not None and groups and groups[-1][0] == key:
+            groups[-1][1].append(j)
+        else:
+            groups.append((key, [j]))
+    return groups
+
+
+def jit_record(args, specs, idx, comps, outs, err, dev):
+    """Per-pass time of a GEMM consumer over the decoder layers with weights
+    (a) resident as BF16, (b) decoded just in time at run-ahead depth 0, 1, 2."""
+    import torch
+
+    from lossless_bf16_weight_huffman_b200 import jit
+
+    groups = [(k, g) for k, g in layer_groups(specs, idx) if k is not None][: args.jit_layers]
+    if not groups:
+        return None
+    B = args.jit_tokens
+    layer_specs = [[specs[idx[j]] for j in g] for _, g in groups]
+    ins = sorted({s.shape[1] for l in layer_specs for s in l if len(s.shape) == 2})
+    outs_f = sorted({s.shape[0] for l in layer_specs for s in l if len(s.shape) == 2})
+    gen = torch.Generator(device=dev).manual_seed(0xDF11)
+    x_in = {k: torch.randn(B, k, generator=gen, device=dev, dtype=torch.float32).to(torch.bfloat16) for k in ins}
+    y_out = {k: torch.empty(B, k, device=dev, dtype=torch.bfloat16) for k in outs_f}
+    flops = sum(2 * B * s.numel for l in layer_specs for s in l if len(s.shape) == 2)
+
+    def consume(l, views):
+        for s, v in zip(layer_specs[l], views):
+            if len(s.shape) != 2:
+                continue
+            w = v.view(torch.bfloat16).view(s.shape[0], s.shape[1])
+            torch.matmul(x_in[s.shape[1]], w.t(), out=y_out[s.shape[0]])
+
+    resident = [[outs[j] for j in g] for _, g in groups]
+
+    def timed(fn, reps=3):
+        fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+
+    t_res = timed(lambda: [consume(l, resident[l]) for l in range(len(groups))])
+    layers = [[comps[j] for j in g] for _, g in groups]
+    rec = {"consumer": f"per layer, y = x W^T for each linear weight (cuBLAS bf16), x: {B} rows",
+           "layers": len(groups), "tokens": B, "gemm_tflops_resident": round(flops / t_res / 1e9, 1),
+           "resident_ms_per_pass": round(t_res, 3)}
+    for depth in (0, 1, 2):
+        st = jit.LayerStreamer(layers, depth=depth, device=dev)
+        t = timed(lambda: st.run(consume))
+        assert st.errors() == 0
+        rec[f"depth{depth}_ms_per_pass"] = round(t, 3)
+        rec[f"depth{depth}_overhead_pct"] = round(100.0 * (t - t_res) / t_res, 2)
+        del st
+    # the decode alone, layer by layer, for scale
+    st = jit.LayerStreamer(layers, depth=0, device=dev)
+    rec["decode_alone_ms_per_pass"] = round(timed(lambda: st.run(lambda l, v: None)), 3)
+    # check the just-in-time weights against the resident ones on the last layer
+    st1 = jit.LayerStreamer(layers, depth=1, device=dev)
+    seen = {}
+    st1.run(lambda l, v: seen.__setitem__(l, [t.clone() for t in v]) if l == len(groups) - 1 else None)
+    torch.cuda.synchronize()
+    for a, b in zip(seen[len(groups) - 1], resident[-1]):
+        if not torch.equal(a, b.view(torch.int16).reshape(-1)):
+            raise SystemExit("jit_layer decode differs from the resident weights")
+    return rec
+
+
+def e2e_record(args, specs, idx, comps, src, dev, world):
+    """Through the public API from pinned host memory: per layer, the container
+    parts are copied in on a copy stream, decoded on a decode stream and the
+    BF16 copied back out to pinned host buffers on the consumer's stream; the
+    three overlap across layers (jit.HostLayerStreamer)."""
+    import torch
+
+    from lossless_bf16_weight_huffman_b200 import jit
+
+    groups = layer_groups(specs, idx)
+    layers = [[comps[j] for j in g] for _, g in groups]
+    hls = jit.HostLayerStreamer(layers, device=dev)
+    cap = max(sum(c.n for c in l) for l in layers)
+    host_out = [torch.empty(cap, dtype=torch.int16, pin_memory=True) for _ in range(2)]
+
+    def consume(i, views):
+        off, dst = 0, host_out[i % 2]
+        for v in views:
+            dst[off: off + v.numel()].copy_(v, non_blocking=True)
+            off += v.numel()
+
+    hls.run(consume)
+    torch.cuda.synchronize()
+    assert hls.errors() == 0
+    last = groups[-1][1]
+    off = 0
+    for j in last:
+        if not torch.equal(host_out[(len(groups) - 1) % 2][off: off + comps[j].n], src[j].cpu()):
+            raise SystemExit("e2e output mismatch")
+        off += comps[j].n
+    barrier(world)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.perf_counter()
+    a.record()
+    for _ in range(args.e2e_steps):
+        hls.run(consume)
+    b.record()
+    torch.cuda.synchronize()
+    wall = (time.perf_counter() - t0) / args.e2e_steps
+    ms = max_over_ranks(a.elapsed_time(b) / args.e2e_steps, world, dev)
+    n_all = sum_over_ranks(sum(c.n for c in comps), world, dev)
+    return {"value": round(2 * n_all / (ms / 1e3) / 1e9, 3), "unit": "GB/s",
+            "h2d_bytes_per_step": int(sum_over_ranks(hls.h2d_bytes, world, dev)),
+            "d2h_bytes_per_step": int(2 * n_all), "ms_per_step": round(ms, 2), "wall_s": round(wall, 3),
+            "how": "jit.HostLayerStreamer: per layer, pinned host container -> HBM on a copy stream, "
+                   "df_decode_batch_run on a decode stream, BF16 -> pinned host on the consumer stream; "
+                   "consecutive layers overlap"}
+
+
+def run_gpu(args, world, rank, local, pool, ncores):
+    import torch
+
+    from lossless_bf16_weight_huffman_b200 import build, codec, shard, synth
+
+    build.build_all()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    peak, peak_src = measured_hbm_peak()
+    all_specs = synth.weight_set(args.workload)
+    parts = shard.partition([s.numel for s in all_specs], world)
+    idx = parts[rank]
+    specs = [all_specs[i] for i in idx]
+    n_all = sum(s.numel for s in all_specs)
+    n_mine = sum(s.numel for s in specs)
+
+    # ---- this rank's share: generated on the host, encoded on the GPU
+    t_setup = time.time()
+    staging = torch.empty(max([s.numel for s in specs] + [1]), dtype=torch.int16, pin_memory=True)
+    src, comps, hist_ms, enc_ms = encode_set(specs, dev, args, staging)
     container = sum(c.container_bytes for c in comps)
     read_bytes = sum(c.read_bytes() for c in comps)
-    log(f"[rank {rank}] setup {time.time() - t_setup:.1f} s: {len(specs)} tensors, {n_total:,} weights, "
-        f"container {100 * container / (2 * n_total):.3f}% of BF16")
+    log(f"[rank {rank}] setup {time.time() - t_setup:.1f} s: {len(specs)} of {len(all_specs)} tensors, "
+        f"{n_mine:,} weights, container {100 * container / (2 * max(n_mine, 1)):.3f}% of BF16")
 
-    # ---- (i) whole-set decode: one grouped launch per step
+    # ---- (i) the share decoded by one grouped launch per step
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
     outs = [torch.empty(c.n, dtype=torch.int16, device=dev) for c in comps]
     dec = codec.BatchDecoder(comps, outs)
-    for _ in range(max(args.warmup, 1)):
-        dec.run(err)
+    dec.run(err)
     torch.cuda.synchronize()
-    assert api.df_read_error(err) == 0, "decode reported an error"
-    for x, o, s in zip(src, outs, specs):
-        if not torch.equal(x, o):
-            raise SystemExit(f"decode mismatch on {s.name}")
+    assert codec.api.df_read_error(err) == 0, "decode reported an error"
+    verify(src, outs, [s.name for s in specs])
     log(f"[rank {rank}] decode verified bit-exact on all {len(specs)} tensors")
-
-    # inputs that fit in L2 (the small weight sets) get an L2 flush before every
-    # step, outside the timed events; the 8B-shaped set touches 26.7 GB per step
     flush = None
-    if read_bytes + 2 * n_total <= L2_FLUSH_BELOW:
+    if read_bytes + 2 * n_mine <= L2_FLUSH_BELOW:
         flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     clocks = ClockSampler(local)
     barrier(world)
     torch.cuda.synchronize()
     clocks.start()
-    if flush is None:
-        evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
-        evs[0].record(stream)
-        for k in range(args.steps):
-            dec.run(err, stream)
-            evs[k + 1].record(stream)
-        torch.cuda.synchronize()
-        step_ms = [evs[k].elapsed_time(evs[k + 1]) for k in range(args.steps)]
-        total_ms = evs[0].elapsed_time(evs[-1])
-    else:
-        pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                 for _ in range(args.steps)]
-        for a, b in pairs:
-            flush.zero_()
-            a.record(stream)
-            dec.run(err, stream)
-            b.record(stream)
-        torch.cuda.synchronize()
-        step_ms = [a.elapsed_time(b) for a, b in pairs]
-        total_ms = sum(step_ms)
+    step_ms = time_launches(lambda: dec.run(err, stream), args.steps, args.warmup, stream, flush)
     barrier(world)
     clk = clocks.stop()
-    total_ms_max = max_over_ranks(total_ms, world, dev)
-    assert api.df_read_error(err) == 0
+    assert codec.api.df_read_error(err) == 0
+    total_ms_max = max_over_ranks(sum(step_ms), world, dev)
     ms_per_step = total_ms_max / args.steps
-    bf16_bytes = 2 * n_total
-    value = world * bf16_bytes * args.steps / (total_ms_max / 1e3) / 1e9
-
-    # roofline of the decode kernel (one launch per step)
-    peak, peak_src = measured_hbm_peak()
-    algo_bytes = read_bytes + bf16_bytes
-    enc_algo = 2 * bf16_bytes + n_total + sum(c.sizes["stream_bytes"] for c in comps)
+    value = 2 * n_all * args.steps / (total_ms_max / 1e3) / 1e9
+    container_all = sum_over_ranks(container, world, dev)
+    algo_bytes = read_bytes + 2 * n_mine
     launch_ms = statistics.mean(step_ms)
     achieved = algo_bytes / (launch_ms / 1e3) / 1e9
-    traffic = None
     rec = decode_traffic_record()
-    if rec and args.workload == "llama8b_shaped":
-        traffic = int(rec["dram_bytes_per_weight"] * n_total)
+    traffic = None
+    if rec and rec.get("workload") == args.workload and world == 1:
+        traffic = int(rec["dram_bytes_read"] + rec["dram_bytes_write"])
+    w_max = max_over_ranks(n_mine, world, dev)
+    w_min = -max_over_ranks(-n_mine, world, dev)
 
-    # ---- (ii) layer by layer into one reused buffer: the tensors of one decoder
-    # layer share a buffer; every other tensor (embedding, lm_head, ...) uses a
-    # second one
-    groups = []
-    for i, s in enumerate(specs):
-        parts = s.name.split(".")
-        key = ".".join(parts[:2]) if parts[0] == "layers" else None
-        if key is not None and groups and groups[-1][0] == key:
-            groups[-1][1].append(i)
-        else:
-            groups.append((key, [i]))
-    layer_need = max([sum(specs[j].numel for j in idx) for key, idx in groups if key] or [0])
-    other_need = max([specs[idx[0]].numel for key, idx in groups if not key] or [0])
-    layer_buf = torch.empty(layer_need, dtype=torch.int16, device=dev) if layer_need else None
-    other_buf = torch.empty(other_need, dtype=torch.int16, device=dev) if other_need else None
-    layer_groups = []
-    for key, idx in groups:
-        buf = layer_buf if key else other_buf
-        views, off = [], 0
-        for j in idx:
-            views.append(buf[off: off + specs[j].numel])
-            off += specs[j].numel
-        layer_groups.append((idx, views))
-    layer_decs = [codec.BatchDecoder([comps[j] for j in idx], views) for idx, views in layer_groups]
-    for (idx, views), d in zip(layer_groups, layer_decs):  # verify each group once
-        d.run(err)
-        for j, v in zip(idx, views):
-            if not torch.equal(v, src[j]):
-                raise SystemExit(f"layer-by-layer decode mismatch on {specs[j].name}")
-    lsteps = max(1, args.steps // 4)
-    for _ in range(args.warmup):
-        for d in layer_decs:
-            d.run(err)
-    barrier(world)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(lsteps):
-        for d in layer_decs:
-            d.run(err, stream)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier(world)
-    lbl_ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / lsteps
-    assert api.df_read_error(err) == 0
+    # ---- extras at N = 1
+    extras = {}
+    if world == 1 and not args.no_extras:
+        # layer by layer into reused buffers
+        groups = layer_groups(all_specs, idx)
+        cap_l = max([sum(comps[j].n for j in g) for k, g in groups if k] or [0])
+        cap_o = max([comps[g[0]].n for k, g in groups if not k] or [0])
+        lbuf = torch.empty(max(cap_l, 1), dtype=torch.int16, device=dev)
+        obuf = torch.empty(max(cap_o, 1), dtype=torch.int16, device=dev)
+        decs = []
+        for k, g in groups:
+            buf, off, views = (lbuf if k else obuf), 0, []
+            for j in g:
+                views.append(buf[off: off + comps[j].n])
+                off += comps[j].n
+            decs.append(codec.BatchDecoder([comps[j] for j in g], views))
+        lsteps = max(1, args.steps // 4)
+        ms = time_launches(lambda: [d.run(err, stream) for d in decs], lsteps, args.warmup, stream)
+        assert codec.api.df_read_error(err) == 0
+        lbl = statistics.median(ms)
+        extras["layer_by_layer"] = {"value": round(2 * n_mine / (lbl / 1e3) / 1e9, 2), "unit": "GB/s",
+                                    "ms_per_pass": round(lbl, 4), "launches_per_pass": len(decs), "steps": lsteps}
+        del decs, lbuf, obuf
+        # every weight set: one grouped launch each
+        cfg = {args.workload: {"gbs": round(2 * n_mine / launch_ms / 1e6, 2),
+                               "weights_per_s": round(n_mine / launch_ms * 1e3, 1),
+                               "ms": round(statistics.median(step_ms), 4),
+                               "roofline_frac": round(algo_bytes / launch_ms / 1e6 / peak, 4),
+                               "compressed_pct": round(100.0 * container / (2 * n_mine), 4),
+                               "weights": n_mine, "tensors": len(comps),
+                               "l2": "flushed before every step" if flush is not None else
+                               "inputs larger than L2: no flush"}}
+        fl = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        for name in ("single_1024x4096", "llama_layer", "heavy_tail_64m", "mixed_2000"):
+            if name == args.workload:
+                continue
+            sp = synth.weight_set(name)
+            stg = torch.empty(max(s.numel for s in sp), dtype=torch.int16, pin_memory=True)
+            s_src, s_comps, _, _ = encode_set(sp, dev, args, stg)
+            s_outs = [torch.empty(c.n, dtype=torch.int16, device=dev) for c in s_comps]
+            cfg[name] = decode_record(s_comps, s_outs, args, stream, err, peak, fl)
+            verify(s_src, s_outs, [s.name for s in sp])
+            del s_src, s_comps, s_outs, stg
+        extras["configs"] = cfg
+        del fl
+        if args.workload == "llama8b_shaped":
+            extras["jit_layer"] = jit_record(args, all_specs, idx, comps, outs, err, dev)
+        torch.cuda.empty_cache()
 
-    # ---- e2e through the public API: pinned host container -> device -> decode -> pinned host BF16
-    host_parts = []
-    for c in comps:
-        host_parts.append({k: getattr(c, k).cpu().pin_memory() for k in ("stream", "gaps", "offsets")} |
-                          {"sm": c.sm[: c.n].cpu().pin_memory()})
-    host_out = torch.empty(max(sum(comps[j].n for j in idx) for idx, _ in layer_groups), dtype=torch.int16,
-                           pin_memory=True)
-    h2d = sum(sum(p.numel() * p.element_size() for p in hp.values()) for hp in host_parts)
-    d2h = bf16_bytes
-
-    def e2e_step():
-        for (idx, views), d in zip(layer_groups, layer_decs):
-            for j in idx:
-                c, hp = comps[j], host_parts[j]
-                c.stream.copy_(hp["stream"], non_blocking=True)
-                c.gaps.copy_(hp["gaps"], non_blocking=True)
-                c.offsets.copy_(hp["offsets"], non_blocking=True)
-                c.sm[: c.n].copy_(hp["sm"], non_blocking=True)
-            d.run(err)
-            off = 0
-            for v in views:
-                host_out[off: off + v.numel()].copy_(v, non_blocking=True)
-                off += v.numel()
-
-    e2e_step()
-    torch.cuda.synchronize()
-    barrier(world)
-    t0 = time.perf_counter()
-    e0.record(stream)
-    for _ in range(args.e2e_steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    wall = time.perf_counter() - t0
-    barrier(world)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / args.e2e_steps
-    assert api.df_read_error(err) == 0
-    # the last decoded group is still in host_out: check it against the source
-    idx, views = layer_groups[-1]
-    off = 0
-    for j in idx:
-        if not torch.equal(host_out[off: off + comps[j].n], src[j].cpu()):
-            raise SystemExit("e2e output mismatch")
-        off += comps[j].n
+    # ---- e2e through the public API (every N)
+    e2e = e2e_record(args, all_specs, idx, comps, src, dev, world)
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline_sample(specs)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and pool is not None:
+        cpu = cpu_baseline(pool, ncores)
 
     if rank == 0:
         line = {
@@ -503,60 +709,67 @@ def run_gpu(args, world, rank, local):
             "warmup": args.warmup,
             "ms_per_step": round(ms_per_step, 4),
             "higher_is_better": True,
-            "scaling": "weak",
+            "scaling": "strong",
             "vs_baseline": None,
             "dtype": "u8",
             "data": "synthetic (seeded; Box-Muller normals rounded to BF16, shapes of an 8B Llama-style model)",
             "config": {"workload": WORKLOAD if args.workload == "llama8b_shaped" else args.workload,
-                       "weights": n_total, "tensors": len(specs),
+                       "weights": n_all, "tensors": len(all_specs),
                        "chunk_bytes": args.chunk_bytes or "32 (16 for tensors whose shortest code is 1 bit)",
                        "threads_per_block": args.threads_per_block, "max_len": 32,
-                       "l2": f"inputs ({(read_bytes + bf16_bytes) / 1e9:.2f} GB) larger than L2: no flush"
+                       "l2": f"inputs ({(read_bytes + 2 * n_mine) / 1e9:.2f} GB per rank) larger than L2: no flush"
                        if flush is None else
                        f"L2 flushed before every step ({L2_FLUSH_BYTES >> 20} MiB written, outside the timed "
                        f"events)",
-                       "parallelism": f"{world} replica(s), no collective" if world > 1 else "1 GPU"},
-            "weights_per_s": round(world * n_total * args.steps / (total_ms_max / 1e3), 1),
-            "compressed_pct": round(100.0 * container / bf16_bytes, 4),
+                       "parallelism": (f"{world} ranks, tensors partitioned by decode bytes (weights per rank "
+                                       f"{int(w_min):,}..{int(w_max):,}), no collective")
+                       if world > 1 else "1 GPU"},
+            "weights_per_s": round(n_all * args.steps / (total_ms_max / 1e3), 1),
+            "compressed_pct": round(100.0 * container_all / (2 * n_all), 4),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": traffic,
+                         "traffic_workload": rec.get("workload") if rec else None,
                          "peak_source": peak_src,
+                         "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
                          "kernel": "decode_kernel<BatchSrc> (df_decode_batch_run), one launch per step",
                          "algorithmic_bytes_per_launch": algo_bytes},
             "step_ms": {"median": round(statistics.median(step_ms), 4), "min": round(min(step_ms), 4),
                         "max": round(max(step_ms), 4)},
-            "layer_by_layer": {"value": round(world * bf16_bytes / (lbl_ms / 1e3) / 1e9, 2), "unit": "GB/s",
-                               "ms_per_pass": round(lbl_ms, 4), "launches_per_pass": len(layer_decs),
-                               "steps": lsteps},
-            "encode": {"value": round(bf16_bytes / ((hist_ms + enc_ms) / 1e3) / 1e9, 2), "unit": "GB/s of BF16 input",
-                       "histogram_ms": round(hist_ms, 3), "encode_ms": round(enc_ms, 3),
-                       "roofline_frac": round(enc_algo / ((hist_ms + enc_ms) / 1e3) / 1e9 / peak, 4),
-                       "algorithmic_bytes": enc_algo,
-                       "note": "device time of df_histogram over all tensors back to back, plus df_encode over "
-                               "all tensors back to back (the host code build between them is not timed); "
-                               "algorithmic bytes: the input read twice (histogram, pack) + sign|fraction "
-                               "bytes + stream written"},
-            "e2e": {"value": round(world * bf16_bytes / (e2e_ms / 1e3) / 1e9, 3), "unit": "GB/s",
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 2),
-                    "wall_s": round(wall / args.e2e_steps, 3),
-                    "how": "per layer: pinned host container parts -> HBM (cudaMemcpyAsync via torch), "
-                           "df_decode_batch_run, BF16 -> pinned host buffer; one stream"},
+            "encode": {"value": round(2 * n_mine / ((hist_ms + enc_ms) / 1e3) / 1e9, 2),
+                       "unit": "GB/s of BF16 input", "histogram_ms": round(hist_ms, 3),
+                       "encode_ms": round(enc_ms, 3),
+                       "roofline_frac": round((4 * n_mine + n_mine + sum(c.sizes["stream_bytes"] for c in comps))
+                                              / ((hist_ms + enc_ms) / 1e3) / 1e9 / peak, 4),
+                       "note": "CUDA events around every df_histogram and df_encode call, summed (device time; "
+                               "host work between calls is not counted); algorithmic bytes: the input read "
+                               "twice (histogram, pack) + sign|fraction bytes + stream written"},
+            "e2e": e2e,
             "gpu_launches": args.steps,
             "clocks": clk,
             "cpu_baseline": cpu,
         }
+        line.update(extras)
         print(json.dumps(line), flush=True)
 
 
 def main():
     args = parse()
     world, rank, local = dist_setup()
+    pool, ncores = None, os.cpu_count() or 1
+    if args.impl == "ours" and rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import multiprocessing as mp
+
+        # the oracle's worker processes start before the first GPU call
+        pool = mp.get_context("spawn").Pool(ncores)
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)
         else:
-            run_gpu(args, world, rank, local)
+            run_gpu(args, world, rank, local, pool, ncores)
     finally:
+        if pool is not None:
+            pool.close()
+            pool.join()
         if world > 1:
             import torch.distributed as dist
 

@@ -26,8 +26,10 @@
  *   sm      n bytes: sm[i] = (w >> 8 & 0x80) | (w & 0x7F).
  *   lengths 256 code lengths (0 = symbol absent), canonical codes: symbols in
  *           (length, symbol) order, code = (previous + 1) << (length step).
- * C (chunk_bytes, a multiple of 16) and T (threads_per_block, a multiple of
- * 32) are per-tensor parameters; the defaults are C = 32 and T = 256.
+ * C (chunk_bytes, a multiple of 16) and T (threads_per_block: chunks per
+ * format block, a multiple of 32) are per-tensor parameters; the defaults are
+ * C = 32 and T = 32 (a block of T chunks is the unit one warp starts on, so
+ * small T spreads small tensors over more warps; each block costs 8 bytes).
  *
  * Conventions for every function:
  *   - returns a df_status; nothing is thrown across the ABI;
@@ -69,7 +71,7 @@ typedef int df_status;
 #define DF_EFLAG_ENC_SYMBOL 32u   /* encode: an exponent without a code                */
 
 #define DF_DEFAULT_CHUNK_BYTES 32u
-#define DF_DEFAULT_THREADS_PER_BLOCK 256u
+#define DF_DEFAULT_THREADS_PER_BLOCK 32u
 #define DF_DEFAULT_MAX_LEN 32u
 #define DF_MAX_WEIGHTS (1ull << 48) /* n above this is DF_ERR_UNSUPPORTED */
 
@@ -116,6 +118,11 @@ typedef struct df_batch_plan {
     uint32_t region_bytes;     /* shared-memory exponent region of a lane       */
     uint32_t max_groups;       /* 16-output groups a round of 32 chunks spans   */
     uint32_t smem_bytes;       /* dynamic shared memory per CUDA block          */
+    uint32_t max_ctas;         /* 0: as many CUDA blocks as fit on the GPU; else
+                                  at most this many (the caller may set it
+                                  between prepare and run, e.g. to leave SMs to
+                                  a kernel running beside the decode)          */
+    uint32_t reserved;         /* 0                                             */
     uint64_t total_blocks;     /* format blocks over all tensors                */
 } df_batch_plan;
 

@@ -93,6 +93,8 @@ class DfBatchPlan(ctypes.Structure):
         ("region_bytes", ctypes.c_uint32),
         ("max_groups", ctypes.c_uint32),
         ("smem_bytes", ctypes.c_uint32),
+        ("max_ctas", ctypes.c_uint32),
+        ("reserved", ctypes.c_uint32),
         ("total_blocks", ctypes.c_uint64),
     ]
 

@@ -16,7 +16,7 @@ from ._native import DfTensor
 
 DEFAULT_MAX_LEN = 32
 DEFAULT_CHUNK_BYTES = 32
-DEFAULT_THREADS_PER_BLOCK = 256
+DEFAULT_THREADS_PER_BLOCK = 32
 
 
 def _as_u16(w: torch.Tensor) -> torch.Tensor:

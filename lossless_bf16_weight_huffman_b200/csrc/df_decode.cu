@@ -689,10 +689,16 @@ df_status device_limits(int* sms, int* max_smem, int* smem_per_sm) {
     return DF_OK;
 }
 
-// Warps per CUDA block: as many resident warps per SM as shared memory allows
-// (at most 32, the register file's limit at 64 registers), with the most
-// warps per block among equals (one copy of the wide table serves them all).
-df_status choose_warps(const LaunchCfg& c, uint32_t* warps) {
+// Warps per CUDA block. For large launches: as many resident warps per SM as
+// shared memory allows (at most 32, the register file's limit at 64
+// registers), with the most warps per block among equals (one copy of the
+// wide table serves them all). Smaller CUDA blocks when that would leave SMs
+// idle or warps waiting: a launch of fewer format blocks than one per warp of
+// the whole GPU spreads its blocks over every SM, and a launch over more
+// tensors than SMs (every tensor change synchronises the CUDA block, and a
+// small tensor keeps most of a wide block's warps waiting) uses blocks of 8
+// warps, two per SM.
+df_status choose_warps(const LaunchCfg& c, uint64_t total_blocks, uint64_t tensors, uint32_t* warps) {
     int sms = 0, max_smem = 0, per_sm = 0;
     df_status st = device_limits(&sms, &max_smem, &per_sm);
     if (st != DF_OK) return st;
@@ -708,12 +714,17 @@ df_status choose_warps(const LaunchCfg& c, uint32_t* warps) {
         }
     }
     if (!best) return DF_ERR_UNSUPPORTED;
-    *warps = best;
+    uint64_t w = best;
+    const uint64_t per_sm_blocks = (total_blocks + sms - 1) / static_cast<uint64_t>(sms);
+    if (per_sm_blocks < w) w = per_sm_blocks;
+    if (tensors > static_cast<uint64_t>(sms) && w > 8) w = 8;  // 8 measured best on 2000 small tensors
+    *warps = static_cast<uint32_t>(w < 1 ? 1 : (w > best ? best : w));
     return DF_OK;
 }
 
 template <class Src>
-df_status launch(const Src& src, const LaunchCfg& cfg, uint32_t warps, uint32_t* d_err, cudaStream_t stream) {
+df_status launch(const Src& src, const LaunchCfg& cfg, uint32_t warps, uint32_t max_ctas, uint32_t* d_err,
+                 cudaStream_t stream) {
     if (cfg.total_blocks == 0) return DF_OK;
     int sms = 0, max_smem = 0, per_sm = 0;
     df_status st = device_limits(&sms, &max_smem, &per_sm);
@@ -731,7 +742,8 @@ df_status launch(const Src& src, const LaunchCfg& cfg, uint32_t warps, uint32_t*
     // blocks; a range is never shorter than one format block per warp
     const uint64_t slots = static_cast<uint64_t>(sms) * resident;
     const uint64_t want = (cfg.total_blocks + warps - 1) / warps;
-    const uint64_t grid = want < slots ? want : slots;
+    uint64_t grid = want < slots ? want : slots;
+    if (max_ctas && grid > max_ctas) grid = max_ctas;
     kern<<<static_cast<unsigned>(grid), warps * kLanes, smem, stream>>>(src, cfg, d_err);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e);
@@ -764,9 +776,9 @@ df_status df_decode(const df_tensor* t, uint16_t* d_out, uint32_t* d_err, void* 
     widen(&cfg, pr);
     cfg.total_blocks = pr.dev.n_blocks;
     uint32_t warps = 0;
-    st = choose_warps(cfg, &warps);
+    st = choose_warps(cfg, cfg.total_blocks, 1, &warps);
     if (st != DF_OK) return st;
-    return launch(src, cfg, warps, d_err, static_cast<cudaStream_t>(stream));
+    return launch(src, cfg, warps, 0, d_err, static_cast<cudaStream_t>(stream));
 }
 
 size_t df_decode_batch_workspace(uint32_t count) {
@@ -803,7 +815,7 @@ df_status df_decode_batch_prepare(const df_tensor* tensors, uint16_t* const* d_o
     plan->total_blocks = start.back();
     if (plan->count == 0) return DF_OK;
     uint32_t warps = 0;
-    df_status st = choose_warps(cfg, &warps);
+    df_status st = choose_warps(cfg, plan->total_blocks, plan->count, &warps);
     if (st != DF_OK) return st;
     plan->cta_threads = warps * kLanes;
     plan->smem_bytes = static_cast<uint32_t>(smem_bytes(cfg, warps));
@@ -838,7 +850,7 @@ df_status df_decode_batch_run(const df_batch_plan* plan, uint32_t* d_err, void* 
     cfg.total_blocks = plan->total_blocks;
     const uint32_t warps = plan->cta_threads / kLanes;
     if (smem_bytes(cfg, warps) != plan->smem_bytes) return DF_ERR_INVALID_ARG;
-    return launch(src, cfg, warps, d_err, static_cast<cudaStream_t>(stream));
+    return launch(src, cfg, warps, plan->max_ctas, d_err, static_cast<cudaStream_t>(stream));
 }
 
 df_status df_decode_batch(const df_tensor* tensors, uint16_t* const* d_outs, uint32_t count, void* d_ws,

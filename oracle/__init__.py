@@ -118,7 +118,7 @@ def canonical_codes(lengths) -> np.ndarray:
     return codes
 
 
-def sizes(n: int, total_bits: int, chunk_bytes: int = 32, threads_per_block: int = 256) -> dict:
+def sizes(n: int, total_bits: int, chunk_bytes: int = 32, threads_per_block: int = 32) -> dict:
     s = Sizes()
     rc = lib().oracle_sizes(n, total_bits, chunk_bytes, threads_per_block, ctypes.byref(s))
     if rc != OK:
@@ -154,7 +154,7 @@ class Encoded:
         return self.sizes["container_bytes"]
 
 
-def encode(w, max_len: int = 32, chunk_bytes: int = 32, threads_per_block: int = 256, lengths=None) -> Encoded:
+def encode(w, max_len: int = 32, chunk_bytes: int = 32, threads_per_block: int = 32, lengths=None) -> Encoded:
     w = _u16(w)
     h = histogram(w)
     if lengths is None:
@@ -173,7 +173,7 @@ def encode(w, max_len: int = 32, chunk_bytes: int = 32, threads_per_block: int =
     return Encoded(w.size, lengths, codes, chunk_bytes, threads_per_block, max_len, sz, stream, gaps, offsets, sm)
 
 
-def decode(stream, total_bits_: int, sm, n: int, lengths, chunk_bytes: int = 32, threads_per_block: int = 256,
+def decode(stream, total_bits_: int, sm, n: int, lengths, chunk_bytes: int = 32, threads_per_block: int = 32,
            rederive: bool = False):
     """Bit-serial decode. Returns the BF16 bit patterns, or (w, gaps, offsets)
     with ``rederive``; raises ValueError on a corrupt container."""

@@ -35,7 +35,7 @@ def main():
         for max_len in (32, 12):
             if max_len == 12 and set_name != "heavy_tail_64m":
                 continue
-            enc = oracle.encode(w, max_len=max_len)
+            enc = oracle.encode(w, max_len=max_len, chunk_bytes=32, threads_per_block=256)
             out["tensors"].append({
                 "set": set_name, "index": idx, "name": spec.name, "n": int(w.size), "max_len": max_len,
                 "chunk_bytes": 32, "threads_per_block": 256,

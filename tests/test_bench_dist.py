@@ -61,3 +61,64 @@ def test_reference_arm_under_the_launcher():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["unit"] == "GB/s" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def _shard_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+
+    from lossless_bf16_weight_huffman_b200 import shard, synth
+
+    dist.init_process_group("gloo")
+    try:
+        loads = [s.numel for s in synth.llama8b_shaped()]
+        mine = shard.partition(loads, world)[rank]
+        got = [None] * world
+        dist.all_gather_object(got, (rank, mine, sum(loads[i] for i in mine)))
+        q.put(got)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_shard_partition_gloo_world2():
+    """Each rank computes its share of the 8B-shaped set on its own; together
+    the shares cover every tensor exactly once and the ranks' loads differ by
+    at most one tensor's."""
+    from lossless_bf16_weight_huffman_b200 import synth
+
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_shard_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    views = [q.get(timeout=10) for _ in range(2)]
+    assert views[0] == views[1]
+    loads = [s.numel for s in synth.llama8b_shaped()]
+    shares = [m for _, m, _ in views[0]]
+    allidx = sorted(i for m in shares for i in m)
+    assert allidx == list(range(len(loads)))
+    tot = [t for _, _, t in views[0]]
+    assert max(tot) - min(tot) <= max(loads)
+
+
+def test_shard_partition_properties():
+    import random
+
+    from lossless_bf16_weight_huffman_b200 import shard
+
+    rnd = random.Random(5)
+    for trial in range(200):
+        loads = [rnd.choice([1, 7, 4096, 10**6, 5 * 10**8]) for _ in range(rnd.randint(0, 60))]
+        world = rnd.randint(1, 8)
+        parts = shard.partition(loads, world)
+        assert len(parts) == world
+        assert sorted(i for p in parts for i in p) == list(range(len(loads)))
+        tot = shard.rank_loads(loads, parts)
+        if loads:
+            assert max(tot) - min(tot) <= max(loads)

@@ -37,7 +37,7 @@ def roundtrip_oracle_to_gpu(w, **kw):
     return enc, c
 
 
-def encode_on_gpu(w, max_len=32, chunk_bytes=32, tpb=256):
+def encode_on_gpu(w, max_len=32, chunk_bytes=32, tpb=32):
     x = dev_u16(w) if w.size else torch.empty(0, dtype=torch.int16, device="cuda")
     err = err_word()
     c = codec.compress(x, max_len=max_len, chunk_bytes=chunk_bytes, threads_per_block=tpb, d_err=err)
@@ -260,7 +260,7 @@ def test_encode_unaligned_input_and_sign_fraction_output(n):
     err = err_word()
     api.df_encode(code, x, z["total_bits"], 32, 256, stream, gaps, offsets, sm, ws, err)
     assert api.df_read_error(err) == 0
-    enc = oracle.encode(w)
+    enc = oracle.encode(w, chunk_bytes=32, threads_per_block=256)
     assert (stream.cpu().numpy() == enc.stream).all()
     assert (gaps.cpu().numpy() == enc.gaps).all()
     assert (offsets.cpu().numpy().view(np.uint64) == enc.offsets).all()

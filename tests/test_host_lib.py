@@ -58,7 +58,7 @@ def test_struct_sizes_match_header_layout():
     assert ctypes.sizeof(_native.DfCode) == 16 + 256 + 1024
     assert ctypes.sizeof(_native.DfSizes) == 9 * 8
     assert ctypes.sizeof(_native.DfTensor) == 16 + 16 + 5 * 8 + 256
-    assert ctypes.sizeof(_native.DfBatchPlan) == 8 + 6 * 4 + 8
+    assert ctypes.sizeof(_native.DfBatchPlan) == 8 + 8 * 4 + 8
 
 
 def _random_hist(rng, kind):
