@@ -69,6 +69,7 @@ typedef int df_status;
 #define DF_EFLAG_TABLES 8u        /* decode: tables not built for this descriptor      */
 #define DF_EFLAG_ENC_TOTAL 16u    /* encode: stream length != the planned total_bits   */
 #define DF_EFLAG_ENC_SYMBOL 32u   /* encode: an exponent without a code                */
+#define DF_EFLAG_ENC_WAIT 64u     /* encode: a tile waited too long for the one before */
 
 #define DF_DEFAULT_CHUNK_BYTES 32u
 #define DF_DEFAULT_THREADS_PER_BLOCK 32u

@@ -24,6 +24,7 @@ DF_EFLAG_OFFSETS = 4
 DF_EFLAG_TABLES = 8
 DF_EFLAG_ENC_TOTAL = 16
 DF_EFLAG_ENC_SYMBOL = 32
+DF_EFLAG_ENC_WAIT = 64
 
 DF_ENCODE_NOALLOC_MAX_WEIGHTS = 1 << 29
 

@@ -1,5 +1,4 @@
-// Encode path: exponent histogram, per-tile code-length sums, a scan of the
-// tile sums into bit offsets, and a warp-level bit packer.
+// Encode path: exponent histogram, then one pass that writes the container.
 //
 // What is coded (mlx-dfloat, PyPI page, intro bit diagram): the 8 exponent
 // bits of each BF16 weight become a variable-length code; the sign and the 7
@@ -8,11 +7,14 @@
 // bits, C-byte chunks with 5-bit start gaps, per-block output offsets) is the
 // one df11.h defines.
 //
-// Tiles of 4096 weights, 256 threads x 16 consecutive weights: a block scan of
-// the threads' code-length sums gives every code its bit offset; the tile's
-// stream words are assembled in shared memory and stored whole, except the two
-// edge words a tile shares with its neighbours, which are OR-ed atomically into
-// the zeroed stream.
+// Tiles of 4096 weights, 256 threads x 16 consecutive weights, one CUDA block
+// each: a block scan of the threads' code-length sums gives every code its bit
+// offset within the tile; the tile's offset in the stream comes from a
+// decoupled look-back over the tiles before it; the tile's stream words and
+// gap fields are assembled in shared memory and stored whole, except the words
+// a tile shares with its neighbours, which are OR-ed atomically into the
+// zeroed buffers. The input is read twice in all: by the histogram and by this
+// pass.
 #include <cuda_runtime.h>
 
 #include <cstring>
@@ -90,223 +92,391 @@ __device__ __forceinline__ uint32_t load16(const uint16_t* __restrict__ in, uint
     return full ? kPerThread : (i0 < n ? static_cast<uint32_t>(n - i0) : 0u);
 }
 
-// Sum of code lengths of each tile of 4096 weights (16 consecutive weights per
-// thread, as the packer reads them).
-__global__ void __launch_bounds__(kEncThreads) tile_bits_kernel(const uint16_t* __restrict__ in, uint64_t n,
-                                                                int vec, EncTables tab,
-                                                                uint64_t* __restrict__ tile_bits, uint32_t* d_err) {
-    __shared__ uint8_t s_len[256];
-    __shared__ uint32_t s_red[kEncThreads / 32];
-    for (uint32_t i = threadIdx.x; i < 256; i += blockDim.x) s_len[i] = tab.lengths[i];
-    const uint64_t i0 = static_cast<uint64_t>(blockIdx.x) * kTile + threadIdx.x * kPerThread;
-    uint32_t wv[kPerThread / 2];
-    const uint32_t cnt = load16(in, n, i0, vec != 0, wv);
-    __syncthreads();  // the length table
-    uint32_t sum = 0;
-    bool missing = false;
-#pragma unroll
-    for (uint32_t k = 0; k < kPerThread; ++k) {
-        if (k < cnt) {
-            const uint32_t l = s_len[(wv[k >> 1] >> (16 * (k & 1) + 7)) & 0xFFu];
-            missing |= (l == 0);
-            sum += l;
-        }
-    }
-    if (__syncthreads_or(missing) && threadIdx.x == 0 && d_err) atomicOr(d_err, DF_EFLAG_ENC_SYMBOL);
-#pragma unroll
-    for (int d = 16; d > 0; d >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, d);
-    if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = sum;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        uint32_t t = 0;
-        for (uint32_t w = 0; w < kEncThreads / 32; ++w) t += s_red[w];
-        tile_bits[blockIdx.x] = t;
-    }
-}
-
-// Exclusive scan of the tile sums (one block): tile_base[0..tiles].
-__global__ void __launch_bounds__(1024) tile_scan_kernel(const uint64_t* __restrict__ tile_bits, uint64_t tiles,
-                                                         uint64_t* __restrict__ tile_base, uint64_t want_total,
-                                                         uint64_t* __restrict__ offsets, uint64_t n_blocks,
-                                                         uint64_t n, uint32_t* d_err) {
-    __shared__ uint64_t s_w[32];
-    __shared__ uint64_t s_carry;
-    if (threadIdx.x == 0) s_carry = 0;
-    __syncthreads();
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (uint64_t start = 0; start < tiles; start += blockDim.x) {
-        const uint64_t i = start + threadIdx.x;
-        const uint64_t v = i < tiles ? tile_bits[i] : 0;
-        uint64_t x = v;
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            const uint64_t u = __shfl_up_sync(0xFFFFFFFFu, x, d);
-            if (lane >= d) x += u;
-        }
-        if (lane == 31) s_w[warp] = x;
-        __syncthreads();
-        if (warp == 0) {
-            uint64_t y = lane < static_cast<int>(blockDim.x >> 5) ? s_w[lane] : 0;
-#pragma unroll
-            for (int d = 1; d < 32; d <<= 1) {
-                const uint64_t u = __shfl_up_sync(0xFFFFFFFFu, y, d);
-                if (lane >= d) y += u;
-            }
-            s_w[lane] = y;
-        }
-        __syncthreads();
-        const uint64_t carry = s_carry;
-        const uint64_t incl = x + (warp > 0 ? s_w[warp - 1] : 0);
-        if (i < tiles) tile_base[i] = carry + incl - v;
-        __syncthreads();
-        if (threadIdx.x == 0) s_carry = carry + s_w[(blockDim.x >> 5) - 1];
-        __syncthreads();
-    }
-    if (threadIdx.x == 0) {
-        tile_base[tiles] = s_carry;
-        if (s_carry != want_total && d_err) atomicOr(d_err, DF_EFLAG_ENC_TOTAL);
-        offsets[0] = 0;
-        offsets[n_blocks] = n;
-    }
-}
-
-struct PackArgs {
+struct EncArgs {
     const uint16_t* in;
     uint64_t n;
-    const uint64_t* tile_base;
-    uint32_t* stream32;   // the stream as 32-bit words (zeroed)
-    uint32_t* gaps32;     // the gap fields as 32-bit words (zeroed)
-    uint64_t* offsets;
+    uint32_t* stream32;     // the stream as 32-bit words (zeroed)
+    uint32_t* gaps32;       // the gap fields as 32-bit words (zeroed)
+    uint64_t* offsets;      // block offsets (zeroed)
     uint8_t* sm;
-    uint64_t total_bits;
+    unsigned long long* state;  // per tile: (kAggregate | bits) or (kPrefix | bits up to its end); zeroed
+    uint32_t* ticket;           // tile counter (zeroed)
+    uint64_t total_bits;        // the planned stream length
     uint64_t n_chunks;
-    uint64_t stream_words;  // words the stream buffer holds: writes beyond are refused
+    uint64_t stream_words;      // words the stream buffer holds: writes beyond are refused
+    uint64_t gap_words;         // words the gap buffer holds
+    uint64_t n_blocks;
     uint32_t chunk_bits;
-    uint32_t threads_per_block;
+    uint32_t threads_per_block;  // T: chunks per format block
+    uint32_t tiles;
     uint32_t* err;
-    uint32_t in_vec;  // input 16-byte aligned
-    uint32_t sm_vec;  // sign|fraction output 16-byte aligned
+    uint32_t in_vec;    // input 16-byte aligned
+    uint32_t sm_vec;    // sign|fraction output 16-byte aligned
+    uint32_t cb_shift;  // log2(chunk_bits) when it is a power of two, else 32
+    uint32_t t_shift;   // log2(threads_per_block) when it is a power of two, else 32
 };
 
-__device__ __forceinline__ void or_gap(uint32_t* gaps32, uint64_t j, uint32_t g) {
-    const uint64_t q = 5 * j;
-    const uint32_t o = static_cast<uint32_t>(q & 31);
-    uint32_t* w = gaps32 + (q >> 5);
-    if (o <= 27) {
-        atomicOr(w, bswap32(g << (27 - o)));
-    } else {
-        atomicOr(w, bswap32(g >> (o - 27)));
-        atomicOr(w + 1, bswap32(g << (59 - o)));
-    }
+// x / d and x % d, by a shift and a mask when d = 2^sh (sh < 32)
+__device__ __forceinline__ uint32_t div_by(uint32_t x, uint32_t d, uint32_t sh) { return sh < 32 ? x >> sh : x / d; }
+__device__ __forceinline__ uint32_t mod_by(uint32_t x, uint32_t d, uint32_t sh) {
+    return sh < 32 ? x & (d - 1) : x % d;
 }
 
-// One tile of 4096 weights per CUDA block, 16 consecutive weights per thread.
-// A block scan of the threads' code-length sums gives every code its bit
-// offset; the codes are OR-ed into the tile's words in shared memory (shared
-// atomics: neighbouring threads may share a word), then the words go out with
-// coalesced stores, byte-swapped to MSB-first order. The first and last word
-// of a tile may hold bits of the neighbouring tiles: those are OR-ed into the
-// zeroed stream atomically. The code that crosses or ends on a chunk boundary
-// writes that chunk's gap (and, at a block boundary, the block offset).
+constexpr unsigned long long kAggregate = 1ull << 62;  // a tile's own bit count is published
+constexpr unsigned long long kPrefix = 2ull << 62;     // ... and the bits of all tiles up to its end
+constexpr unsigned long long kValue = (1ull << 62) - 1;
+constexpr uint32_t kSpinLimit = 1u << 20;  // polls of a predecessor before giving up (DF_EFLAG_ENC_WAIT)
 
-__global__ void __launch_bounds__(kEncThreads) pack_kernel(PackArgs a, EncTables tab) {
-    __shared__ uint32_t s_code[256];
-    __shared__ uint8_t s_len[256];
-    __shared__ uint32_t s_warp[kEncThreads / 32];
-    __shared__ uint32_t s_words[kTile + 2];  // a tile holds at most 4096 codes of at most 32 bits
-    const uint32_t tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    for (uint32_t i = tid; i < 256; i += kEncThreads) {
-        s_code[i] = tab.codes[i];
-        s_len[i] = tab.lengths[i];
-    }
-    const uint64_t i0 = static_cast<uint64_t>(blockIdx.x) * kTile + tid * kPerThread;
-    uint32_t wv[kPerThread / 2];  // this thread's 16 weights
-    const uint32_t cnt = load16(a.in, a.n, i0, a.in_vec != 0, wv);
-    const bool full = cnt == kPerThread;
-    // sign|fraction bytes
-    uint32_t smw[kPerThread / 4];
+__device__ __forceinline__ unsigned long long ld_acquire(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release(unsigned long long* p, unsigned long long v) {
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ uint64_t warp_sum64(uint64_t x) {
 #pragma unroll
-    for (uint32_t k = 0; k < kPerThread / 4; ++k) {
-        const uint32_t x = wv[2 * k], y = wv[2 * k + 1];
-        // byte j of the word: (w >> 8 & 0x80) | (w & 0x7F) of weight 4k + j
-        const uint32_t hi = __byte_perm(x, y, 0x7531) & 0x80808080u;
-        const uint32_t lo = __byte_perm(x, y, 0x6420) & 0x7F7F7F7Fu;
-        smw[k] = hi | lo;
+    for (int d = 16; d > 0; d >>= 1) x += __shfl_xor_sync(0xFFFFFFFFu, x, d);
+    return x;
+}
+
+// The stream bits before range `tile` (warp 0): decoupled look-back over the
+// ranges before it, 128 at a time (4 per lane, polled together). Every range
+// publishes its own bit count as soon as it has it and its prefix once it
+// knows it; ranges take their index from a counter in launch order, so a range
+// only waits on ranges whose CUDA blocks are already running. Each wait is
+// bounded: when a predecessor stays silent for kSpinLimit polls, the error
+// word gets DF_EFLAG_ENC_WAIT and the range goes on with what it has (its
+// output is then wrong, and flagged).
+constexpr uint32_t kLookPerLane = 4;
+
+__device__ uint64_t look_back(const EncArgs& a, uint32_t tile, uint64_t total, uint32_t lane) {
+    if (tile == 0) {
+        if (lane == 0) st_release(a.state, kPrefix | total);
+        return 0;
     }
-    if (full && a.sm_vec) {
-        *reinterpret_cast<uint4*>(a.sm + i0) = make_uint4(smw[0], smw[1], smw[2], smw[3]);
-    } else {
-        for (uint32_t k = 0; k < cnt; ++k) a.sm[i0 + k] = static_cast<uint8_t>(smw[k >> 2] >> (8 * (k & 3)));
+    if (lane == 0) st_release(a.state + tile, kAggregate | total);
+    uint64_t acc = 0;
+    int64_t top = static_cast<int64_t>(tile) - 1;  // the nearest predecessor not yet accounted for
+    uint32_t spins = 0;
+    for (;;) {
+        // entry q of this lane: predecessor top - (4 lane + q), at distance 4 lane + q
+        unsigned long long v[kLookPerLane];
+#pragma unroll
+        for (uint32_t q = 0; q < kLookPerLane; ++q) {
+            const int64_t i = top - static_cast<int64_t>(kLookPerLane * lane + q);
+            v[q] = i >= 0 ? ld_acquire(a.state + i) : kPrefix;  // before tile 0: prefix 0
+        }
+        for (;;) {
+            bool wait = false;
+#pragma unroll
+            for (uint32_t q = 0; q < kLookPerLane; ++q) wait |= (v[q] >> 62) == 0;
+            if (!__any_sync(0xFFFFFFFFu, wait)) break;
+            const bool give_up = ++spins > kSpinLimit;
+            if (give_up && lane == 0 && a.err) atomicOr(a.err, DF_EFLAG_ENC_WAIT);
+#pragma unroll
+            for (uint32_t q = 0; q < kLookPerLane; ++q) {
+                if ((v[q] >> 62) == 0) {
+                    const int64_t i = top - static_cast<int64_t>(kLookPerLane * lane + q);
+                    v[q] = give_up ? kPrefix : ld_acquire(a.state + i);
+                }
+            }
+        }
+        // the nearest tile with a prefix ends the walk
+        uint32_t qpre = kLookPerLane;
+#pragma unroll
+        for (int q = kLookPerLane - 1; q >= 0; --q)
+            if ((v[q] >> 62) == 2) qpre = q;
+        const uint32_t pre = __ballot_sync(0xFFFFFFFFu, qpre < kLookPerLane);
+        const uint32_t lp = pre ? __ffs(pre) - 1 : 32u;  // the nearest lane with one
+        const uint32_t qlim = lane < lp ? kLookPerLane : (lane == lp ? qpre + 1 : 0u);
+        uint64_t x = 0;
+#pragma unroll
+        for (uint32_t q = 0; q < kLookPerLane; ++q) x += q < qlim ? (v[q] & kValue) : 0;
+        acc += warp_sum64(x);
+        if (pre) break;
+        top -= 32 * kLookPerLane;
     }
-    __syncthreads();  // the code tables
+    if (lane == 0) st_release(a.state + tile, kPrefix | (acc + total));
+    return acc;
+}
+
+// Code lengths of a thread's weights, their sum, and whether an exponent
+// without a code occurs (kFull: all 16 weights are below n).
+template <bool kFull>
+__device__ __forceinline__ uint32_t length_sum(const uint2* s_cl, const uint32_t wv[kPerThread / 2], uint32_t cnt,
+                                               bool* missing) {
     uint32_t sum = 0;
 #pragma unroll
     for (uint32_t k = 0; k < kPerThread; ++k) {
-        const uint32_t e = (wv[k >> 1] >> (16 * (k & 1) + 7)) & 0xFFu;
-        sum += k < cnt ? s_len[e] : 0u;
+        const uint32_t l = (kFull || k < cnt) ? s_cl[(wv[k >> 1] >> (16 * (k & 1) + 7)) & 0xFFu].y : 1u;
+        *missing |= l == 0;
+        sum += (kFull || k < cnt) ? l : 0u;
     }
-    // block scan of the sums
-    uint32_t incl = sum;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-        const uint32_t u = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-        if (lane >= static_cast<uint32_t>(d)) incl += u;
-    }
-    if (lane == 31) s_warp[warp] = incl;
-    const uint64_t tile_bit0 = a.tile_base[blockIdx.x];
-    const uint32_t head = static_cast<uint32_t>(tile_bit0 & 31);  // bits of the first word before the tile
-    __syncthreads();
-    uint32_t wprefix = 0, total = 0;
-#pragma unroll
-    for (uint32_t w = 0; w < kEncThreads / 32; ++w) {
-        const uint32_t t = s_warp[w];
-        wprefix += w < warp ? t : 0u;
-        total += t;
-    }
-    const uint32_t nw = (head + total + 31) >> 5;  // words the tile touches
-    for (uint32_t k = tid; k < nw; k += kEncThreads) s_words[k] = 0;
-    __syncthreads();
-    // OR the codes into the tile's words (bit q of the tile -> bit 31 - q % 32 of word q / 32)
-    const uint32_t off = wprefix + incl - sum;  // this thread's first bit within the tile
-    uint32_t lp = head + off;
-    uint64_t gb = tile_bit0 + off;  // ... and in the stream
-    // the first chunk boundary after gb, and its chunk index
-    uint64_t jn = gb / a.chunk_bits + 1;
-    uint64_t nb = jn * a.chunk_bits;
+    return sum;
+}
+
+// The code lengths' sum and, when it is at most 64, the codes packed into
+// one register MSB-first (the first code in the highest bits of the sum).
+template <bool kFull>
+__device__ __forceinline__ uint32_t pack64(const uint2* s_cl, const uint32_t wv[kPerThread / 2], uint32_t cnt,
+                                           unsigned long long* v) {
+    uint32_t sum = 0;
+    unsigned long long x = 0;
 #pragma unroll
     for (uint32_t k = 0; k < kPerThread; ++k) {
-        if (k >= cnt) break;
-        const uint32_t e = (wv[k >> 1] >> (16 * (k & 1) + 7)) & 0xFFu;
-        const uint32_t l = s_len[e];
-        if (l == 0) continue;
-        const uint32_t v = s_code[e] << (32 - l);  // the code, left-aligned
-        const uint32_t sh = lp & 31;
-        atomicOr(&s_words[lp >> 5], v >> sh);
-        if (sh + l > 32) atomicOr(&s_words[(lp >> 5) + 1], v << (32 - sh));
-        lp += l;
-        gb += l;
-        if (gb >= nb) {  // this code crosses or ends on chunk boundary nb: the next start is gb
-            if (jn < a.n_chunks) {
-                or_gap(a.gaps32, jn, static_cast<uint32_t>(gb - nb));
-                if (jn % a.threads_per_block == 0) a.offsets[jn / a.threads_per_block] = i0 + k + 1;
-            }
-            ++jn;
-            nb += a.chunk_bits;
+        if (kFull || k < cnt) {
+            const uint2 cl = s_cl[(wv[k >> 1] >> (16 * (k & 1) + 7)) & 0xFFu];
+            x = (x << cl.y) | cl.x;
+            sum += cl.y;
         }
     }
+    *v = x;
+    return sum;
+}
+
+constexpr uint32_t kWarpTile = 32 * kPerThread;      // 512 weights: a warp, 16 consecutive weights per lane
+constexpr uint32_t kEncWarps = kEncThreads / 32;
+constexpr uint32_t kWarpWords = kWarpTile + 2;       // a warp tile holds at most 512 codes of at most 32 bits
+// gap fields a warp tile can hold (every code 32 bits, 16-byte chunks) as
+// words, plus the partial words at both ends
+constexpr uint32_t kWarpGapWords = (5 * (kWarpTile * 32 / 128 + 2) + 31) / 32 + 4;
+
+// Persistent CUDA blocks, each over a contiguous range of the tensor's warp
+// tiles (512 weights, 16 consecutive weights per lane), split into one
+// sub-range per warp, in two passes:
+//   1. every warp writes the sign|fraction bytes of its sub-range and sums
+//      its code lengths; the CUDA block's range gets its stream offset from a
+//      look-back over the ranges before it (once per CUDA block), and every
+//      warp its own from the sums of the warps before it
+//   2. every warp packs its tiles on its own, with no block-wide barrier: a
+//      warp scan of the lanes' code-length sums gives every code its bit
+//      offset; each lane packs its codes MSB-first into a 64-bit register and
+//      writes the tile's words in the warp's shared memory, whole words with
+//      plain stores and the two partial words it shares with its neighbours
+//      with shared OR. The code that crosses or ends on a chunk boundary
+//      writes that chunk's gap into the warp's gap words (and, at a
+//      format-block boundary, the block offset). The tile's stream and gap
+//      words go out with coalesced stores, except the end words shared with
+//      the neighbouring tiles, which are OR-ed into the zeroed buffers.
+__global__ void __launch_bounds__(kEncThreads) encode_kernel(EncArgs a, EncTables tab) {
+    __shared__ uint2 s_cl[256];  // per exponent: (code right-aligned, length)
+    __shared__ uint32_t s_range;
+    __shared__ unsigned long long s_sum[kEncWarps];
+    __shared__ unsigned long long s_pre[kEncWarps];
+    __shared__ uint32_t s_words[kEncWarps][kWarpWords];
+    __shared__ uint32_t s_gaps[kEncWarps][kWarpGapWords];
+    const uint32_t tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid == 0) s_range = atomicAdd(a.ticket, 1u);  // ranges start in index order
+    for (uint32_t i = tid; i < 256; i += kEncThreads) {
+        s_cl[i] = make_uint2(tab.codes[i], tab.lengths[i]);
+    }
     __syncthreads();
-    // out: whole words inside the tile are stored, the two edge words OR-ed in
-    const uint64_t w0 = tile_bit0 >> 5;
-    for (uint32_t k = tid; k < nw; k += kEncThreads) {
-        const uint64_t W = w0 + k;
-        const uint32_t val = bswap32(s_words[k]);
-        if (W >= a.stream_words) {
-            if (a.err) atomicOr(a.err, DF_EFLAG_ENC_TOTAL);
-        } else if (k == 0 || k + 1 == nw) {
-            if (val) atomicOr(a.stream32 + W, val);
-        } else {
-            a.stream32[W] = val;
+    const uint64_t range = s_range, R = gridDim.x;
+    const uint64_t wtiles = (a.n + kWarpTile - 1) / kWarpTile;
+    // balanced contiguous splits (no products that could overflow)
+    const uint64_t r_begin = (wtiles / R) * range + min(range, wtiles % R);
+    const uint64_t r_len = wtiles / R + (range < wtiles % R ? 1 : 0);
+    const uint64_t t_begin = r_begin + (r_len / kEncWarps) * warp + min(static_cast<uint64_t>(warp), r_len % kEncWarps);
+    const uint64_t t_end = t_begin + r_len / kEncWarps + (warp < r_len % kEncWarps ? 1 : 0);
+
+    // 1. sign|fraction bytes and the bit count of this warp's sub-range
+    uint64_t lsum = 0;
+    bool missing = false;
+    for (uint64_t t = t_begin; t < t_end; ++t) {
+        const uint64_t i0 = t * kWarpTile + lane * kPerThread;
+        uint32_t wv[kPerThread / 2];
+        const uint32_t cnt = load16(a.in, a.n, i0, a.in_vec != 0, wv);
+        uint32_t smw[kPerThread / 4];
+#pragma unroll
+        for (uint32_t k = 0; k < kPerThread / 4; ++k) {
+            const uint32_t x = wv[2 * k], y = wv[2 * k + 1];
+            // byte j of the word: (w >> 8 & 0x80) | (w & 0x7F) of weight 4k + j
+            const uint32_t hi = __byte_perm(x, y, 0x7531) & 0x80808080u;
+            const uint32_t lo = __byte_perm(x, y, 0x6420) & 0x7F7F7F7Fu;
+            smw[k] = hi | lo;
         }
+        if (cnt == kPerThread && a.sm_vec) {
+            *reinterpret_cast<uint4*>(a.sm + i0) = make_uint4(smw[0], smw[1], smw[2], smw[3]);
+        } else {
+            for (uint32_t k = 0; k < cnt; ++k) a.sm[i0 + k] = static_cast<uint8_t>(smw[k >> 2] >> (8 * (k & 3)));
+        }
+        lsum += cnt == kPerThread ? length_sum<true>(s_cl, wv, cnt, &missing) : length_sum<false>(s_cl, wv, cnt, &missing);
+    }
+    const uint64_t wsum = warp_sum64(lsum);
+    if (lane == 0) s_sum[warp] = wsum;
+    if (__syncthreads_or(missing) && tid == 0 && a.err) atomicOr(a.err, DF_EFLAG_ENC_SYMBOL);
+    if (warp == 0) {
+        uint64_t total = 0, before = 0;
+#pragma unroll
+        for (uint32_t w = 0; w < kEncWarps; ++w) {
+            const uint64_t v = s_sum[w];
+            before += w < lane ? v : 0;
+            total += v;
+        }
+        const uint64_t pre = look_back(a, static_cast<uint32_t>(range), total, lane);
+        if (lane < kEncWarps) s_pre[lane] = pre + before;
+    }
+    __syncthreads();
+
+    // 2. pack, warp tile by warp tile
+    uint32_t* words = s_words[warp];
+    uint32_t* gapw = s_gaps[warp];
+    const uint32_t cbits = a.chunk_bits, T = a.threads_per_block, csh = a.cb_shift, tsh = a.t_shift;
+    uint64_t bit0 = s_pre[warp];              // the first stream bit of the next tile
+    uint32_t rr = static_cast<uint32_t>(bit0 % cbits);  // bit0 = jc * cbits + rr
+    uint64_t jc = bit0 / cbits;
+    uint32_t jcT = static_cast<uint32_t>(jc % T);
+    for (uint64_t t = t_begin; t < t_end; ++t) {
+        const uint64_t i0 = t * kWarpTile + lane * kPerThread;
+        uint32_t wv[kPerThread / 2];
+        const uint32_t cnt = load16(a.in, a.n, i0, a.in_vec != 0, wv);
+        unsigned long long v;
+        const uint32_t sum = cnt == kPerThread ? pack64<true>(s_cl, wv, cnt, &v) : pack64<false>(s_cl, wv, cnt, &v);
+        uint32_t incl = sum;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const uint32_t u = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+            if (lane >= static_cast<uint32_t>(d)) incl += u;
+        }
+        const uint32_t total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+        const uint32_t head = static_cast<uint32_t>(bit0 & 31);  // bits of the first word before the tile
+        const uint32_t nw = (head + total + 31) >> 5;          // words the tile touches
+        for (uint32_t k = lane; k < nw; k += 32) words[k] = 0;
+        if (lane < kWarpGapWords) gapw[lane] = 0;
+        // chunk boundaries in tile-relative bits: B0 + m * cbits is the start of
+        // chunk jt0 + m. This tile writes the gaps of the boundaries B with
+        // 0 < B <= total (the code that crosses or ends on B starts before it);
+        // a boundary at 0 belongs to the previous tile's last code.
+        const uint32_t B0 = rr ? cbits - rr : 0u;
+        const uint64_t jt0 = jc + (rr ? 1u : 0u);
+        const uint64_t j_first = jt0 + (B0 == 0 ? 1u : 0u);
+        const uint32_t gw0 = static_cast<uint32_t>((5 * j_first) >> 5);  // the tile's first gap word
+        const uint32_t jt0_mod_T = mod_by(jcT + (rr ? 1u : 0u), T, tsh);
+        __syncwarp();  // zeroed
+
+        // this lane's codes into the tile's words
+        const uint32_t off = incl - sum;  // this lane's first bit within the tile
+        const uint32_t q = head + off;
+        uint32_t* wp = words + (q >> 5);
+        const uint32_t sh = q & 31;  // bits of the first word before this lane's
+        if (sum <= 64) {
+            // the packed codes placed at bit sh of a three-word window (only
+            // the first and last words are shared with the neighbours)
+            if (sum) {
+                const unsigned long long x = v << (64 - sum);  // left-aligned
+                const uint32_t xh = static_cast<uint32_t>(x >> 32), xl = static_cast<uint32_t>(x);
+                const uint32_t n = (sh + sum + 31) >> 5;  // words touched: 1..3
+                atomicOr(wp, xh >> sh);
+                if (n == 2) atomicOr(wp + 1, __funnelshift_r(xl, xh, sh));
+                if (n == 3) {
+                    wp[1] = __funnelshift_r(xl, xh, sh);
+                    atomicOr(wp + 2, xl << (32 - sh));
+                }
+            }
+        } else {  // longer codes: a running 64-bit register, whole words as they fill
+            uint32_t nbits = sh;
+            unsigned long long acc = 0;  // pending bits, left-aligned
+            bool first = true;
+#pragma unroll
+            for (uint32_t k = 0; k < kPerThread; ++k) {
+                const uint2 cl = k < cnt ? s_cl[(wv[k >> 1] >> (16 * (k & 1) + 7)) & 0xFFu] : make_uint2(0u, 0u);
+                if (cl.y) {
+                    acc |= (static_cast<unsigned long long>(cl.x << (32 - cl.y)) << 32) >> nbits;
+                    nbits += cl.y;
+                    if (nbits >= 32) {
+                        const uint32_t word = static_cast<uint32_t>(acc >> 32);
+                        if (first)
+                            atomicOr(wp, word);
+                        else
+                            *wp = word;
+                        first = false;
+                        ++wp;
+                        acc <<= 32;
+                        nbits -= 32;
+                    }
+                }
+            }
+            if (nbits) atomicOr(wp, static_cast<uint32_t>(acc >> 32));
+        }
+        // chunk boundaries in (off, off + sum]: the code that crosses or ends on
+        // one writes its chunk's gap (the next code start - the boundary) and,
+        // at a format-block boundary, the block offset
+        uint32_t m = off < B0 ? 0u : div_by(off - B0, cbits, csh) + 1;
+        uint32_t nb = B0 + m * cbits;  // the first boundary after this lane's start
+        if (nb <= off + sum) {
+            uint32_t end = off;
+#pragma unroll
+            for (uint32_t k = 0; k < kPerThread; ++k) {
+                const uint32_t l = k < cnt ? s_cl[(wv[k >> 1] >> (16 * (k & 1) + 7)) & 0xFFu].y : 0u;
+                end += l;
+                if (l && end >= nb) {
+                    const uint64_t j = jt0 + m;
+                    if (j < a.n_chunks) {
+                        const uint64_t gq = 5 * j;
+                        const uint32_t gw = static_cast<uint32_t>(gq >> 5) - gw0;
+                        const uint32_t o = static_cast<uint32_t>(gq & 31);
+                        const uint32_t g = end - nb;
+                        if (o <= 27) {
+                            atomicOr(gapw + gw, g << (27 - o));
+                        } else {
+                            atomicOr(gapw + gw, g >> (o - 27));
+                            atomicOr(gapw + gw + 1, g << (59 - o));
+                        }
+                        if (mod_by(jt0_mod_T + m, T, tsh) == 0) a.offsets[tsh < 32 ? j >> tsh : j / T] = i0 + k + 1;
+                    }
+                    ++m;
+                    nb += cbits;
+                }
+            }
+        }
+        if (t + 1 == wtiles && lane == 0) {  // the last tile closes the stream
+            if (bit0 + total != a.total_bits && a.err) atomicOr(a.err, DF_EFLAG_ENC_TOTAL);
+            a.offsets[a.n_blocks] = a.n;
+        }
+        __syncwarp();
+        // out: whole words inside the tile are stored, the two edge words OR-ed in
+        const uint64_t w0 = bit0 >> 5;
+        for (uint32_t k = lane; k < nw; k += 32) {
+            const uint64_t W = w0 + k;
+            const uint32_t val = bswap32(words[k]);
+            if (W >= a.stream_words) {
+                if (a.err) atomicOr(a.err, DF_EFLAG_ENC_TOTAL);
+            } else if (k == 0 || k + 1 == nw) {
+                if (val) atomicOr(a.stream32 + W, val);
+            } else {
+                a.stream32[W] = val;
+            }
+        }
+        // the tile's gap fields: chunks j_first .. j_last; the words at both
+        // ends may hold fields of the neighbouring tiles
+        if (total >= B0) {
+            uint64_t j_last = jt0 + div_by(total - B0, cbits, csh);
+            if (j_last >= a.n_chunks) j_last = a.n_chunks - 1;
+            if (j_last >= j_first) {
+                const uint32_t gwn = static_cast<uint32_t>((5 * j_last + 4) >> 5) - gw0 + 1;
+                for (uint32_t k = lane; k < gwn; k += 32) {
+                    const uint64_t W = gw0 + k;
+                    const uint32_t val = bswap32(gapw[k]);
+                    if (W >= a.gap_words) continue;
+                    if (k == 0 || k + 1 == gwn) {
+                        if (val) atomicOr(a.gaps32 + W, val);
+                    } else {
+                        a.gaps32[W] = val;
+                    }
+                }
+            }
+        }
+        __syncwarp();  // the next tile zeroes the words
+        bit0 += total;
+        const uint32_t rn = rr + total;
+        const uint32_t qn = div_by(rn, cbits, csh);
+        jc += qn;
+        jcT = mod_by(jcT + qn, T, tsh);
+        rr = rn - qn * cbits;
     }
 }
 
@@ -418,29 +588,44 @@ df_status df_encode(const df_code* code, const uint16_t* d_in, uint64_t n, uint6
     EncTables tab;
     std::memcpy(tab.codes, code->codes, sizeof(tab.codes));
     std::memcpy(tab.lengths, code->lengths, sizeof(tab.lengths));
-    uint64_t* tile_bits = static_cast<uint64_t*>(d_ws);
-    uint64_t* tile_base = tile_bits + tiles;
-    tile_bits_kernel<<<static_cast<unsigned>(tiles), kEncThreads, 0, s>>>(d_in, n, aligned(d_in, 16) ? 1 : 0, tab,
-                                                                         tile_bits, d_err);
-    tile_scan_kernel<<<1, 1024, 0, s>>>(tile_bits, tiles, tile_base, total_bits, d_block_offsets, n_blocks, n,
-                                         d_err);
-    PackArgs a;
+    // workspace: per-tile look-back state, then the tile counter; both zeroed
+    e = cudaMemsetAsync(d_ws, 0, 8 * tiles + 16, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    EncArgs a;
     a.in = d_in;
     a.n = n;
-    a.tile_base = tile_base;
     a.stream32 = reinterpret_cast<uint32_t*>(d_stream);
     a.gaps32 = reinterpret_cast<uint32_t*>(d_gaps);
     a.offsets = d_block_offsets;
     a.sm = d_sm;
+    a.state = static_cast<unsigned long long*>(d_ws);
+    a.ticket = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(d_ws) + 8 * tiles);
     a.total_bits = total_bits;
     a.n_chunks = n_chunks;
     a.stream_words = stream_bytes / 4;
-    a.err = d_err;
+    a.gap_words = gap_bytes / 4;
+    a.n_blocks = n_blocks;
     a.chunk_bits = static_cast<uint32_t>(cbits);
     a.threads_per_block = tpb;
+    a.tiles = static_cast<uint32_t>(tiles);
+    a.err = d_err;
     a.in_vec = aligned(d_in, 16) ? 1u : 0u;
     a.sm_vec = aligned(d_sm, 16) ? 1u : 0u;
-    pack_kernel<<<static_cast<unsigned>(tiles), kEncThreads, 0, s>>>(a, tab);
+    a.cb_shift = a.t_shift = 32;
+    for (uint32_t k = 0; k < 32; ++k) {
+        if ((1ull << k) == cbits) a.cb_shift = k;
+        if ((1u << k) == tpb) a.t_shift = k;
+    }
+    // persistent CUDA blocks: as many as are resident at once, at most one per tile
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, encode_kernel, kEncThreads, 0);
+    if (e != cudaSuccess) return cuda_fail(e);
+    int sms = 0;
+    const df_status st = sm_count(&sms);
+    if (st != DF_OK) return st;
+    const uint64_t slots = static_cast<uint64_t>(sms) * static_cast<uint64_t>(per_sm < 1 ? 1 : per_sm);
+    const uint64_t grid = tiles < slots ? tiles : slots;  // at least one warp tile per warp (8 per block)
+    encode_kernel<<<static_cast<unsigned>(grid), kEncThreads, 0, s>>>(a, tab);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e);
     return DF_OK;
