@@ -308,6 +308,45 @@ df_status df_decode_batch(const df_tensor* tensors, uint16_t* const* d_outs, uin
  * Errors: DF_ERR_INVALID_ARG, DF_ERR_CUDA. */
 df_status df_read_error(const uint32_t* d_err, void* stream, uint32_t* flags);
 
+/* ---- checks (df11pack, GitHub page, "Use": verify checks a container's
+ * structure with no source, decodes sampled chunks, or all of them, and
+ * compares them with the source, exiting 0 on pass, 1 when a check fails, 2
+ * when it could not check; "What is checked": --hashes, a per-tensor SHA-256
+ * that lets verify catch corruption without the source) ------------------- */
+
+/* df_check_structure: the container's block offsets, without decoding:
+ * offsets[0] = 0, offsets never decrease, offsets[n_blocks] = n, and no block
+ * holds more codes than its chunks can (T * ceil(8C / shortest code length)).
+ * Sizes no container can have (total_bits outside [n, 32n], a bad format) also
+ * fail. A failure ORs DF_EFLAG_OFFSETS into *d_flags (device word, caller
+ * zeroes it; read it with df_read_error). Source: df11pack, "Use" (verify:
+ * structure, no source needed). Errors: DF_ERR_INVALID_ARG, DF_ERR_CUDA. */
+df_status df_check_structure(const df_tensor* t, uint32_t* d_flags, void* stream);
+
+/* df_compare: *d_first_diff (device uint64) = the first i < n with
+ * d_a[i] != d_b[i], or UINT64_MAX when they are equal (both device arrays of n
+ * uint16). Source: df11pack, "Use" (decoded chunks compared with the source).
+ * Errors: DF_ERR_INVALID_ARG, DF_ERR_CUDA. */
+df_status df_compare(const uint16_t* d_a, const uint16_t* d_b, uint64_t n, uint64_t* d_first_diff, void* stream);
+
+/* Device workspace bytes df_sha256_device needs for nbytes of data (32 per
+ * leaf). Source: as df_sha256_device. */
+size_t df_sha256_workspace(uint64_t nbytes);
+
+/* df_sha256_device: the digest of nbytes of device data, a tree over SHA-256
+ * (FIPS 180-4): the data is cut into leaves of 65,536 bytes (the last one
+ * shorter; none for nbytes = 0), each leaf is hashed on the GPU, and digest =
+ * SHA-256 of the leaf digests in order (computed on the host after waiting
+ * for `stream`). Source: df11pack, "What is checked" (--hashes: a per-tensor
+ * SHA-256); the leaf tree is this library's own, so that a large tensor hashes
+ * in parallel. Errors: DF_ERR_INVALID_ARG, DF_ERR_WORKSPACE, DF_ERR_CUDA. */
+df_status df_sha256_device(const void* d_data, uint64_t nbytes, void* d_ws, size_t ws_bytes, uint8_t digest[32],
+                           void* stream);
+
+/* df_sha256: plain SHA-256 (FIPS 180-4) of nbytes of host data. Source: as
+ * df_sha256_device. Errors: DF_ERR_INVALID_ARG. */
+df_status df_sha256(const void* data, uint64_t nbytes, uint8_t digest[32]);
+
 #ifdef __cplusplus
 }
 #endif

@@ -33,7 +33,8 @@ EXPORTS = (
     "df_status_string", "df_last_cuda_error", "df_build_code", "df_code_from_lengths", "df_lut_words", "df_build_lut", "df_plan",
     "df_container_sizes",
     "df_histogram", "df_encode", "df_encode_noalloc", "df_decode", "df_decode_batch_workspace", "df_decode_batch_prepare",
-    "df_decode_batch_run", "df_decode_batch", "df_read_error",
+    "df_decode_batch_run", "df_decode_batch", "df_read_error", "df_check_structure", "df_compare",
+    "df_sha256_workspace", "df_sha256_device", "df_sha256",
 )
 
 
@@ -153,6 +154,16 @@ def lib() -> ctypes.CDLL:
     L.df_decode_batch.restype = i32
     L.df_read_error.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
     L.df_read_error.restype = i32
+    L.df_check_structure.argtypes = [ctypes.POINTER(DfTensor), vp, vp]
+    L.df_check_structure.restype = i32
+    L.df_compare.argtypes = [vp, vp, u64, vp, vp]
+    L.df_compare.restype = i32
+    L.df_sha256_workspace.argtypes = [u64]
+    L.df_sha256_workspace.restype = sz
+    L.df_sha256_device.argtypes = [vp, u64, vp, sz, vp, vp]
+    L.df_sha256_device.restype = i32
+    L.df_sha256.argtypes = [vp, u64, vp]
+    L.df_sha256.restype = i32
     _lib = L
     return L
 

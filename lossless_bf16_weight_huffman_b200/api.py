@@ -170,7 +170,9 @@ def _batch_arrays(tensors, d_outs):
         if isinstance(o, torch.Tensor):
             _need(o, 2 * t.n, f"d_outs[{i}]")
     arr = (DfTensor * max(1, len(tensors)))(*tensors)
-    outs = (ctypes.c_void_p * max(1, len(d_outs)))(*[_dev(o, "d_outs[i]").value for o in d_outs])
+    # an int is a raw device pointer, passed through unchecked
+    outs = (ctypes.c_void_p * max(1, len(d_outs)))(
+        *[o if isinstance(o, int) else _dev(o, "d_outs[i]").value for o in d_outs])
     return arr, outs
 
 
@@ -205,3 +207,45 @@ def df_read_error(d_err: torch.Tensor, stream=None) -> int:
     if status not in (0, 3):
         check("df_read_error", status)
     return int(flags.value)
+
+
+def df_check_structure(t: DfTensor, d_flags: torch.Tensor, stream=None) -> None:
+    _need_err(d_flags)
+    check("df_check_structure", lib().df_check_structure(ctypes.byref(t), _dev(d_flags, "d_flags"),
+                                                         _stream_ptr(stream)))
+
+
+def df_compare(d_a: torch.Tensor, d_b: torch.Tensor, d_first_diff: torch.Tensor, stream=None) -> None:
+    _need_u16(d_a, "d_a")
+    _need_u16(d_b, "d_b")
+    if d_a.numel() != d_b.numel():
+        raise ValueError("d_a and d_b differ in size")
+    _need(d_first_diff, 8, "d_first_diff")
+    check("df_compare", lib().df_compare(_dev(d_a, "d_a"), _dev(d_b, "d_b"), d_a.numel(),
+                                         _dev(d_first_diff, "d_first_diff"), _stream_ptr(stream)))
+
+
+def df_sha256_workspace(nbytes: int) -> int:
+    return int(lib().df_sha256_workspace(nbytes))
+
+
+def df_sha256_device(d_data: torch.Tensor, d_ws: torch.Tensor | None = None, stream=None) -> bytes:
+    """The leaf-tree SHA-256 of a device tensor's bytes (waits for the stream)."""
+    nbytes = d_data.numel() * d_data.element_size()
+    need = df_sha256_workspace(nbytes)
+    if d_ws is None:
+        d_ws = torch.empty(need, dtype=torch.uint8, device=d_data.device)
+    _need(d_ws, need, "d_ws")
+    out = (ctypes.c_uint8 * 32)()
+    check("df_sha256_device", lib().df_sha256_device(_dev(d_data, "d_data"), nbytes, _dev(d_ws, "d_ws"),
+                                                     d_ws.numel() * d_ws.element_size(), out, _stream_ptr(stream)))
+    return bytes(out)
+
+
+def df_sha256(data) -> bytes:
+    """Plain SHA-256 of host bytes (a numpy array or bytes)."""
+    arr = np.ascontiguousarray(np.frombuffer(data, np.uint8) if isinstance(data, (bytes, bytearray)) else data)
+    buf = arr.view(np.uint8).reshape(-1)
+    out = (ctypes.c_uint8 * 32)()
+    check("df_sha256", lib().df_sha256(buf.ctypes.data if buf.size else None, buf.size, out))
+    return bytes(out)

@@ -114,11 +114,17 @@ def auto_chunk_bytes(code) -> int:
     return DEFAULT_CHUNK_BYTES if code.min_len >= 2 else 16
 
 
+class SafeCheckError(RuntimeError):
+    pass
+
+
 def compress(w: torch.Tensor, max_len: int = DEFAULT_MAX_LEN, chunk_bytes: int | None = None,
              threads_per_block: int = DEFAULT_THREADS_PER_BLOCK, d_err: torch.Tensor | None = None,
-             stream=None) -> Compressed:
+             stream=None, safe: bool = False) -> Compressed:
     """Histogram on the GPU, code build on the host, encode on the GPU.
-    chunk_bytes=None picks auto_chunk_bytes(code)."""
+    chunk_bytes=None picks auto_chunk_bytes(code). safe=True decodes the new
+    container and compares it with w on the GPU before returning (df11pack,
+    "Use": --safe), raising SafeCheckError on any difference."""
     x = _as_u16(w)
     dev = x.device
     n = x.numel()
@@ -137,8 +143,18 @@ def compress(w: torch.Tensor, max_len: int = DEFAULT_MAX_LEN, chunk_bytes: int |
     ws = torch.empty(max(z["encode_ws_bytes"], 16), dtype=torch.uint8, device=dev)
     api.df_encode(code, x, z["total_bits"], chunk_bytes, threads_per_block, stream_buf, gaps, offsets,
                   sm, ws, d_err, stream)
-    return Compressed(n=n, shape=tuple(w.shape), code=code, lut=lut, sizes=z, chunk_bytes=chunk_bytes,
-                      threads_per_block=threads_per_block, stream=stream_buf, gaps=gaps, offsets=offsets, sm=sm)
+    c = Compressed(n=n, shape=tuple(w.shape), code=code, lut=lut, sizes=z, chunk_bytes=chunk_bytes,
+                   threads_per_block=threads_per_block, stream=stream_buf, gaps=gaps, offsets=offsets, sm=sm)
+    if safe and n:
+        err = torch.zeros(1, dtype=torch.int32, device=dev)
+        api.df_read_error(err, stream)
+        back = torch.empty(n, dtype=torch.int16, device=dev)
+        decompress(c, back, err, stream)
+        first = torch.empty(1, dtype=torch.int64, device=dev)
+        api.df_compare(back, x, first, stream)
+        if api.df_read_error(err, stream) or int(first.cpu().numpy().view(np.uint64)[0]) != 2**64 - 1:
+            raise SafeCheckError("the container does not decode to its source")
+    return c
 
 
 def decompress(c: Compressed, out: torch.Tensor | None = None, d_err: torch.Tensor | None = None,
