@@ -1,4 +1,5 @@
-"""ctypes view of libdf11.so (the C ABI declared in include/df11.h).
+"""ctypes view of libdf11.so (the C ABI declared in include/df11.h and
+include/nf12.h).
 
 The library is loaded on first use. There is no fallback: if the CUDA library
 has not been built, every call raises ``NativeLibraryMissing``.
@@ -25,16 +26,22 @@ DF_EFLAG_TABLES = 8
 DF_EFLAG_ENC_TOTAL = 16
 DF_EFLAG_ENC_SYMBOL = 32
 DF_EFLAG_ENC_WAIT = 64
+DF_EFLAG_NF12_SIDE = 128
+
+DF_NF12_TOP = 7
+DF_NF12_TILE_GROUPS = 2048
 
 DF_ENCODE_NOALLOC_MAX_WEIGHTS = 1 << 29
 
-# every function declared in include/df11.h
+# every function declared in include/df11.h and include/nf12.h
 EXPORTS = (
     "df_status_string", "df_last_cuda_error", "df_build_code", "df_code_from_lengths", "df_lut_words", "df_build_lut", "df_plan",
     "df_container_sizes",
     "df_histogram", "df_encode", "df_encode_noalloc", "df_decode", "df_decode_batch_workspace", "df_decode_batch_prepare",
     "df_decode_batch_run", "df_decode_batch", "df_read_error", "df_check_structure", "df_compare",
     "df_sha256_workspace", "df_sha256_device", "df_sha256",
+    "df_nf12_sizes_for", "df_nf12_encode_groups", "df_nf12_encode_escapes", "df_nf12_decode",
+    "df_nf12_decode_batch_workspace", "df_nf12_decode_batch_prepare", "df_nf12_decode_batch_run",
 )
 
 
@@ -101,6 +108,35 @@ class DfBatchPlan(ctypes.Structure):
     ]
 
 
+class DfNf12Sizes(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_uint64) for name in ("groups", "slots_bytes", "bitmap_bytes", "tiles", "encode_ws_bytes")]
+
+    def as_dict(self) -> dict:
+        return {name: int(getattr(self, name)) for name, _ in self._fields_}
+
+
+class DfNf12Tensor(ctypes.Structure):
+    _fields_ = [
+        ("n", ctypes.c_uint64),
+        ("n_escaped", ctypes.c_uint64),
+        ("slots", ctypes.c_void_p),
+        ("bitmap", ctypes.c_void_p),
+        ("side", ctypes.c_void_p),
+        ("out", ctypes.c_void_p),
+        ("top", ctypes.c_uint32),
+        ("reserved", ctypes.c_uint32),
+    ]
+
+
+class DfNf12Plan(ctypes.Structure):
+    _fields_ = [
+        ("d_ws", ctypes.c_void_p),
+        ("count", ctypes.c_uint32),
+        ("reserved", ctypes.c_uint32),
+        ("total_tiles", ctypes.c_uint64),
+    ]
+
+
 _lib = None
 
 
@@ -164,6 +200,20 @@ def lib() -> ctypes.CDLL:
     L.df_sha256_device.restype = i32
     L.df_sha256.argtypes = [vp, u64, vp]
     L.df_sha256.restype = i32
+    L.df_nf12_sizes_for.argtypes = [u64, ctypes.POINTER(DfNf12Sizes)]
+    L.df_nf12_sizes_for.restype = i32
+    L.df_nf12_encode_groups.argtypes = [vp, u64, u32, vp, vp, vp, sz, vp, vp]
+    L.df_nf12_encode_groups.restype = i32
+    L.df_nf12_encode_escapes.argtypes = [vp, u64, u32, vp, vp, vp, sz, vp, u64, vp, vp]
+    L.df_nf12_encode_escapes.restype = i32
+    L.df_nf12_decode.argtypes = [ctypes.POINTER(DfNf12Tensor), vp, vp]
+    L.df_nf12_decode.restype = i32
+    L.df_nf12_decode_batch_workspace.argtypes = [u32]
+    L.df_nf12_decode_batch_workspace.restype = sz
+    L.df_nf12_decode_batch_prepare.argtypes = [ctypes.POINTER(DfNf12Tensor), u32, vp, sz, ctypes.POINTER(DfNf12Plan), vp]
+    L.df_nf12_decode_batch_prepare.restype = i32
+    L.df_nf12_decode_batch_run.argtypes = [ctypes.POINTER(DfNf12Plan), vp, vp]
+    L.df_nf12_decode_batch_run.restype = i32
     _lib = L
     return L
 

@@ -1,5 +1,5 @@
-"""Python binding of the C ABI: one function per entry point of include/df11.h,
-same names, argument marshalling only. Device buffers are torch CUDA tensors
+"""Python binding of the C ABI: one function per entry point of include/df11.h
+and include/nf12.h, same names, argument marshalling only. Device buffers are torch CUDA tensors
 (PyTorch supplies memory and streams); every computation runs in libdf11.so.
 """
 from __future__ import annotations
@@ -9,7 +9,8 @@ import ctypes
 import numpy as np
 import torch
 
-from ._native import DfBatchPlan, DfCode, DfSizes, DfTensor, check, lib
+from ._native import (DfBatchPlan, DfCode, DfNf12Plan, DfNf12Sizes, DfNf12Tensor, DfSizes, DfTensor, check,
+                      lib)
 
 
 def _stream_ptr(stream=None):
@@ -249,3 +250,81 @@ def df_sha256(data) -> bytes:
     out = (ctypes.c_uint8 * 32)()
     check("df_sha256", lib().df_sha256(buf.ctypes.data if buf.size else None, buf.size, out))
     return bytes(out)
+
+
+# ---------------------------------------------------------------- nf12.h
+
+
+def df_nf12_sizes_for(n: int) -> DfNf12Sizes:
+    z = DfNf12Sizes()
+    check("df_nf12_sizes_for", lib().df_nf12_sizes_for(n, ctypes.byref(z)))
+    return z
+
+
+def df_nf12_encode_groups(d_in: torch.Tensor, top: int, d_slots: torch.Tensor, d_bitmap: torch.Tensor,
+                          d_ws: torch.Tensor, d_escaped: torch.Tensor, stream=None) -> None:
+    _need_u16(d_in, "d_in")
+    n = d_in.numel()
+    z = df_nf12_sizes_for(n)
+    _need(d_slots, z.slots_bytes, "d_slots")
+    _need(d_bitmap, z.bitmap_bytes, "d_bitmap")
+    _need(d_escaped, 8, "d_escaped")
+    check("df_nf12_encode_groups", lib().df_nf12_encode_groups(
+        _dev(d_in, "d_in"), n, top, _dev(d_slots, "d_slots"), _dev(d_bitmap, "d_bitmap"), _dev(d_ws, "d_ws"),
+        d_ws.numel() * d_ws.element_size(), _dev(d_escaped, "d_escaped"), _stream_ptr(stream)))
+
+
+def df_nf12_encode_escapes(d_in: torch.Tensor, top: int, d_slots: torch.Tensor, d_bitmap: torch.Tensor,
+                           d_ws: torch.Tensor, d_side: torch.Tensor | None, d_err: torch.Tensor | None = None,
+                           stream=None) -> None:
+    _need_u16(d_in, "d_in")
+    _need_err(d_err)
+    n = d_in.numel()
+    z = df_nf12_sizes_for(n)
+    _need(d_slots, z.slots_bytes, "d_slots")
+    _need(d_bitmap, z.bitmap_bytes, "d_bitmap")
+    cap = 0 if d_side is None else (d_side.numel() * d_side.element_size()) // 16
+    check("df_nf12_encode_escapes", lib().df_nf12_encode_escapes(
+        _dev(d_in, "d_in"), n, top, _dev(d_slots, "d_slots"), _dev(d_bitmap, "d_bitmap"), _dev(d_ws, "d_ws"),
+        d_ws.numel() * d_ws.element_size(), _dev(d_side, "d_side") if cap else None, cap, _dev(d_err, "d_err"),
+        _stream_ptr(stream)))
+
+
+def _nf12_check_tensor(t: DfNf12Tensor, d_out, name: str) -> None:
+    if isinstance(d_out, torch.Tensor):
+        _need_u16(d_out, name)
+        _need(d_out, 2 * t.n, name)
+
+
+def df_nf12_decode(t: DfNf12Tensor, d_out: torch.Tensor, d_err: torch.Tensor | None = None, stream=None) -> None:
+    """Decode one tensor into d_out (t.out is set from d_out)."""
+    _nf12_check_tensor(t, d_out, "d_out")
+    _need_err(d_err)
+    t.out = d_out if isinstance(d_out, int) else _dev(d_out, "d_out").value
+    check("df_nf12_decode", lib().df_nf12_decode(ctypes.byref(t), _dev(d_err, "d_err"), _stream_ptr(stream)))
+
+
+def df_nf12_decode_batch_workspace(count: int) -> int:
+    return int(lib().df_nf12_decode_batch_workspace(count))
+
+
+def df_nf12_decode_batch_prepare(tensors, d_outs, d_ws: torch.Tensor, stream=None) -> DfNf12Plan:
+    """tensors: DfNf12Tensor list; d_outs: one output (tensor or raw device pointer) each."""
+    if len(tensors) != len(d_outs):
+        raise ValueError("one output per tensor")
+    for i, (t, o) in enumerate(zip(tensors, d_outs)):
+        _nf12_check_tensor(t, o, f"d_outs[{i}]")
+        t.out = o if isinstance(o, int) else _dev(o, f"d_outs[{i}]").value
+    arr = (DfNf12Tensor * max(1, len(tensors)))(*tensors)
+    _need(d_ws, df_nf12_decode_batch_workspace(len(tensors)), "d_ws")
+    plan = DfNf12Plan()
+    check("df_nf12_decode_batch_prepare", lib().df_nf12_decode_batch_prepare(
+        arr, len(tensors), _dev(d_ws, "d_ws"), d_ws.numel() * d_ws.element_size(), ctypes.byref(plan),
+        _stream_ptr(stream)))
+    return plan
+
+
+def df_nf12_decode_batch_run(plan: DfNf12Plan, d_err: torch.Tensor | None = None, stream=None) -> None:
+    _need_err(d_err)
+    check("df_nf12_decode_batch_run", lib().df_nf12_decode_batch_run(ctypes.byref(plan), _dev(d_err, "d_err"),
+                                                                     _stream_ptr(stream)))

@@ -1,6 +1,7 @@
 """Build the in-tree native libraries.
 
-* ``libdf11.so``  the CUDA library (sm_100a only) behind ``include/df11.h``:
+* ``libdf11.so``  the CUDA library (sm_100a only) behind ``include/df11.h``
+  and ``include/nf12.h``:
   nvcc -gencode arch=compute_100a,code=sm_100a, static CUDA runtime.
 * ``libdfsynth.so``  the host-side seeded input generators (gcc).
 
@@ -19,7 +20,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libdf11.so")
 
-SOURCES = ["df_host.cpp", "df_decode.cu", "df_encode.cu", "df_verify.cu"]
+SOURCES = ["df_host.cpp", "df_decode.cu", "df_encode.cu", "df_verify.cu", "nf12.cu"]
 HEADERS = ["df_internal.h"]
 
 NVCC_FLAGS = [
@@ -44,7 +45,7 @@ def _stale(target: str, deps: list[str]) -> bool:
 
 def build_native(force: bool = False, verbose: bool = False) -> str:
     srcs = [os.path.join(CSRC, s) for s in SOURCES]
-    deps = srcs + [os.path.join(CSRC, h) for h in HEADERS] + [os.path.join(INCLUDE, "df11.h")]
+    deps = srcs + [os.path.join(CSRC, h) for h in HEADERS] + [os.path.join(INCLUDE, h) for h in ("df11.h", "nf12.h")]
     if not force and not _stale(LIB, deps):
         return LIB
     tmp = LIB + f".tmp{os.getpid()}"

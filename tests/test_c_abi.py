@@ -1,4 +1,5 @@
-"""The boundary is a C ABI: a C11 program that includes include/df11.h,
+"""The boundary is a C ABI: a C11 program that includes include/df11.h and
+include/nf12.h,
 links libdf11.so and calls the host-side entry points (no CUDA call is made).
 
 The program builds the code of a small histogram whose optimal lengths are
@@ -19,6 +20,7 @@ C_PROGRAM = textwrap.dedent(r"""
     #include <stdio.h>
     #include <string.h>
     #include "df11.h"
+    #include "nf12.h"
 
     int main(void) {
         uint64_t hist[256];
@@ -41,6 +43,10 @@ C_PROGRAM = textwrap.dedent(r"""
         if (df_plan(&code, hist, 16, 32, 256, &z) != DF_OK) return 7;
         if (z.total_bits != 8 * 1 + 4 * 2 + 2 * 3 + 1 * 4 + 1 * 4) return 8;
         if (df_plan(&code, hist, 17, 32, 256, &z) != DF_ERR_INVALID_ARG) return 9;  /* total != n */
+        df_nf12_sizes nz;
+        if (df_nf12_sizes_for(17, &nz) != DF_OK) return 11;
+        if (nz.groups != 3 || nz.slots_bytes != 36 || nz.bitmap_bytes != 4 || nz.tiles != 1) return 12;
+        if (df_nf12_sizes_for(17, NULL) != DF_ERR_INVALID_ARG) return 13;
         const char* s = df_status_string(DF_ERR_CORRUPT);
         if (!s || !s[0]) return 10;
         printf("c abi ok: %u symbols, %zu table words, %llu bits\n", code.n_symbols, words,
@@ -60,7 +66,7 @@ def libdir():
 
 def test_header_compiles_as_c11(tmp_path):
     src = tmp_path / "h.c"
-    src.write_text('#include "df11.h"\nint main(void) { return DF_OK; }\n')
+    src.write_text('#include "df11.h"\n#include "nf12.h"\nint main(void) { return DF_OK; }\n')
     subprocess.check_call(["gcc", "-std=c11", "-Wall", "-Wextra", "-Werror", "-pedantic", "-fsyntax-only",
                            "-I", os.path.join(ROOT, "include"), str(src)])
 

@@ -24,9 +24,15 @@ def built():
     build.build_native()
 
 
+HEADERS = ("df11.h", "nf12.h")
+
+
+def header_text() -> str:
+    return "\n".join(open(os.path.join(ROOT, "include", h)).read() for h in HEADERS)
+
+
 def header_functions():
-    text = open(os.path.join(ROOT, "include", "df11.h")).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"/\*.*?\*/", "", header_text(), flags=re.S)
     return sorted(set(re.findall(r"\b(df_[a-z0-9_]+)\s*\(", text)))
 
 
@@ -43,7 +49,7 @@ def test_every_declaration_names_its_source():
     """Each function declared in the header is preceded by a comment that
     names the page passage it follows ("Source: ...") or says that the pages
     have none."""
-    text = open(os.path.join(ROOT, "include", "df11.h")).read()
+    text = header_text()
     for name in header_functions():
         m = re.search(r"/\*((?:(?!\*/).)*)\*/\s*(?:#define[^\n]*\n\s*)*[A-Za-z_][A-Za-z_0-9 *]*\b" + name + r"\(",
                       text, flags=re.S)
@@ -59,6 +65,20 @@ def test_struct_sizes_match_header_layout():
     assert ctypes.sizeof(_native.DfSizes) == 9 * 8
     assert ctypes.sizeof(_native.DfTensor) == 16 + 16 + 5 * 8 + 256
     assert ctypes.sizeof(_native.DfBatchPlan) == 8 + 8 * 4 + 8
+    assert ctypes.sizeof(_native.DfNf12Sizes) == 5 * 8
+    assert ctypes.sizeof(_native.DfNf12Tensor) == 16 + 4 * 8 + 8
+    assert ctypes.sizeof(_native.DfNf12Plan) == 8 + 8 + 8
+
+
+@pytest.mark.parametrize("n", [0, 1, 7, 8, 9, 16383, 16384, 16385, 10**7 + 3])
+def test_nf12_sizes_match_the_oracle(n):
+    from oracle import nf12_oracle
+
+    z = api.df_nf12_sizes_for(n).as_dict()
+    o = nf12_oracle.sizes(n, 0)
+    assert (z["groups"], z["slots_bytes"], z["bitmap_bytes"]) == (o["groups"], o["slots_bytes"], o["bitmap_bytes"])
+    assert z["tiles"] == -(-o["groups"] // 2048)
+    assert z["encode_ws_bytes"] == 8 * (z["tiles"] + 1)
 
 
 def _random_hist(rng, kind):
