@@ -70,6 +70,8 @@ typedef int df_status;
 #define DF_EFLAG_ENC_TOTAL 16u    /* encode: stream length != the planned total_bits   */
 #define DF_EFLAG_ENC_SYMBOL 32u   /* encode: an exponent without a code                */
 #define DF_EFLAG_ENC_WAIT 64u     /* encode: a tile waited too long for the one before */
+#define DF_EFLAG_INDEX8 256u      /* compact index: wide superblocks past the room given,
+                                     or an overflow slot past the wide count          */
 
 #define DF_DEFAULT_CHUNK_BYTES 32u
 #define DF_DEFAULT_THREADS_PER_BLOCK 32u
@@ -104,10 +106,15 @@ typedef struct df_tensor {
     uint32_t n_tables;
     const uint8_t* stream;         /* 16-byte aligned                 */
     const uint8_t* gaps;
-    const uint64_t* block_offsets; /* 8-byte aligned                  */
+    const uint64_t* block_offsets; /* 8-byte aligned; NULL when the compact
+                                      index below is given instead     */
     const uint8_t* sm;             /* 8-byte aligned for vector loads  */
     const uint32_t* lut;           /* 16-byte aligned                 */
     uint8_t lengths[256];          /* host copy of the code lengths   */
+    const uint8_t* index8;         /* compact block index (df_index8_build),
+                                      8-byte aligned; used when
+                                      block_offsets is NULL, else NULL */
+    uint64_t index8_wide;          /* its wide superblocks (df_index8_build) */
 } df_tensor;
 
 /* Host plan of a grouped decode, filled by df_decode_batch_prepare. */
@@ -346,6 +353,46 @@ df_status df_sha256_device(const void* d_data, uint64_t nbytes, void* d_ws, size
 /* df_sha256: plain SHA-256 (FIPS 180-4) of nbytes of host data. Source: as
  * df_sha256_device. Errors: DF_ERR_INVALID_ARG. */
 df_status df_sha256(const void* data, uint64_t nbytes, uint8_t digest[32]);
+
+/* ---- compact block index ----------------------------------------------
+ * In place of one uint64 output offset per format block (block_offsets,
+ * O[0] = 0 .. O[B] = n; block b holds c_b = O[b+1] - O[b] codes), blocks are
+ * grouped in superblocks of 64, S = ceil(B / 64), and one buffer holds:
+ *   [0, 8S)          anchor[s], uint64: O[64 s]
+ *   [8S, 12S)        base[s], uint32: the smallest count of superblock s when
+ *                    all its counts lie within 255 of it; else 2^31 | k, k =
+ *                    how many wide superblocks come before s
+ *   [12S, 76S)       delta[b], uint8: c_b - base[s] (0 in a wide superblock
+ *                    and past the last block)
+ *   [76S, 76S+256W)  overflow: the 64 counts (uint32) of each of the W wide
+ *                    superblocks, in order (0 past the last block)
+ * So O[64 s + j] = anchor[s] + c_{64 s} + ... + c_{64 s + j - 1}. Source:
+ * df11pack (GitHub page), "What is checked, and what is not", opt-in
+ * --index idx8: an experimental 8-bit block index that makes the file
+ * smaller; the page gives no layout, this one is the library's own. */
+
+/* Bytes of a compact index of n_blocks blocks with n_wide wide superblocks:
+ * 76 ceil(n_blocks / 64) + 256 n_wide. Source: as above. */
+uint64_t df_index8_bytes(uint64_t n_blocks, uint64_t n_wide);
+
+/* Build the compact index of d_offsets (n_blocks + 1 device uint64 offsets)
+ * into d_index8 (index8_bytes bytes, 8-byte aligned). Wide superblocks past
+ * the room that index8_bytes leaves for the overflow are not written and set
+ * DF_EFLAG_INDEX8 in d_err (nullable); *d_n_wide (device uint64) gets the
+ * number of wide superblocks, so a caller that gave room for none reads it
+ * and builds again. A count of 2^31 or more also sets DF_EFLAG_INDEX8.
+ * Source: as above. Errors: DF_ERR_INVALID_ARG (null, misaligned, index8_bytes
+ * below df_index8_bytes(n_blocks, 0)), DF_ERR_UNSUPPORTED (n_blocks >= 2^32),
+ * DF_ERR_CUDA. */
+df_status df_index8_build(const uint64_t* d_offsets, uint64_t n_blocks, void* d_index8, size_t index8_bytes,
+                          uint64_t* d_n_wide, uint32_t* d_err, void* stream);
+
+/* The block offsets (n_blocks + 1 device uint64, O[0] from anchor[0]) back
+ * from a compact index with n_wide wide superblocks. An overflow slot at or
+ * past n_wide sets DF_EFLAG_INDEX8 in d_err (nullable) and counts as 0.
+ * Source: as above. Errors: DF_ERR_INVALID_ARG, DF_ERR_UNSUPPORTED, DF_ERR_CUDA. */
+df_status df_index8_expand(const void* d_index8, uint64_t n_blocks, uint64_t n_wide, uint64_t* d_offsets,
+                           uint32_t* d_err, void* stream);
 
 #ifdef __cplusplus
 }

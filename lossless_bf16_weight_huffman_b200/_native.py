@@ -27,6 +27,7 @@ DF_EFLAG_ENC_TOTAL = 16
 DF_EFLAG_ENC_SYMBOL = 32
 DF_EFLAG_ENC_WAIT = 64
 DF_EFLAG_NF12_SIDE = 128
+DF_EFLAG_INDEX8 = 256
 
 DF_NF12_TOP = 7
 DF_NF12_TILE_GROUPS = 2048
@@ -39,7 +40,8 @@ EXPORTS = (
     "df_container_sizes",
     "df_histogram", "df_encode", "df_encode_noalloc", "df_decode", "df_decode_batch_workspace", "df_decode_batch_prepare",
     "df_decode_batch_run", "df_decode_batch", "df_read_error", "df_check_structure", "df_compare",
-    "df_sha256_workspace", "df_sha256_device", "df_sha256",
+    "df_sha256_workspace", "df_sha256_device", "df_sha256", "df_index8_bytes", "df_index8_build",
+    "df_index8_expand",
     "df_nf12_sizes_for", "df_nf12_encode_groups", "df_nf12_encode_escapes", "df_nf12_decode",
     "df_nf12_decode_batch_workspace", "df_nf12_decode_batch_prepare", "df_nf12_decode_batch_run",
 )
@@ -90,6 +92,8 @@ class DfTensor(ctypes.Structure):
         ("sm", ctypes.c_void_p),
         ("lut", ctypes.c_void_p),
         ("lengths", ctypes.c_uint8 * 256),
+        ("index8", ctypes.c_void_p),
+        ("index8_wide", ctypes.c_uint64),
     ]
 
 
@@ -200,6 +204,12 @@ def lib() -> ctypes.CDLL:
     L.df_sha256_device.restype = i32
     L.df_sha256.argtypes = [vp, u64, vp]
     L.df_sha256.restype = i32
+    L.df_index8_bytes.argtypes = [u64, u64]
+    L.df_index8_bytes.restype = u64
+    L.df_index8_build.argtypes = [vp, u64, vp, sz, vp, vp, vp]
+    L.df_index8_build.restype = i32
+    L.df_index8_expand.argtypes = [vp, u64, u64, vp, vp, vp]
+    L.df_index8_expand.restype = i32
     L.df_nf12_sizes_for.argtypes = [u64, ctypes.POINTER(DfNf12Sizes)]
     L.df_nf12_sizes_for.restype = i32
     L.df_nf12_encode_groups.argtypes = [vp, u64, u32, vp, vp, vp, sz, vp, vp]

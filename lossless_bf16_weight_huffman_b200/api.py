@@ -252,6 +252,30 @@ def df_sha256(data) -> bytes:
     return bytes(out)
 
 
+def df_index8_bytes(n_blocks: int, n_wide: int) -> int:
+    return int(lib().df_index8_bytes(n_blocks, n_wide))
+
+
+def df_index8_build(d_offsets: torch.Tensor, n_blocks: int, d_index8: torch.Tensor, d_n_wide: torch.Tensor,
+                    d_err: torch.Tensor | None = None, stream=None) -> None:
+    _need(d_offsets, 8 * (n_blocks + 1), "d_offsets")
+    _need(d_n_wide, 8, "d_n_wide")
+    _need_err(d_err)
+    check("df_index8_build", lib().df_index8_build(
+        _dev(d_offsets, "d_offsets"), n_blocks, _dev(d_index8, "d_index8"), d_index8.numel() * d_index8.element_size(),
+        _dev(d_n_wide, "d_n_wide"), _dev(d_err, "d_err"), _stream_ptr(stream)))
+
+
+def df_index8_expand(d_index8: torch.Tensor, n_blocks: int, n_wide: int, d_offsets: torch.Tensor,
+                     d_err: torch.Tensor | None = None, stream=None) -> None:
+    _need(d_index8, df_index8_bytes(n_blocks, n_wide), "d_index8")
+    _need(d_offsets, 8 * (n_blocks + 1), "d_offsets")
+    _need_err(d_err)
+    check("df_index8_expand", lib().df_index8_expand(
+        _dev(d_index8, "d_index8"), n_blocks, n_wide, _dev(d_offsets, "d_offsets"), _dev(d_err, "d_err"),
+        _stream_ptr(stream)))
+
+
 # ---------------------------------------------------------------- nf12.h
 
 

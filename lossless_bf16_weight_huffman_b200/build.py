@@ -20,7 +20,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libdf11.so")
 
-SOURCES = ["df_host.cpp", "df_decode.cu", "df_encode.cu", "df_verify.cu", "nf12.cu"]
+SOURCES = ["df_host.cpp", "df_decode.cu", "df_encode.cu", "df_verify.cu", "df_index8.cu", "nf12.cu"]
 HEADERS = ["df_internal.h"]
 
 NVCC_FLAGS = [

@@ -30,7 +30,10 @@ def _as_u16(w: torch.Tensor) -> torch.Tensor:
 class Compressed:
     """One tensor's container in device memory."""
 
-    def __init__(self, *, n, shape, code, lut, sizes, chunk_bytes, threads_per_block, stream, gaps, offsets, sm):
+    def __init__(self, *, n, shape, code, lut, sizes, chunk_bytes, threads_per_block, stream, gaps, offsets, sm,
+                 index8=None, index8_wide=0):
+        if (offsets is None) == (index8 is None):
+            raise ValueError("a container holds exactly one block index: offsets or index8")
         self.n = int(n)
         self.shape = tuple(shape)
         self.code = code
@@ -40,7 +43,9 @@ class Compressed:
         self.threads_per_block = threads_per_block
         self.stream = stream
         self.gaps = gaps
-        self.offsets = offsets
+        self.offsets = offsets      # uint64 block offsets, or None with the compact index
+        self.index8 = index8        # compact block index (df_index8_build), or None
+        self.index8_wide = int(index8_wide)
         self.sm = sm
         self._desc = None
 
@@ -49,8 +54,24 @@ class Compressed:
         return self.sizes["total_bits"]
 
     @property
+    def index_kind(self) -> str:
+        return "u64" if self.offsets is not None else "idx8"
+
+    @property
+    def index_bytes(self) -> int:
+        """Bytes of the block index this container holds."""
+        if self.offsets is not None:
+            return self.sizes["offsets_bytes"]
+        return api.df_index8_bytes(self.sizes["n_blocks"], self.index8_wide)
+
+    @property
+    def index(self) -> torch.Tensor:
+        """The block index part: uint64 offsets or the compact index bytes."""
+        return self.offsets if self.offsets is not None else self.index8
+
+    @property
     def container_bytes(self) -> int:
-        return self.sizes["container_bytes"]
+        return self.sizes["container_bytes"] - self.sizes["offsets_bytes"] + self.index_bytes
 
     @property
     def ratio(self) -> float:
@@ -61,9 +82,36 @@ class Compressed:
         return np.frombuffer(bytes(self.code.lengths), np.uint8).copy()
 
     def read_bytes(self) -> int:
-        """Bytes a full decode must read: the stream, gaps, offsets and sm bytes."""
+        """Bytes a full decode must read: the stream, gaps, block index and sm bytes."""
         z = self.sizes
-        return z["stream_bytes"] + z["gap_bytes"] + z["offsets_bytes"] + z["sm_bytes"]
+        return z["stream_bytes"] + z["gap_bytes"] + self.index_bytes + z["sm_bytes"]
+
+    def block_offsets(self, stream=None) -> torch.Tensor:
+        """The uint64 block offsets on the device (expanded from the compact
+        index into a new tensor when that is what the container holds)."""
+        if self.offsets is not None:
+            return self.offsets
+        o = torch.empty(self.sizes["n_blocks"] + 1, dtype=torch.int64, device=self.stream.device)
+        api.df_index8_expand(self.index8, self.sizes["n_blocks"], self.index8_wide, o, None, stream)
+        return o
+
+    def use_index8(self, d_err: torch.Tensor | None = None, stream=None) -> "Compressed":
+        """Replace the uint64 block offsets by the compact index (df11pack,
+        "What is checked": --index idx8). Waits for the stream once to learn
+        the number of wide superblocks."""
+        if self.offsets is None:
+            return self
+        nb = self.sizes["n_blocks"]
+        dev = self.offsets.device
+        wide = torch.zeros(1, dtype=torch.int64, device=dev)
+        ix = torch.empty(max(api.df_index8_bytes(nb, 0), 16), dtype=torch.uint8, device=dev)
+        api.df_index8_build(self.offsets, nb, ix, wide, None, stream)
+        w = int(wide.cpu().item())
+        if w:  # room for the wide superblocks' counts, then again
+            ix = torch.empty(api.df_index8_bytes(nb, w), dtype=torch.uint8, device=dev)
+            api.df_index8_build(self.offsets, nb, ix, wide, d_err, stream)
+        self.index8, self.index8_wide, self.offsets, self._desc = ix, w, None, None
+        return self
 
     def descriptor(self) -> DfTensor:
         if self._desc is None:
@@ -76,7 +124,11 @@ class Compressed:
             d.n_tables = self.code.n_tables
             d.stream = self.stream.data_ptr()
             d.gaps = self.gaps.data_ptr()
-            d.block_offsets = self.offsets.data_ptr()
+            if self.offsets is not None:
+                d.block_offsets = self.offsets.data_ptr()
+            else:
+                d.index8 = self.index8.data_ptr()
+                d.index8_wide = self.index8_wide
             d.sm = self.sm.data_ptr() if self.n else self.stream.data_ptr()
             d.lut = self.lut.data_ptr()
             d.lengths[:] = self.code.lengths[:]
@@ -86,16 +138,22 @@ class Compressed:
     @classmethod
     def from_host(cls, *, lengths, max_len, total_bits, n, stream, gaps, offsets, sm, shape=None,
                   chunk_bytes=DEFAULT_CHUNK_BYTES, threads_per_block=DEFAULT_THREADS_PER_BLOCK,
-                  device="cuda"):
-        """Upload a container whose parts are host arrays (e.g. read from a file)."""
+                  device="cuda", index8=None, index8_wide=0):
+        """Upload a container whose parts are host arrays (e.g. read from a
+        file); give either offsets or index8 (with index8_wide)."""
         code = api.df_code_from_lengths(lengths, max_len)
         lut = torch.from_numpy(api.df_build_lut(code).view(np.int32)).to(device)
+        if offsets is not None:
+            n_blocks = int(np.asarray(offsets).size) - 1
+        else:
+            n_blocks = api.df_container_sizes(int(n), int(total_bits), chunk_bytes, threads_per_block).n_blocks
         hist_free = {
             "total_bits": int(total_bits),
             "stream_bytes": int(np.asarray(stream).size),
             "gap_bytes": int(np.asarray(gaps).size),
-            "offsets_bytes": 8 * int(np.asarray(offsets).size),
+            "offsets_bytes": 8 * (n_blocks + 1),
             "sm_bytes": int(n),
+            "n_blocks": n_blocks,
         }
         hist_free["container_bytes"] = (hist_free["stream_bytes"] + hist_free["gap_bytes"] +
                                         hist_free["offsets_bytes"] + int(n) + 256 + 64)
@@ -104,8 +162,10 @@ class Compressed:
         return cls(n=n, shape=shape or (n,), code=code, lut=lut, sizes=hist_free, chunk_bytes=chunk_bytes,
                    threads_per_block=threads_per_block, stream=t(np.asarray(stream, np.uint8), np.uint8),
                    gaps=t(np.asarray(gaps, np.uint8), np.uint8),
-                   offsets=t(np.asarray(offsets, np.uint64), np.int64),
-                   sm=t(sm_arr if sm_arr.size else np.zeros(16, np.uint8), np.uint8))
+                   offsets=t(np.asarray(offsets, np.uint64), np.int64) if offsets is not None else None,
+                   sm=t(sm_arr if sm_arr.size else np.zeros(16, np.uint8), np.uint8),
+                   index8=t(np.asarray(index8, np.uint8), np.uint8) if index8 is not None else None,
+                   index8_wide=index8_wide)
 
 
 def auto_chunk_bytes(code) -> int:
@@ -120,11 +180,14 @@ class SafeCheckError(RuntimeError):
 
 def compress(w: torch.Tensor, max_len: int = DEFAULT_MAX_LEN, chunk_bytes: int | None = None,
              threads_per_block: int = DEFAULT_THREADS_PER_BLOCK, d_err: torch.Tensor | None = None,
-             stream=None, safe: bool = False) -> Compressed:
+             stream=None, safe: bool = False, index: str = "u64") -> Compressed:
     """Histogram on the GPU, code build on the host, encode on the GPU.
     chunk_bytes=None picks auto_chunk_bytes(code). safe=True decodes the new
     container and compares it with w on the GPU before returning (df11pack,
-    "Use": --safe), raising SafeCheckError on any difference."""
+    "Use": --safe), raising SafeCheckError on any difference. index="idx8"
+    keeps the compact block index in place of the uint64 offsets."""
+    if index not in ("u64", "idx8"):
+        raise ValueError("index is 'u64' or 'idx8'")
     x = _as_u16(w)
     dev = x.device
     n = x.numel()
@@ -145,6 +208,8 @@ def compress(w: torch.Tensor, max_len: int = DEFAULT_MAX_LEN, chunk_bytes: int |
                   sm, ws, d_err, stream)
     c = Compressed(n=n, shape=tuple(w.shape), code=code, lut=lut, sizes=z, chunk_bytes=chunk_bytes,
                    threads_per_block=threads_per_block, stream=stream_buf, gaps=gaps, offsets=offsets, sm=sm)
+    if index == "idx8":
+        c.use_index8(d_err, stream)
     if safe and n:
         err = torch.zeros(1, dtype=torch.int32, device=dev)
         api.df_read_error(err, stream)

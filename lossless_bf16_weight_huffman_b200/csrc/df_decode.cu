@@ -121,6 +121,35 @@ __device__ __noinline__ uint32_t long_code(uint32_t win, const uint32_t* __restr
     return ((e >> kNsymShift) & 3u) ? e : 0;
 }
 
+// Compact block index (superblocks of 64 format blocks): codes in block b.
+// A wide superblock's overflow slot past the wide count marks *bad.
+__device__ __forceinline__ uint32_t idx8_count(const DevTensor* td, uint64_t b, bool* bad) {
+    const uint64_t S = (static_cast<uint64_t>(td->n_blocks) + 63) >> 6;
+    const uint8_t* ix = reinterpret_cast<const uint8_t*>(td->offs);
+    const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(ix + 8 * S) + (b >> 6));
+    if (!(w & 0x80000000u)) return w + __ldg(ix + 12 * S + b);
+    const uint32_t slot = w & 0x7FFFFFFFu;
+    if (slot + 1 >= td->idx8) {
+        *bad = true;
+        return 0;
+    }
+    return __ldg(reinterpret_cast<const uint32_t*>(ix + 76 * S) + 64ull * slot + (b & 63));
+}
+
+// Output index of block b's first code from the compact index: its
+// superblock's anchor plus the counts of the blocks before it there (each
+// lane adds two of them). Called by the whole warp.
+__device__ __noinline__ uint64_t idx8_start(const DevTensor* td, uint64_t b, uint32_t lane, bool* bad) {
+    const uint64_t s0 = b & ~63ull;
+    bool bd = false;
+    uint32_t c = 0;
+    if (s0 + lane < b) c += idx8_count(td, s0 + lane, &bd);
+    if (s0 + lane + 32 < b) c += idx8_count(td, s0 + lane + 32, &bd);
+    const uint32_t sum = __reduce_add_sync(0xffffffffu, c);  // a valid superblock's counts sum below 2^29
+    if (__any_sync(0xffffffffu, bd)) *bad = true;
+    return __ldg(reinterpret_cast<const uint64_t*>(td->offs) + (b >> 6)) + sum;
+}
+
 __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v, uint32_t lane) {
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
@@ -371,14 +400,24 @@ __global__ void __launch_bounds__(kMaxWarps * kLanes, 1)
         uint64_t b = wb0 - t_lo;  // local index of the current block
         const uint64_t c_end = min((wb1 - t_lo) * T, n_chunks);
         uint64_t c = b * T;                 // first chunk of the current round
-        uint64_t outr = td->offs[b];        // output index of the round's first code
+        bool bad_index = false;
+        uint64_t outr = td->idx8 ? idx8_start(td, b, lane, &bad_index)  // output index of the round's first code
+                                 : td->offs[b];
         const uint64_t vstart = outr;       // outputs before it belong to the previous run
         bool pre = false;      // this lane's chunk of the round is already in its slot
         uint32_t pre_two = 0;  // and its two gap bytes
-        bool ok = outr <= td->n;
+        bool ok = outr <= td->n && !bad_index;
         if (!ok && lane == 0 && d_err) atomicOr(d_err, DF_EFLAG_OFFSETS);
         while (ok && c < c_end) {  // the run's blocks
-            const uint64_t out1 = td->offs[b + 1];
+            // a block starts where the one before ended (checked at its end)
+            uint64_t out1;
+            if (td->idx8) {
+                bool bad = false;
+                const uint32_t cnt = idx8_count(td, b, &bad);
+                out1 = bad ? ~0ull : outr + cnt;
+            } else {
+                out1 = td->offs[b + 1];
+            }
             if (out1 < outr || out1 > td->n || (b + 1 == td->n_blocks && out1 != td->n)) {
                 if (lane == 0 && d_err) atomicOr(d_err, DF_EFLAG_OFFSETS);
                 break;
@@ -620,8 +659,10 @@ df_status prepare(const df_tensor* t, uint16_t* out, Prepared* pr) {
     if (C > 1024) return DF_ERR_UNSUPPORTED;
     if (t->max_len < 1 || t->max_len > 32 || t->n_tables < 1) return DF_ERR_INVALID_ARG;
     if (t->n > DF_MAX_WEIGHTS) return DF_ERR_UNSUPPORTED;
-    if (!t->stream || !t->gaps || !t->block_offsets || !t->sm || !t->lut) return DF_ERR_INVALID_ARG;
-    if (!aligned(t->stream, 16) || !aligned(t->lut, 16) || !aligned(t->block_offsets, 8) || !aligned(out, 2))
+    if (!t->stream || !t->gaps || !t->sm || !t->lut) return DF_ERR_INVALID_ARG;
+    if (!t->block_offsets == !t->index8) return DF_ERR_INVALID_ARG;  // exactly one block index
+    if (!aligned(t->stream, 16) || !aligned(t->lut, 16) || !aligned(t->block_offsets, 8) ||
+        !aligned(t->index8, 8) || !aligned(out, 2))
         return DF_ERR_INVALID_ARG;
     const uint32_t minl = min_len_of(t->lengths);
     if (t->n > 0 && minl == 0) return DF_ERR_INVALID_ARG;
@@ -635,7 +676,13 @@ df_status prepare(const df_tensor* t, uint16_t* out, Prepared* pr) {
     std::memset(&d, 0, sizeof(d));
     d.stream = t->stream;
     d.gaps = t->gaps;
-    d.offs = t->block_offsets;
+    if (t->index8) {
+        if (t->index8_wide > (n_blocks + 63) / 64) return DF_ERR_INVALID_ARG;
+        d.offs = reinterpret_cast<const uint64_t*>(t->index8);
+        d.idx8 = static_cast<uint32_t>(t->index8_wide + 1);
+    } else {
+        d.offs = t->block_offsets;
+    }
     d.sm = t->sm;
     d.lut = t->lut;
     d.out = out;

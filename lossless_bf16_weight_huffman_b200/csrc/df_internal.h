@@ -12,7 +12,7 @@ namespace df {
 struct DevTensor {
     const uint8_t* stream;
     const uint8_t* gaps;
-    const uint64_t* offs;
+    const uint64_t* offs;  // block offsets, or the compact index when idx8 != 0
     const uint8_t* sm;
     const uint32_t* lut;   // n_tables*256 table words, then 64 words of lengths
     uint16_t* out;
@@ -24,7 +24,8 @@ struct DevTensor {
     uint32_t chunk_bytes;  // C
     uint32_t tpb;          // T: chunks per format block
     uint32_t vec_ok;       // sm and out 16-byte aligned
-    uint32_t pad;
+    uint32_t idx8;         // 0: offs holds uint64 block offsets; else the compact
+                           // index with idx8 - 1 wide superblocks
 };
 static_assert(sizeof(DevTensor) % 16 == 0, "descriptors are copied and placed in 16-byte units");
 

@@ -111,7 +111,7 @@ class HostLayerStreamer:
     consumer on its stream; copy, decode and consumption of consecutive layers
     overlap."""
 
-    PARTS = ("stream", "gaps", "offsets", "sm")
+    PARTS = ("stream", "gaps", "index", "sm")  # index: uint64 offsets or the compact index
 
     def __init__(self, layers: Sequence[Sequence[codec.Compressed]], device=None):
         self.layers = [list(l) for l in layers]
@@ -167,10 +167,11 @@ class HostLayerStreamer:
             h = self.host[i][j][k]
             view = self.stage[s][k][off: off + h.numel() * h.element_size()]
             parts[k] = view.view(h.dtype)
+        u64 = c.offsets is not None
         return codec.Compressed(n=c.n, shape=c.shape, code=c.code, lut=c.lut, sizes=c.sizes,
                                 chunk_bytes=c.chunk_bytes, threads_per_block=c.threads_per_block,
-                                stream=parts["stream"], gaps=parts["gaps"], offsets=parts["offsets"],
-                                sm=parts["sm"])
+                                stream=parts["stream"], gaps=parts["gaps"], offsets=parts["index"] if u64 else None,
+                                sm=parts["sm"], index8=None if u64 else parts["index"], index8_wide=c.index8_wide)
 
     def _copy_in(self, i: int) -> None:
         s = i % 2

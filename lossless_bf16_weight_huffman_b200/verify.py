@@ -24,6 +24,7 @@ Every step runs in libdf11.so; this module builds descriptors and reads flags.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import sys
 
 import numpy as np
@@ -53,10 +54,16 @@ def check_structure(c: codec.Compressed) -> str | None:
         z = api.df_container_sizes(c.n, c.total_bits, c.chunk_bytes, c.threads_per_block).as_dict()
     except DfError as e:
         return f"impossible sizes: {e}"
-    have = {"stream_bytes": c.stream.numel(), "gap_bytes": c.gaps.numel(), "offsets_bytes": 8 * c.offsets.numel()}
+    have = {"stream_bytes": c.stream.numel(), "gap_bytes": c.gaps.numel()}
+    if c.offsets is not None:
+        have["offsets_bytes"] = 8 * c.offsets.numel()
     for k, v in have.items():
         if v < z[k]:
             return f"{k}: {v} < {z[k]}"
+    if c.index8 is not None:
+        need = api.df_index8_bytes(z["n_blocks"], c.index8_wide)
+        if c.index8.numel() < need or c.index8_wide > (z["n_blocks"] + 63) // 64:
+            return f"compact block index: {c.index8.numel()} bytes for {c.index8_wide} wide superblocks"
     if c.sm.numel() < c.n:
         return "sign|fraction bytes shorter than n"
     try:
@@ -66,11 +73,32 @@ def check_structure(c: codec.Compressed) -> str | None:
     if c.n == 0:
         return None
     fl = _flags(c.stream.device)
-    api.df_check_structure(c.descriptor(), fl)
+    d = _with_offsets(c, _offsets_of(c, fl))
+    api.df_check_structure(d, fl)
     return "block offsets" if api.df_read_error(fl) else None
 
 
-def _block_descriptor(c: codec.Compressed, b: int, offs: tuple[int, int]) -> DfTensor:
+def _offsets_of(c: codec.Compressed, fl: torch.Tensor) -> torch.Tensor:
+    """The container's uint64 block offsets (expanded on the GPU from a
+    compact index; a bad overflow slot there sets DF_EFLAG_INDEX8 in fl)."""
+    if c.offsets is not None:
+        return c.offsets
+    o = torch.empty(c.sizes["n_blocks"] + 1, dtype=torch.int64, device=c.stream.device)
+    api.df_index8_expand(c.index8, c.sizes["n_blocks"], c.index8_wide, o, fl)
+    return o
+
+
+def _with_offsets(c: codec.Compressed, offsets: torch.Tensor) -> DfTensor:
+    d = DfTensor()
+    ctypes.memmove(ctypes.byref(d), ctypes.byref(c.descriptor()), ctypes.sizeof(d))
+    d.block_offsets = offsets.data_ptr()
+    d.index8 = None
+    d.index8_wide = 0
+    d._keep = offsets
+    return d
+
+
+def _block_descriptor(c: codec.Compressed, offsets: torch.Tensor, b: int, offs: tuple[int, int]) -> DfTensor:
     """A descriptor of format block b alone: the stream, gaps and offsets from
     the block's start; output indices stay absolute (n = the block's end)."""
     T, C = c.threads_per_block, c.chunk_bytes
@@ -84,7 +112,7 @@ def _block_descriptor(c: codec.Compressed, b: int, offs: tuple[int, int]) -> DfT
     d.n_tables = c.code.n_tables
     d.stream = c.stream.data_ptr() + b * T * C
     d.gaps = c.gaps.data_ptr() + (5 * T * b) // 8  # T is a multiple of 32: the block's fields start on a byte
-    d.block_offsets = c.offsets.data_ptr() + 8 * b
+    d.block_offsets = offsets.data_ptr() + 8 * b
     d.sm = c.sm.data_ptr()
     d.lut = c.lut.data_ptr()
     d.lengths[:] = c.code.lengths[:]
@@ -109,9 +137,13 @@ def check_sampled(entries, source: dict, samples: int = 1000, seed: int = 0) -> 
         ti = int(np.searchsorted(starts, g, side="right") - 1)
         chosen.append((ti, int(g - starts[ti])))
     # the block offsets of the chosen blocks
+    fl0 = _flags(dev)
+    full = {ti: _offsets_of(comps[ti][1], fl0) for ti in sorted({ti for ti, _ in chosen})}
+    if api.df_read_error(fl0):
+        return FAIL, "compact block index"
     offs = []
     for ti, b in chosen:
-        o = comps[ti][1].offsets[b: b + 2].cpu().numpy().view(np.uint64)
+        o = full[ti][b: b + 2].cpu().numpy().view(np.uint64)
         offs.append((int(o[0]), int(o[1])))
     if any(o[1] < o[0] or o[1] > comps[ti][1].n for (ti, _), o in zip(chosen, offs)):
         return FAIL, "block offsets out of range"
@@ -122,7 +154,7 @@ def check_sampled(entries, source: dict, samples: int = 1000, seed: int = 0) -> 
         # place the block's outputs so that its absolute index o[0] lands at a
         # 16-byte-aligned view (the decoder then takes its vector path)
         pos += (-(pos - o[0])) % 8
-        descs.append(_block_descriptor(comps[ti][1], b, o))
+        descs.append(_block_descriptor(comps[ti][1], full[ti], b, o))
         outs.append(buf.data_ptr() + 2 * (pos - o[0]))
         views.append(buf[pos: pos + n])
         pos += n

@@ -77,3 +77,46 @@ def test_damaged_files_are_refused(tmp_path):
     open(bad, "wb").write(raw[:24] + hb + raw[24 + old_len:])
     with pytest.raises(container_file.FormatError):
         container_file.load(bad, device="cpu")
+
+
+def _index8_bytes(offsets):
+    from oracle import index8
+
+    a, b, d, o = index8.build(offsets)
+    return np.concatenate([a.view(np.uint8), b.view(np.uint8), d, o.view(np.uint8)]), o.size // 64
+
+
+def test_save_load_compact_index(tmp_path):
+    """A container that holds the compact block index (oracle-built) in place
+    of the uint64 offsets: saved, loaded back byte for byte, with a wide
+    superblock among its superblocks."""
+    w = np.concatenate([synth.generate(synth.single_1024x4096()[0])[:600_000], np.full(400_000, 0x3F80, np.uint16),
+                        synth.generate(synth.heavy_tail_64m()[0])[:300_001]])
+    enc = oracle.encode(w, chunk_bytes=32, threads_per_block=32)
+    ix, wide = _index8_bytes(enc.offsets)
+    assert wide >= 1  # the constant run packs many more codes per block
+    c = codec.Compressed.from_host(lengths=enc.lengths, max_len=32, total_bits=enc.total_bits, n=enc.n,
+                                   stream=enc.stream, gaps=enc.gaps, offsets=None, sm=enc.sm, shape=(w.size,),
+                                   device="cpu", index8=ix, index8_wide=wide)
+    assert c.index_kind == "idx8" and c.index_bytes == ix.size < 8 * enc.offsets.size
+    path = os.path.join(tmp_path, "ix.df11")
+    container_file.save(path, [("t", c)])
+    (name, bc, _), = container_file.load(path, device="cpu")
+    assert bc.index_kind == "idx8" and bc.index8_wide == wide
+    assert (bc.index8.numpy() == ix).all() and (bc.stream.numpy() == enc.stream).all()
+    assert bc.container_bytes == c.container_bytes
+    head = container_file.read_header(path)
+    assert head["tensors"][0]["index"] == "idx8"
+
+
+def test_compact_index_of_wrong_size_is_refused(tmp_path):
+    w = synth.generate(synth.single_1024x4096()[0])[:200_000]
+    enc = oracle.encode(w, chunk_bytes=32, threads_per_block=32)
+    ix, wide = _index8_bytes(enc.offsets)
+    c = codec.Compressed.from_host(lengths=enc.lengths, max_len=32, total_bits=enc.total_bits, n=enc.n,
+                                   stream=enc.stream, gaps=enc.gaps, offsets=None, sm=enc.sm, device="cpu",
+                                   index8=np.concatenate([ix, np.zeros(4, np.uint8)]), index8_wide=wide)
+    path = os.path.join(tmp_path, "bad.df11")
+    container_file.save(path, [("t", c)])
+    with pytest.raises(container_file.FormatError):
+        container_file.load(path, device="cpu")

@@ -127,3 +127,27 @@ def test_safe_compress_decodes_and_compares(cuda_device):
     c = codec.compress(x, safe=True)
     out = codec.decompress(c)
     assert torch.equal(out.view(torch.int16).reshape(-1), x)
+
+
+def test_levels_with_compact_index(cuda_device, tmp_path):
+    """Containers that hold the compact block index verify at every level
+    (the offsets are expanded on the GPU first); a corrupt delta byte fails
+    the structure check or the sampled decode."""
+    w = np.concatenate([synth.generate(synth.single_1024x4096()[0])[:900_000], np.full(500_000, 0x3F80, np.uint16),
+                        synth.generate(synth.heavy_tail_64m()[0])[:700_001]])
+    x = dev_u16(w)
+    c = codec.compress(x, index="idx8")
+    assert c.index_kind == "idx8" and c.index8_wide >= 1
+    path = os.path.join(tmp_path, "ix.df11")
+    container_file.save(path, [("t", c)], {"t": api.df_sha256_device(x)})
+    entries = container_file.load(path)
+    src = {"t": x}
+    for level in ("structure", "sampled", "full"):
+        assert verify.verify(entries, level, src, samples=10**9)[0] == verify.PASS, level
+    nb = entries[0][1].sizes["n_blocks"]
+    S = (nb + 63) // 64
+    entries[0][1].index8[12 * S + 3] ^= 0x40  # block 3's count off by 64
+    code = verify.verify(entries, "structure")[0]
+    if code == verify.PASS:
+        code = verify.verify(entries, "sampled", src, samples=10**9)[0]
+    assert code == verify.FAIL

@@ -63,11 +63,18 @@ def test_struct_sizes_match_header_layout():
 
     assert ctypes.sizeof(_native.DfCode) == 16 + 256 + 1024
     assert ctypes.sizeof(_native.DfSizes) == 9 * 8
-    assert ctypes.sizeof(_native.DfTensor) == 16 + 16 + 5 * 8 + 256
+    assert ctypes.sizeof(_native.DfTensor) == 16 + 16 + 5 * 8 + 256 + 16
     assert ctypes.sizeof(_native.DfBatchPlan) == 8 + 8 * 4 + 8
     assert ctypes.sizeof(_native.DfNf12Sizes) == 5 * 8
     assert ctypes.sizeof(_native.DfNf12Tensor) == 16 + 4 * 8 + 8
     assert ctypes.sizeof(_native.DfNf12Plan) == 8 + 8 + 8
+
+
+@pytest.mark.parametrize("n_blocks,n_wide", [(0, 0), (1, 0), (3, 0), (64, 1), (65, 2), (10**6 + 1, 17)])
+def test_index8_bytes_match_the_oracle(n_blocks, n_wide):
+    from oracle import index8
+
+    assert api.df_index8_bytes(n_blocks, n_wide) == index8.index_bytes(n_blocks, n_wide)
 
 
 @pytest.mark.parametrize("n", [0, 1, 7, 8, 9, 16383, 16384, 16385, 10**7 + 3])
