@@ -239,6 +239,8 @@ struct Lane {
     uint32_t endst;  // codes must start before bit endst >> 18: st < endst
     uint32_t acc;
     uint32_t wp;
+    uint32_t kw;          // c0, c1, c2: stream words kw, kw + 1, kw + 2 of the chunk
+    uint32_t c0, c1, c2;  // (big-endian), so the window needs no shared load
     bool bad;
 };
 
@@ -263,7 +265,16 @@ __device__ __forceinline__ void append(Lane& L, uint32_t w, uint32_t sy) {
 // One lookup at the lane's bit position: up to 4 codes from the wide table
 // (at shared address tb), or one longer code from the 8-bit tables.
 __device__ __forceinline__ void step(Lane& L, uint32_t wb, uint32_t tb, const uint32_t* hier) {
-    const uint32_t win = window_at(wb, L.st >> kStepShift);
+    const uint32_t p = L.st >> kStepShift;
+    if ((p >> 5) != L.kw) {  // a lookup moves at most 32 bits: one word on
+        L.c0 = L.c1;
+        L.c1 = L.c2;
+        L.kw += 1;
+        // used two words from now; past the chunk's words this reads the
+        // warp's position words, whose bits no lookup uses
+        L.c2 = lds32(wb + (L.kw + 2) * (kLanes * 4));
+    }
+    const uint32_t win = __funnelshift_l(L.c1, L.c0, p);
     const uint2 e = lds64(tb + (win >> (32 - kWideBits)) * 8u);
     uint32_t sy = e.x, w = e.y;
     if (w == 0) {
@@ -295,6 +306,10 @@ __device__ __noinline__ uint32_t decode_chunk(uint32_t st, uint32_t endst, uint3
     L.endst = endst;
     L.acc = acc;
     L.wp = region + ((st & kStepCountMask) >> 3 & ~3u);
+    L.kw = st >> (kStepShift + 5);
+    L.c0 = lds32(wb + L.kw * (kLanes * 4));
+    L.c1 = lds32(wb + (L.kw + 1) * (kLanes * 4));
+    L.c2 = lds32(wb + (L.kw + 2) * (kLanes * 4));
     L.bad = false;
     uint32_t prev = st;  // the state before the last lookup
     for (;;) {  // two lookups per vote
