@@ -220,21 +220,26 @@ __device__ __forceinline__ uint32_t length_sum(const uint2* s_cl, const uint32_t
 }
 
 // The code lengths' sum and, when it is at most 64, the codes packed into
-// one register MSB-first (the first code in the highest bits of the sum).
+// one register MSB-first (the first code in the highest bits of the sum),
+// with a mask of the same layout that marks the last bit of every code: a
+// code that ends `d` bits after the lane's first bit has its mark at bit
+// sum - d.
 template <bool kFull>
 __device__ __forceinline__ uint32_t pack64(const uint2* s_cl, const uint32_t wv[kPerThread / 2], uint32_t cnt,
-                                           unsigned long long* v) {
+                                           unsigned long long* v, unsigned long long* ends) {
     uint32_t sum = 0;
-    unsigned long long x = 0;
+    unsigned long long x = 0, e = 0;
 #pragma unroll
     for (uint32_t k = 0; k < kPerThread; ++k) {
         if (kFull || k < cnt) {
             const uint2 cl = s_cl[(wv[k >> 1] >> (16 * (k & 1) + 7)) & 0xFFu];
             x = (x << cl.y) | cl.x;
+            e = (e << cl.y) | 1ull;
             sum += cl.y;
         }
     }
     *v = x;
+    *ends = e;
     return sum;
 }
 
@@ -334,8 +339,9 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(EncArgs a, EncTable
         const uint64_t i0 = t * kWarpTile + lane * kPerThread;
         uint32_t wv[kPerThread / 2];
         const uint32_t cnt = load16(a.in, a.n, i0, a.in_vec != 0, wv);
-        unsigned long long v;
-        const uint32_t sum = cnt == kPerThread ? pack64<true>(s_cl, wv, cnt, &v) : pack64<false>(s_cl, wv, cnt, &v);
+        unsigned long long v, ends;
+        const uint32_t sum =
+            cnt == kPerThread ? pack64<true>(s_cl, wv, cnt, &v, &ends) : pack64<false>(s_cl, wv, cnt, &v, &ends);
         uint32_t incl = sum;
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
@@ -407,7 +413,31 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(EncArgs a, EncTable
         // at a format-block boundary, the block offset
         uint32_t m = off < B0 ? 0u : div_by(off - B0, cbits, csh) + 1;
         uint32_t nb = B0 + m * cbits;  // the first boundary after this lane's start
-        if (nb <= off + sum) {
+        if (nb <= off + sum && sum <= 64) {
+            // a chunk (at least 128 bits) holds this lane's codes at most once:
+            // one boundary; the code that crosses or ends on it is the first
+            // whose end is at or past it, i.e. the highest end mark at or
+            // below bit sum - (nb - off) (the last code's mark, bit 0, always is)
+            const uint32_t jmax = sum - (nb - off);
+            const unsigned long long cand = jmax >= 63 ? ends : (ends & ((2ull << jmax) - 1ull));
+            const uint32_t jb = 63u - static_cast<uint32_t>(__clzll(cand));
+            const uint32_t end = off + sum - jb;
+            const uint32_t codes = static_cast<uint32_t>(__popcll(ends >> jb));  // up to and with that code
+            const uint64_t j = jt0 + m;
+            if (j < a.n_chunks) {
+                const uint64_t gq = 5 * j;
+                const uint32_t gw = static_cast<uint32_t>(gq >> 5) - gw0;
+                const uint32_t o = static_cast<uint32_t>(gq & 31);
+                const uint32_t g = end - nb;
+                if (o <= 27) {
+                    atomicOr(gapw + gw, g << (27 - o));
+                } else {
+                    atomicOr(gapw + gw, g >> (o - 27));
+                    atomicOr(gapw + gw + 1, g << (59 - o));
+                }
+                if (mod_by(jt0_mod_T + m, T, tsh) == 0) a.offsets[tsh < 32 ? j >> tsh : j / T] = i0 + codes;
+            }
+        } else if (nb <= off + sum) {  // longer codes: walk them
             uint32_t end = off;
 #pragma unroll
             for (uint32_t k = 0; k < kPerThread; ++k) {
