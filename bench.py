@@ -14,7 +14,11 @@ Also reported on the same line (N = 1 unless said otherwise):
   configs         decode GB/s, weights/s, roofline fraction and compressed % of
                   every weight set (single_1024x4096, llama_layer,
                   heavy_tail_64m, llama8b_shaped, mixed_2000); sets that fit in
-                  L2 get an L2 flush before every timed step
+                  L2 get an L2 flush before every timed step. Each set also
+                  carries "nf12": the same figures for the fixed 12-bit format
+                  on the same tensors, with its encoder's device time; the
+                  main set also carries "idx8": its containers with the
+                  compact block index in place of the uint64 offsets
   layer_by_layer  the 8B-shaped set decoded layer by layer into reused buffers
   jit_layer       per-step overhead of decoding each layer just in time, one or
                   two layers ahead of a GEMM consumer, against BF16-resident
@@ -473,6 +477,93 @@ def decode_record(comps, outs, args, stream, err, peak, flush):
             "l2": "flushed before every step" if use_flush else "inputs larger than L2: no flush"}
 
 
+def nf12_record(src, outs, args, stream, err, peak, flush):
+    """The fixed 12-bit format on the same tensors: compressed size, one
+    grouped decode launch per step (GB/s, weights/s, roofline fraction of its
+    algorithmic bytes), and the encoder's device time (both halves of every
+    tensor captured as one CUDA graph, replayed under CUDA events)."""
+    import torch
+
+    from lossless_bf16_weight_huffman_b200 import api, nf12
+
+    comps = [nf12.compress(x) for x in src]
+    dec = nf12.BatchDecoder(comps, outs)
+    n = sum(c.n for c in comps)
+    read = sum(c.read_bytes() for c in comps)
+    use_flush = flush is not None and read + 2 * n <= L2_FLUSH_BELOW
+    ms = time_launches(lambda: dec.run(err, stream), args.steps, args.warmup, stream, flush if use_flush else None)
+    assert api.df_read_error(err) == 0
+    verify(src, outs, [f"nf12 tensor {i}" for i in range(len(src))])
+    med = statistics.median(ms)
+    dev = src[0].device
+    sizes = [api.df_nf12_sizes_for(c.n) for c in comps]
+    ws = torch.empty(max(z.encode_ws_bytes for z in sizes), dtype=torch.uint8, device=dev)
+    esc = torch.empty(1, dtype=torch.int64, device=dev)
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side), torch.cuda.graph(g, stream=side):
+        for x, c in zip(src, comps):
+            api.df_nf12_encode_groups(x, c.top, c.slots, c.bitmap, ws, esc)
+            api.df_nf12_encode_escapes(x, c.top, c.slots, c.bitmap, ws, c.side, err)
+    torch.cuda.synchronize(dev)
+    g.replay()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    g.replay()
+    b.record()
+    torch.cuda.synchronize(dev)
+    enc_ms = a.elapsed_time(b)
+    assert api.df_read_error(err) == 0
+    del g
+    enc_bytes = sum(2 * c.n + 12 * c.groups + 4 * ((c.groups + 31) // 32) + 32 * c.n_escaped for c in comps)
+    return {"compressed_pct": round(100.0 * sum(c.container_bytes for c in comps) / (2 * n), 4),
+            "escaped_groups_pct": round(100.0 * sum(c.n_escaped for c in comps) / max(1, sum(c.groups for c in comps)), 4),
+            "gbs": round(2 * n / med / 1e6, 2), "weights_per_s": round(n / med * 1e3, 1), "ms": round(med, 4),
+            "roofline_frac": round((read + 2 * n) / med / 1e6 / peak, 4),
+            "encode_ms": round(enc_ms, 4),
+            "encode_roofline_frac": round(enc_bytes / enc_ms / 1e6 / peak, 4),
+            "l2": "flushed before every step" if use_flush else "inputs larger than L2: no flush"}
+
+
+def idx8_record(comps, outs, src, args, stream, err, peak, flush):
+    """The same containers with the compact block index in place of the
+    uint64 offsets: index bytes, the index build's device time (all builds
+    as one CUDA graph), and one grouped decode launch per step through it."""
+    import torch
+
+    from lossless_bf16_weight_huffman_b200 import api, codec
+
+    ix = [codec.Compressed(n=c.n, shape=c.shape, code=c.code, lut=c.lut, sizes=c.sizes, chunk_bytes=c.chunk_bytes,
+                           threads_per_block=c.threads_per_block, stream=c.stream, gaps=c.gaps, offsets=c.offsets,
+                           sm=c.sm).use_index8() for c in comps]
+    dev = comps[0].stream.device
+    wide = torch.zeros(1, dtype=torch.int64, device=dev)
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side), torch.cuda.graph(g, stream=side):
+        for c, d in zip(comps, ix):
+            api.df_index8_build(c.offsets, c.sizes["n_blocks"], d.index8, wide, err)
+    torch.cuda.synchronize(dev)
+    g.replay()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    g.replay()
+    b.record()
+    torch.cuda.synchronize(dev)
+    build_ms = a.elapsed_time(b)
+    del g
+    rec = decode_record(ix, outs, args, stream, err, peak, flush)
+    verify(src, outs, [f"tensor {i} through the compact index" for i in range(len(src))])
+    rec.update({"index_bytes": sum(c.index_bytes for c in ix),
+                "u64_offsets_bytes": sum(c.sizes["offsets_bytes"] for c in comps),
+                "wide_superblocks": sum(c.index8_wide for c in ix),
+                "superblocks": sum((c.sizes["n_blocks"] + 63) // 64 for c in ix),
+                "build_ms": round(build_ms, 4)})
+    return rec
+
+
 def layer_groups(specs, idx):
     """Indices (into idx) grouped by decoder layer; every other tensor alone."""
     groups = []
@@ -694,6 +785,9 @@ def run_gpu(args, world, rank, local, pool, ncores):
                                "l2": "flushed before every step" if flush is not None else
                                "inputs larger than L2: no flush"}}
         fl = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        cfg[args.workload]["nf12"] = nf12_record(src, outs, args, stream, err, peak, fl)
+        torch.cuda.empty_cache()
+        cfg[args.workload]["idx8"] = idx8_record(comps, outs, src, args, stream, err, peak, fl)
         for name in ("single_1024x4096", "llama_layer", "heavy_tail_64m", "mixed_2000"):
             if name == args.workload:
                 continue
@@ -703,6 +797,7 @@ def run_gpu(args, world, rank, local, pool, ncores):
             s_outs = [torch.empty(c.n, dtype=torch.int16, device=dev) for c in s_comps]
             cfg[name] = decode_record(s_comps, s_outs, args, stream, err, peak, fl)
             verify(s_src, s_outs, [s.name for s in sp])
+            cfg[name]["nf12"] = nf12_record(s_src, s_outs, args, stream, err, peak, fl)
             del s_src, s_comps, s_outs, stg
         extras["configs"] = cfg
         del fl

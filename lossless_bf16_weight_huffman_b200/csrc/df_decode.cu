@@ -6,7 +6,8 @@
 // The layout of the work below is this library's own, written for sm_100a.
 //
 // Every warp is an independent decoder: it owns a contiguous run of whole
-// format blocks (T chunks of C stream bytes, one block offset each) of one
+// format blocks (T chunks of C stream bytes, one block index entry each:
+// a uint64 offset, or the compact index's anchor, base and delta) of one
 // tensor and streams through it in rounds of 32 chunks, one chunk per lane.
 // Nothing a warp does waits for another warp, so a CUDA block only
 // synchronises when its tensor changes (to restage the decode tables). A CUDA
@@ -20,7 +21,9 @@
 //   2. one decode pass per lane from chunk start + gap until the bit position
 //      reaches the chunk end: a state word (bit position << 18) | (exponents
 //      so far << 3) advances by one add per lookup of the wide table (the
-//      exponents of up to 4 codes and their step word); the exponents go to
+//      exponents of up to 4 codes and their step word); the 32-bit window
+//      comes from three stream words held in registers (one slot load per 32
+//      bits consumed, off the lookup's critical path); the exponents go to
 //      the lane's own shared-memory region, one 32-bit store per lookup; codes
 //      longer than the window walk the 8-bit tables. The last lookup may take
 //      codes that start past the chunk end (they belong to the next chunk):

@@ -7,14 +7,20 @@
 // bits, C-byte chunks with 5-bit start gaps, per-block output offsets) is the
 // one df11.h defines.
 //
-// Tiles of 4096 weights, 256 threads x 16 consecutive weights, one CUDA block
-// each: a block scan of the threads' code-length sums gives every code its bit
-// offset within the tile; the tile's offset in the stream comes from a
-// decoupled look-back over the tiles before it; the tile's stream words and
-// gap fields are assembled in shared memory and stored whole, except the words
-// a tile shares with its neighbours, which are OR-ed atomically into the
-// zeroed buffers. The input is read twice in all: by the histogram and by this
-// pass.
+// One encode kernel after the histogram: persistent CUDA blocks of 8 warps,
+// each over a contiguous range of 512-weight warp tiles (16 consecutive
+// weights per lane), taken in launch order from a counter. Pass 1 writes the
+// sign|fraction bytes of the range and sums its code lengths; the range's
+// first stream bit comes from a decoupled look-back over the ranges before it
+// (warp 0, 128 predecessors per poll, bounded waits). Pass 2 packs warp tile
+// by warp tile: a warp scan of the lanes' bit counts places every lane's
+// codes (at most 64 bits in one register in the common case) in the tile's
+// stream words in shared memory; a lane's code-end mask gives the code that
+// crosses a chunk boundary, hence that chunk's gap and, at a format-block
+// boundary, the block offset. Whole words go out with plain stores, the
+// words a tile shares with its neighbours with atomic ORs into the zeroed
+// buffers. The input is read three times in all: by the histogram and by
+// both passes.
 #include <cuda_runtime.h>
 
 #include <cstring>
