@@ -577,12 +577,13 @@ def layer_groups(specs, idx):
     return groups
 
 
-def jit_record(args, specs, idx, comps, outs, err, dev):
+def jit_record(args, specs, idx, comps, outs, src, err, dev):
     """Per-pass time of a GEMM consumer over the decoder layers with weights
-    (a) resident as BF16, (b) decoded just in time at run-ahead depth 0, 1, 2."""
+    (a) resident as BF16, (b) decoded just in time at run-ahead depth 0, 1, 2,
+    (c) the same from the fixed 12-bit format."""
     import torch
 
-    from lossless_bf16_weight_huffman_b200 import jit
+    from lossless_bf16_weight_huffman_b200 import jit, nf12
 
     groups = [(k, g) for k, g in layer_groups(specs, idx) if k is not None][: args.jit_layers]
     if not groups:
@@ -631,6 +632,26 @@ def jit_record(args, specs, idx, comps, outs, err, dev):
     # the decode alone, layer by layer, for scale
     st = jit.LayerStreamer(layers, depth=0, device=dev)
     rec["decode_alone_ms_per_pass"] = round(timed(lambda: st.run(lambda l, v: None)), 3)
+    del st
+    # the same schedule from the fixed 12-bit format
+    n12 = [[nf12.compress(src[j]) for j in g] for _, g in groups]
+    for depth in (0, 1, 2):
+        st = jit.LayerStreamer(n12, depth=depth, device=dev)
+        t = timed(lambda: st.run(consume))
+        assert st.errors() == 0
+        rec[f"nf12_depth{depth}_ms_per_pass"] = round(t, 3)
+        rec[f"nf12_depth{depth}_overhead_pct"] = round(100.0 * (t - t_res) / t_res, 2)
+        del st
+    st = jit.LayerStreamer(n12, depth=0, device=dev)
+    rec["nf12_decode_alone_ms_per_pass"] = round(timed(lambda: st.run(lambda l, v: None)), 3)
+    def check(l, views):
+        for a, b in zip(views, resident[l]):
+            if not torch.equal(a, b.view(torch.int16).reshape(-1)):
+                raise SystemExit(f"nf12 just-in-time decode mismatch, layer {l}")
+
+    st.run(check)
+    torch.cuda.synchronize()
+    del st, n12
     # check the just-in-time weights against the resident ones on the last layer
     st1 = jit.LayerStreamer(layers, depth=1, device=dev)
     seen = {}
@@ -802,7 +823,7 @@ def run_gpu(args, world, rank, local, pool, ncores):
         extras["configs"] = cfg
         del fl
         if args.workload == "llama8b_shaped":
-            extras["jit_layer"] = jit_record(args, all_specs, idx, comps, outs, err, dev)
+            extras["jit_layer"] = jit_record(args, all_specs, idx, comps, outs, src, err, dev)
         torch.cuda.empty_cache()
 
     # ---- e2e through the public API (every N)

@@ -7,8 +7,8 @@ that schedule on CUDA streams: while the caller computes with layer l on its
 stream, layers l+1 .. l+depth are decoded on a side stream into a ring of
 depth+1 buffer sets; CUDA events order each decode after the computation
 that last read its buffer set, and each computation after its layer's decode.
-Every decode is one grouped launch (df_decode_batch_run) of the layer's
-tensors.
+Every decode is one grouped launch of the layer's tensors (df_decode_batch_run
+for the Huffman format, df_nf12_decode_batch_run for the fixed 12-bit one).
 
 HostLayerStreamer adds the copy of each layer's container from pinned host
 memory into device staging buffers on a copy stream, one layer ahead of the
@@ -20,7 +20,7 @@ from typing import Callable, Sequence
 
 import torch
 
-from . import api, codec
+from . import api, codec, nf12
 
 
 def _flat_views(buf: torch.Tensor, sizes: Sequence[int]) -> list[torch.Tensor]:
@@ -31,11 +31,29 @@ def _flat_views(buf: torch.Tensor, sizes: Sequence[int]) -> list[torch.Tensor]:
     return views
 
 
+def _device_of(c) -> torch.device:
+    return c.slots.device if isinstance(c, nf12.Nf12) else c.stream.device
+
+
+def _batch_decoder(comps, views, max_ctas: int):
+    """One prepared grouped launch over a layer's containers: the Huffman
+    format's (df_decode_batch_*) or the fixed 12-bit format's
+    (df_nf12_decode_batch_*)."""
+    if all(isinstance(c, nf12.Nf12) for c in comps):
+        return nf12.BatchDecoder(comps, views)
+    if any(isinstance(c, nf12.Nf12) for c in comps):
+        raise TypeError("a layer mixes the two formats")
+    dec = codec.BatchDecoder(comps, views)
+    dec.plan.max_ctas = max_ctas
+    return dec
+
+
 class LayerStreamer:
-    """Decode `layers` (each a list of device-resident containers) one layer
-    at a time into a ring of depth+1 buffer sets, `depth` layers ahead of the
-    consumer. depth=0 decodes each layer on the consumer's own stream right
-    before it is used (no overlap)."""
+    """Decode `layers` (each a list of device-resident containers, of either
+    format) one layer at a time into a ring of depth+1 buffer sets, `depth`
+    layers ahead of the consumer. depth=0 decodes each layer on the
+    consumer's own stream right before it is used (no overlap). max_ctas caps
+    the CUDA blocks of a Huffman-format decode (0: all that fit)."""
 
     def __init__(self, layers: Sequence[Sequence[codec.Compressed]], depth: int = 1, max_ctas: int = 0,
                  device=None):
@@ -45,7 +63,7 @@ class LayerStreamer:
             raise ValueError("no layers")
         self.layers = [list(l) for l in layers]
         self.depth = depth
-        dev = torch.device(device) if device is not None else self.layers[0][0].stream.device
+        dev = torch.device(device) if device is not None else _device_of(self.layers[0][0])
         self.device = dev
         self.nslots = depth + 1
         cap = max(sum(c.n for c in l) for l in self.layers)
@@ -60,9 +78,7 @@ class LayerStreamer:
             per_slot, per_views = [], []
             for s in range(self.nslots):
                 views = _flat_views(self.bufs[s], [c.n for c in l])
-                dec = codec.BatchDecoder(l, views)
-                dec.plan.max_ctas = max_ctas
-                per_slot.append(dec)
+                per_slot.append(_batch_decoder(l, views, max_ctas))
                 per_views.append(views)
             self.decoders.append(per_slot)
             self.views.append(per_views)

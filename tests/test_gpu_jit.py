@@ -76,3 +76,20 @@ def test_grouped_launch_with_few_blocks(layers, max_ctas):
     assert api.df_read_error(err) == 0
     for o, x in zip(outs, [x for l in src for x in l]):
         assert torch.equal(o, x)
+
+
+@pytest.mark.parametrize("depth", [0, 2])
+def test_layer_streamer_fixed_12_bit_format(layers, depth):
+    """The same schedule over layers held in the fixed 12-bit format."""
+    from lossless_bf16_weight_huffman_b200 import nf12
+
+    src, _ = layers
+    n12 = [[nf12.compress(x) for x in l] for l in src]
+    st = jit.LayerStreamer(n12, depth=depth)
+    seen = {}
+    st.run(lambda l, views: seen.__setitem__(l, [v.clone() for v in views]))
+    torch.cuda.synchronize()
+    assert st.errors() == 0
+    for l in range(len(src)):
+        for v, x in zip(seen[l], src[l]):
+            assert torch.equal(v, x)
