@@ -220,18 +220,20 @@ def source_digest(paths):
     return h.hexdigest()[:16]
 
 
-def decode_traffic_record():
-    """ncu DRAM bytes of one decode launch, if captured for the current kernel
-    source (profiles/decode_traffic.json), with the workload it was taken on."""
+def decode_traffic_record(workload: str):
+    """ncu DRAM bytes of one decode launch captured on `workload` with the
+    current kernel source (profiles/decode_traffic.json), or None."""
     path = os.path.join(ROOT, "profiles", "decode_traffic.json")
     src = os.path.join(ROOT, "lossless_bf16_weight_huffman_b200", "csrc", "df_decode.cu")
     try:
-        rec = json.load(open(path))
+        caps = json.load(open(path))["captures"]
     except Exception:
         return None
-    if rec.get("kernel_source_sha") != source_digest([src]):
-        return None
-    return rec
+    digest = source_digest([src])
+    for rec in caps:
+        if rec.get("workload") == workload and rec.get("kernel_source_sha") == digest:
+            return rec
+    return None
 
 
 # ---------------------------------------------------------------------------------------------
@@ -766,10 +768,8 @@ def run_gpu(args, world, rank, local, pool, ncores):
     algo_bytes = read_bytes + 2 * n_mine
     launch_ms = statistics.mean(step_ms)
     achieved = algo_bytes / (launch_ms / 1e3) / 1e9
-    rec = decode_traffic_record()
-    traffic = None
-    if rec and rec.get("workload") == args.workload and world == 1:
-        traffic = int(rec["dram_bytes_read"] + rec["dram_bytes_write"])
+    rec = decode_traffic_record(args.workload) if world == 1 else None
+    traffic = int(rec["dram_bytes_read"] + rec["dram_bytes_write"]) if rec else None
     w_max = max_over_ranks(n_mine, world, dev)
     w_min = -max_over_ranks(-n_mine, world, dev)
 
