@@ -558,24 +558,57 @@ __global__ void __launch_bounds__(kMaxWarps * kLanes, 1)
                 }
                 __syncwarp();
 
+                // 4b. complete the group this lane's range ends inside: the
+                // round's last group has all its exponents here already; any
+                // other takes the next lane's first 16 exponents into the slack
+                // after this lane's own, so that 5a finds all 16 in one region.
+                // Both regions must hold at least 20 exponents (this lane's
+                // writes start past the bytes the lane before reads, and the
+                // next lane's writes past the bytes read here) and this region
+                // must have 20 bytes to spare; the rest stay for 5b.
+                const uint32_t bend = pos + ext;
+                const uint32_t ext_next = __shfl_down_sync(kFull, ext, 1);
+                if (ext && (bend & 15) && (bend & ~15u) >= pos) {  // this lane owns that group
+                    const uint32_t gi = bend >> 4;
+                    if (bend == vend) {
+                        s_owner[gi] = static_cast<uint8_t>(lane);
+                    } else if (lane + 1 < kLanes && ext >= 20 && ext_next >= 20 && ext + 20 <= RB) {
+                        const uint32_t sa = shared_addr(s_priv + region_off(lane + 1, RB));
+                        const uint32_t w0 = lds32(sa), w1 = lds32(sa + 4), w2 = lds32(sa + 8), w3 = lds32(sa + 12);
+                        const uint32_t da = shared_addr(s_priv + my_off) + (ext & ~3u);
+                        const uint32_t r8 = 8 * (ext & 3);
+                        const uint32_t keep = r8 ? lds32(da) & ((1u << r8) - 1u) : 0u;
+                        sts32(da, keep | (w0 << r8));
+                        sts32(da + 4, __funnelshift_l(w0, w1, r8));
+                        sts32(da + 8, __funnelshift_l(w1, w2, r8));
+                        sts32(da + 12, __funnelshift_l(w2, w3, r8));
+                        if (r8) sts32(da + 16, w3 >> (32 - r8));
+                        s_owner[gi] = static_cast<uint8_t>(lane);
+                    }
+                }
+                __syncwarp();
+
                 // 5. merge and store; stage position p <-> output gbase + p,
                 // group gi <-> the 16 sign|fraction bytes at smg + 16gi
                 const uint64_t gbase = outr - align;
                 const uint64_t rend = outr + total;  // this round's outputs end here
                 const uint32_t ngroups = (vend + 15) >> 4;
                 const uint32_t gv0 = gbase < vstart ? 1u : 0u;      // group 0 may start before the run
+                const uint32_t glast = (vend & 15) ? ngroups - 1 : ngroups;  // a last group the round ends inside
                 const uint8_t* __restrict__ smg = sm + gbase;
                 uint16_t* __restrict__ outg = out + gbase;
                 // 5a. groups inside their owner's range (bit 7 of the owner byte
                 // clear); the others are merged in 5b. Two groups per lane and
-                // iteration: both sign|fraction loads are in flight first.
+                // iteration: both sign|fraction loads are in flight first. A
+                // run's first group and a round's unfinished last group are
+                // merged below.
                 if (vec) {
                     for (uint32_t g0 = lane; g0 < ngroups; g0 += 2 * kLanes) {
                         const uint32_t g1 = g0 + kLanes;
                         const uint32_t o0 = s_owner[g0];
                         const uint32_t o1 = g1 < ngroups ? s_owner[g1] : 0x80u;
-                        const bool v0 = !(o0 & 0x80u) && g0 >= gv0;  // a run's first group is merged below
-                        const bool v1 = !(o1 & 0x80u);
+                        const bool v0 = !(o0 & 0x80u) && g0 >= gv0 && g0 != glast;
+                        const bool v1 = !(o1 & 0x80u) && g1 != glast;
                         uint4 s0 = make_uint4(0, 0, 0, 0), s1 = make_uint4(0, 0, 0, 0);
                         if (v0) s0 = __ldg(reinterpret_cast<const uint4*>(smg) + g0);
                         if (v1) s1 = __ldg(reinterpret_cast<const uint4*>(smg) + g1);
@@ -590,24 +623,35 @@ __global__ void __launch_bounds__(kMaxWarps * kLanes, 1)
                         }
                     }
                 }
-                // a run's first group (it starts before the run's outputs), and
-                // every group of buffers without 16-byte alignment: element stores
-                for (uint32_t gi = vec ? (gv0 && lane == 0 ? 0u : ngroups) : lane; gi < ngroups; gi += kLanes) {
+                // edge groups, element stores: a run's first group (it starts
+                // before the run's outputs), the round's unfinished last group
+                // (carried into the next round unless the run ends here), and
+                // every group of buffers without 16-byte alignment
+                auto edge = [&](uint32_t gi) {
                     const uint32_t o = s_owner[gi];
-                    if (o & 0x80u) continue;
+                    if (o & 0x80u) return;  // 5b takes it
                     uint32_t e[4];
                     gather16(s_priv, s_base[o & 31u] + static_cast<int>(16 * gi), e);
-                    for (uint32_t q = 0; q < 16; ++q) {
-                        const uint64_t i = gbase + 16 * gi + q;
-                        if (i >= vstart) out[i] = merge1(sm[i], static_cast<uint8_t>(e[q >> 2] >> (8 * (q & 3))));
+                    if (gi == glast && !run_last) {
+                        *reinterpret_cast<uint4*>(s_carry) = make_uint4(e[0], e[1], e[2], e[3]);
+                        return;
                     }
-                    if (vec) break;
+                    const uint64_t G = gbase + 16 * gi;
+                    const uint64_t lo_i = max(G, vstart), hi_i = min(G + 16, rend);
+                    for (uint64_t i = lo_i; i < hi_i; ++i)
+                        out[i] = merge1(sm[i], static_cast<uint8_t>(e[(i - G) >> 2] >> (8 * ((i - G) & 3))));
+                };
+                if (!vec) {
+                    for (uint32_t gi = lane; gi < ngroups; gi += kLanes) edge(gi);
+                } else {
+                    if (lane == 0 && gv0) edge(0);
+                    if (lane == 1 && glast < ngroups && !(gv0 && glast == 0)) edge(glast);
                 }
-                // 5b. the group this lane's range ends inside, when it owns that
-                // group: it runs past the range into later regions, or it is the
-                // round's last group (kept open for the next round of the run)
-                const uint32_t bend = pos + ext;
-                if (ext && (bend & 15) && (s_owner[bend >> 4] & 31u) == lane) {
+                // 5b. a group that spans regions and was not completed in 4b:
+                // the lane whose range it starts in gathers it from the regions
+                // (rare: short or full regions, three or more regions)
+                const bool span = ext && (bend & 15) && s_owner[bend >> 4] == (lane | 0x80u);
+                if (__any_sync(kFull, span) && span) {
                     const uint32_t c0 = bend & ~15u;
                     const uint64_t G = gbase + c0;
                     const uint32_t hi = min(c0 + 16, vend);
