@@ -102,6 +102,10 @@ def dist_setup():
         import torch.distributed as dist
 
         backend = "nccl" if _cuda_ok() else "gloo"
+        if backend == "nccl":
+            import torch
+
+            torch.cuda.set_device(local)  # NCCL binds each rank's communicator to its own GPU
         dist.init_process_group(backend, timeout=datetime.timedelta(seconds=600))
     return world, rank, local
 
