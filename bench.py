@@ -486,13 +486,14 @@ def decode_record(comps, outs, args, stream, err, peak, flush):
 def nf12_record(src, outs, args, stream, err, peak, flush):
     """The fixed 12-bit format on the same tensors: compressed size, one
     grouped decode launch per step (GB/s, weights/s, roofline fraction of its
-    algorithmic bytes), and the encoder's device time (both halves of every
-    tensor captured as one CUDA graph, replayed under CUDA events)."""
+    algorithmic bytes), and the grouped encoder's device time (its launches
+    captured as one CUDA graph, replayed under CUDA events)."""
     import torch
 
     from lossless_bf16_weight_huffman_b200 import api, nf12
 
-    comps = [nf12.compress(x) for x in src]
+    encoder = nf12.BatchEncoder(src)
+    comps = encoder.run(err)
     dec = nf12.BatchDecoder(comps, outs)
     n = sum(c.n for c in comps)
     read = sum(c.read_bytes() for c in comps)
@@ -502,16 +503,12 @@ def nf12_record(src, outs, args, stream, err, peak, flush):
     verify(src, outs, [f"nf12 tensor {i}" for i in range(len(src))])
     med = statistics.median(ms)
     dev = src[0].device
-    sizes = [api.df_nf12_sizes_for(c.n) for c in comps]
-    ws = torch.empty(max(z.encode_ws_bytes for z in sizes), dtype=torch.uint8, device=dev)
-    esc = torch.empty(1, dtype=torch.int64, device=dev)
     side = torch.cuda.Stream(dev)
     side.wait_stream(torch.cuda.current_stream(dev))
     g = torch.cuda.CUDAGraph()
     with torch.cuda.stream(side), torch.cuda.graph(g, stream=side):
-        for x, c in zip(src, comps):
-            api.df_nf12_encode_groups(x, c.top, c.slots, c.bitmap, ws, esc)
-            api.df_nf12_encode_escapes(x, c.top, c.slots, c.bitmap, ws, c.side, err)
+        api.df_nf12_encode_batch_groups(encoder.plan, encoder.escaped)
+        api.df_nf12_encode_batch_escapes(encoder.plan, err)
     torch.cuda.synchronize(dev)
     g.replay()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)

@@ -126,6 +126,46 @@ df_status df_nf12_decode_batch_prepare(const df_nf12_tensor* h_tensors, uint32_t
  * agihunt.info nf12 item, "Confirmed". */
 df_status df_nf12_decode_batch_run(const df_nf12_plan* plan, uint32_t* d_err, void* stream);
 
+/* One tensor of a grouped encode (host array; copied by the prepare call). */
+typedef struct df_nf12_encode_tensor {
+    const uint16_t* in;       /* device, n weights (BF16 bits), 2-byte aligned   */
+    uint64_t n;
+    void* slots;              /* device, 12 G bytes, 4-byte aligned             */
+    void* bitmap;             /* device, 4 ceil(G / 32) bytes, 4-byte aligned    */
+    void* side;               /* device, 16 side_capacity bytes, 16-byte aligned;
+                                 NULL before the escape counts are known        */
+    uint64_t side_capacity;   /* side entries (groups) the buffer holds         */
+    uint32_t top;             /* shared top exponent bits, 0..15                */
+    uint32_t reserved;        /* 0                                              */
+    uint64_t reserved2;       /* 0                                              */
+} df_nf12_encode_tensor;
+
+/* Bytes of device workspace a grouped encode of these tensors needs
+ * (descriptors, tile starts, per-tile escape counts and per-tensor totals).
+ * Source: no counterpart in the pages (a launch detail). */
+size_t df_nf12_encode_batch_workspace(const df_nf12_encode_tensor* h_tensors, uint32_t count);
+
+/* Grouped encode, set-up: copies the descriptors into d_ws (enqueued on
+ * `stream`; h_tensors is read before the call returns) and fills *plan. Call
+ * it again with the side buffers filled in before the escapes (the escape
+ * counts in d_ws are kept). Source: agihunt.info nf12 item, "Confirmed".
+ * Errors: DF_ERR_INVALID_ARG, DF_ERR_WORKSPACE, DF_ERR_UNSUPPORTED,
+ * DF_ERR_CUDA. */
+df_status df_nf12_encode_batch_prepare(const df_nf12_encode_tensor* h_tensors, uint32_t count, void* d_ws,
+                                       size_t ws_bytes, df_nf12_plan* plan, void* stream);
+
+/* Grouped encode, first half: the slots and bitmap of every tensor (one
+ * launch over all their tiles) and each tensor's escape count, written to
+ * d_escaped[0 .. count) (device uint64). Source: as df_nf12_encode_groups.
+ * Errors: DF_ERR_INVALID_ARG, DF_ERR_CUDA. */
+df_status df_nf12_encode_batch_groups(const df_nf12_plan* plan, uint64_t* d_escaped, void* stream);
+
+/* Grouped encode, second half: every tensor's side buffer and side indices,
+ * as df_nf12_encode_escapes does for one (a tensor whose escapes exceed its
+ * side_capacity sets DF_EFLAG_NF12_SIDE in d_err). Source: as
+ * df_nf12_encode_escapes. Errors: DF_ERR_INVALID_ARG, DF_ERR_CUDA. */
+df_status df_nf12_encode_batch_escapes(const df_nf12_plan* plan, uint32_t* d_err, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -44,6 +44,8 @@ EXPORTS = (
     "df_index8_expand",
     "df_nf12_sizes_for", "df_nf12_encode_groups", "df_nf12_encode_escapes", "df_nf12_decode",
     "df_nf12_decode_batch_workspace", "df_nf12_decode_batch_prepare", "df_nf12_decode_batch_run",
+    "df_nf12_encode_batch_workspace", "df_nf12_encode_batch_prepare", "df_nf12_encode_batch_groups",
+    "df_nf12_encode_batch_escapes",
 )
 
 
@@ -129,6 +131,20 @@ class DfNf12Tensor(ctypes.Structure):
         ("out", ctypes.c_void_p),
         ("top", ctypes.c_uint32),
         ("reserved", ctypes.c_uint32),
+    ]
+
+
+class DfNf12EncodeTensor(ctypes.Structure):
+    _fields_ = [
+        ("input", ctypes.c_void_p),
+        ("n", ctypes.c_uint64),
+        ("slots", ctypes.c_void_p),
+        ("bitmap", ctypes.c_void_p),
+        ("side", ctypes.c_void_p),
+        ("side_capacity", ctypes.c_uint64),
+        ("top", ctypes.c_uint32),
+        ("reserved", ctypes.c_uint32),
+        ("reserved2", ctypes.c_uint64),
     ]
 
 
@@ -224,6 +240,15 @@ def lib() -> ctypes.CDLL:
     L.df_nf12_decode_batch_prepare.restype = i32
     L.df_nf12_decode_batch_run.argtypes = [ctypes.POINTER(DfNf12Plan), vp, vp]
     L.df_nf12_decode_batch_run.restype = i32
+    L.df_nf12_encode_batch_workspace.argtypes = [ctypes.POINTER(DfNf12EncodeTensor), u32]
+    L.df_nf12_encode_batch_workspace.restype = sz
+    L.df_nf12_encode_batch_prepare.argtypes = [ctypes.POINTER(DfNf12EncodeTensor), u32, vp, sz,
+                                               ctypes.POINTER(DfNf12Plan), vp]
+    L.df_nf12_encode_batch_prepare.restype = i32
+    L.df_nf12_encode_batch_groups.argtypes = [ctypes.POINTER(DfNf12Plan), vp, vp]
+    L.df_nf12_encode_batch_groups.restype = i32
+    L.df_nf12_encode_batch_escapes.argtypes = [ctypes.POINTER(DfNf12Plan), vp, vp]
+    L.df_nf12_encode_batch_escapes.restype = i32
     _lib = L
     return L
 

@@ -9,8 +9,8 @@ import ctypes
 import numpy as np
 import torch
 
-from ._native import (DfBatchPlan, DfCode, DfNf12Plan, DfNf12Sizes, DfNf12Tensor, DfSizes, DfTensor, check,
-                      lib)
+from ._native import (DfBatchPlan, DfCode, DfNf12EncodeTensor, DfNf12Plan, DfNf12Sizes, DfNf12Tensor, DfSizes,
+                      DfTensor, check, lib)
 
 
 def _stream_ptr(stream=None):
@@ -352,3 +352,33 @@ def df_nf12_decode_batch_run(plan: DfNf12Plan, d_err: torch.Tensor | None = None
     _need_err(d_err)
     check("df_nf12_decode_batch_run", lib().df_nf12_decode_batch_run(ctypes.byref(plan), _dev(d_err, "d_err"),
                                                                      _stream_ptr(stream)))
+
+
+def _nf12_encode_array(tensors):
+    return (DfNf12EncodeTensor * max(1, len(tensors)))(*tensors)
+
+
+def df_nf12_encode_batch_workspace(tensors) -> int:
+    return int(lib().df_nf12_encode_batch_workspace(_nf12_encode_array(tensors), len(tensors)))
+
+
+def df_nf12_encode_batch_prepare(tensors, d_ws: torch.Tensor, stream=None) -> DfNf12Plan:
+    """tensors: DfNf12EncodeTensor list (device pointers as ints)."""
+    _need(d_ws, df_nf12_encode_batch_workspace(tensors), "d_ws")
+    plan = DfNf12Plan()
+    check("df_nf12_encode_batch_prepare", lib().df_nf12_encode_batch_prepare(
+        _nf12_encode_array(tensors), len(tensors), _dev(d_ws, "d_ws"), d_ws.numel() * d_ws.element_size(),
+        ctypes.byref(plan), _stream_ptr(stream)))
+    return plan
+
+
+def df_nf12_encode_batch_groups(plan: DfNf12Plan, d_escaped: torch.Tensor, stream=None) -> None:
+    _need(d_escaped, 8 * plan.count, "d_escaped")
+    check("df_nf12_encode_batch_groups", lib().df_nf12_encode_batch_groups(
+        ctypes.byref(plan), _dev(d_escaped, "d_escaped"), _stream_ptr(stream)))
+
+
+def df_nf12_encode_batch_escapes(plan: DfNf12Plan, d_err: torch.Tensor | None = None, stream=None) -> None:
+    _need_err(d_err)
+    check("df_nf12_encode_batch_escapes", lib().df_nf12_encode_batch_escapes(
+        ctypes.byref(plan), _dev(d_err, "d_err"), _stream_ptr(stream)))

@@ -178,7 +178,7 @@ __global__ void __launch_bounds__(kNfThreads)
 template <bool kVec>
 __device__ __forceinline__ void pack_tile(const uint16_t* __restrict__ in, uint64_t n, uint32_t top,
                                           uint32_t* __restrict__ slots, uint32_t* __restrict__ bitmap,
-                                          uint64_t* __restrict__ counts, uint64_t tile) {
+                                          uint64_t* __restrict__ count_out, uint64_t tile) {
     __shared__ uint32_t warp_count[kNfWarps];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const uint64_t G = (n + 7) >> 3;
@@ -228,7 +228,7 @@ __device__ __forceinline__ void pack_tile(const uint16_t* __restrict__ in, uint6
         uint32_t t = 0;
 #pragma unroll
         for (int w = 0; w < kNfWarps; ++w) t += warp_count[w];
-        counts[tile] = t;
+        *count_out = t;
     }
 }
 
@@ -236,9 +236,9 @@ __global__ void __launch_bounds__(kNfThreads)
     pack_kernel(const uint16_t* __restrict__ in, uint64_t n, uint32_t top, uint32_t* __restrict__ slots,
                 uint32_t* __restrict__ bitmap, uint64_t* __restrict__ counts, int vec) {
     if (vec)
-        pack_tile<true>(in, n, top, slots, bitmap, counts, blockIdx.x);
+        pack_tile<true>(in, n, top, slots, bitmap, counts + blockIdx.x, blockIdx.x);
     else
-        pack_tile<false>(in, n, top, slots, bitmap, counts, blockIdx.x);
+        pack_tile<false>(in, n, top, slots, bitmap, counts + blockIdx.x, blockIdx.x);
 }
 
 // Exclusive prefix of counts[0 .. tiles) in place; counts[tiles] and
@@ -273,16 +273,14 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(uint64_t* counts, ui
 }
 
 // One block of 64 threads per tile; thread i owns the tile's bitmap word i
-// (32 groups) and writes the side entries of its escaped groups in order.
+// (32 groups) and writes the side entries of its escaped groups in order,
+// from side index `base` (the escapes of the tensor's tiles before this one).
 template <bool kVec>
 __device__ __forceinline__ void escape_tile(const uint16_t* __restrict__ in, uint64_t n, uint32_t top,
                                             uint32_t* __restrict__ slots, const uint32_t* __restrict__ bitmap,
-                                            const uint64_t* __restrict__ prefix, uint4* __restrict__ side,
-                                            uint64_t cap, uint32_t* err) {
+                                            uint64_t tile, uint64_t base, uint4* __restrict__ side, uint64_t cap,
+                                            uint32_t* err) {
     __shared__ uint32_t warp_total[kWordsPerTile / 32];
-    const uint64_t tile = blockIdx.x;
-    const uint64_t base = prefix[tile];
-    if (prefix[tile + 1] == base) return;  // block-uniform
     const uint64_t G = (n + 7) >> 3;
     const uint64_t wi = tile * kWordsPerTile + threadIdx.x;
     uint32_t word = wi < ((G + 31) >> 5) ? bitmap[wi] : 0;
@@ -318,10 +316,101 @@ __global__ void __launch_bounds__(kWordsPerTile)
     escape_kernel(const uint16_t* __restrict__ in, uint64_t n, uint32_t top, uint32_t* __restrict__ slots,
                   const uint32_t* __restrict__ bitmap, const uint64_t* __restrict__ prefix, uint4* __restrict__ side,
                   uint64_t cap, uint32_t* err, int vec) {
+    const uint64_t tile = blockIdx.x, base = prefix[tile];
+    if (prefix[tile + 1] == base) return;  // no escapes in this tile
     if (vec)
-        escape_tile<true>(in, n, top, slots, bitmap, prefix, side, cap, err);
+        escape_tile<true>(in, n, top, slots, bitmap, tile, base, side, cap, err);
     else
-        escape_tile<false>(in, n, top, slots, bitmap, prefix, side, cap, err);
+        escape_tile<false>(in, n, top, slots, bitmap, tile, base, side, cap, err);
+}
+
+// ---------------------------------------------------------------- grouped encode
+
+struct Nf12EncDev {
+    const uint16_t* in;
+    uint32_t* slots;
+    uint32_t* bitmap;
+    uint4* side;
+    uint64_t n;
+    uint64_t cap;
+    uint32_t top;
+    uint32_t in_vec;  // in is 16-byte aligned
+    uint64_t pad;
+};
+static_assert(sizeof(Nf12EncDev) == 64, "descriptors are copied in 64-byte units");
+
+// The tensor of global tile `tile` (starts[t] <= tile < starts[t + 1]).
+__device__ __forceinline__ uint32_t tensor_of(const uint64_t* __restrict__ starts, uint32_t count, uint64_t tile) {
+    uint32_t lo = 0, hi = count;
+    while (hi - lo > 1) {
+        const uint32_t mid = (lo + hi) >> 1;
+        if (__ldg(starts + mid) <= tile)
+            lo = mid;
+        else
+            hi = mid;
+    }
+    return lo;
+}
+
+__global__ void __launch_bounds__(kNfThreads)
+    pack_batch_kernel(const Nf12EncDev* __restrict__ descs, const uint64_t* __restrict__ starts, uint32_t count,
+                      uint64_t* __restrict__ counts) {
+    const uint64_t tile = blockIdx.x;
+    const uint32_t ti = tensor_of(starts, count, tile);
+    const Nf12EncDev d = descs[ti];
+    const uint64_t t = tile - __ldg(starts + ti);
+    if (d.in_vec)
+        pack_tile<true>(d.in, d.n, d.top, d.slots, d.bitmap, counts + tile, t);
+    else
+        pack_tile<false>(d.in, d.n, d.top, d.slots, d.bitmap, counts + tile, t);
+}
+
+// Per tensor (one CUDA block each): the exclusive prefix of its tiles' escape
+// counts in place, and its total.
+constexpr int kBatchScanThreads = 256;
+__global__ void __launch_bounds__(kBatchScanThreads)
+    scan_batch_kernel(const uint64_t* __restrict__ starts, uint64_t* __restrict__ counts, uint64_t* __restrict__ totals) {
+    __shared__ uint64_t warp_sum[kBatchScanThreads / 32];
+    const uint32_t ti = blockIdx.x;
+    const uint64_t t0 = starts[ti], tiles = starts[ti + 1] - t0;
+    uint64_t* c = counts + t0;
+    const uint64_t per = (tiles + kBatchScanThreads - 1) / kBatchScanThreads;
+    const uint64_t b = threadIdx.x * per, e = b + per < tiles ? b + per : tiles;
+    uint64_t s = 0;
+    for (uint64_t i = b; i < e; ++i) s += c[i];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint64_t incl = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint64_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) warp_sum[warp] = incl;
+    __syncthreads();
+    uint64_t run = incl - s;
+    for (int w = 0; w < warp; ++w) run += warp_sum[w];
+    for (uint64_t i = b; i < e; ++i) {
+        const uint64_t x = c[i];
+        c[i] = run;
+        run += x;
+    }
+    if (threadIdx.x == kBatchScanThreads - 1) totals[ti] = run;
+}
+
+__global__ void __launch_bounds__(kWordsPerTile)
+    escape_batch_kernel(const Nf12EncDev* __restrict__ descs, const uint64_t* __restrict__ starts, uint32_t count,
+                        const uint64_t* __restrict__ prefix, const uint64_t* __restrict__ totals, uint32_t* err) {
+    const uint64_t tile = blockIdx.x;
+    const uint32_t ti = tensor_of(starts, count, tile);
+    const uint64_t base = prefix[tile];
+    const uint64_t next = tile + 1 < __ldg(starts + ti + 1) ? prefix[tile + 1] : totals[ti];
+    if (next == base) return;  // no escapes in this tile
+    const Nf12EncDev d = descs[ti];
+    const uint64_t t = tile - __ldg(starts + ti);
+    if (d.in_vec)
+        escape_tile<true>(d.in, d.n, d.top, d.slots, d.bitmap, t, base, d.side, d.cap, err);
+    else
+        escape_tile<false>(d.in, d.n, d.top, d.slots, d.bitmap, t, base, d.side, d.cap, err);
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -468,6 +557,126 @@ df_status df_nf12_decode_batch_run(const df_nf12_plan* plan, uint32_t* d_err, vo
     decode_batch_kernel<<<static_cast<unsigned>(plan->total_tiles), kNfThreads, 0,
                           static_cast<cudaStream_t>(stream)>>>(descs, starts, plan->count, d_err);
     return launched();
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- grouped encode, host side
+
+namespace {
+
+struct EncLayout {
+    size_t descs, starts, counts, totals, bytes;
+};
+
+EncLayout enc_layout(uint32_t count, uint64_t total_tiles) {
+    EncLayout l;
+    l.descs = 0;
+    l.starts = static_cast<size_t>(count) * sizeof(df::Nf12EncDev);
+    l.counts = l.starts + 8 * (static_cast<size_t>(count) + 1);
+    l.totals = l.counts + 8 * static_cast<size_t>(total_tiles);
+    l.bytes = l.totals + 8 * static_cast<size_t>(count);
+    return l;
+}
+
+uint64_t enc_tiles(const df_nf12_encode_tensor* h, uint32_t count) {
+    uint64_t t = 0;
+    for (uint32_t i = 0; i < count; ++i) t += df::tiles_of(h[i].n);
+    return t;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t df_nf12_encode_batch_workspace(const df_nf12_encode_tensor* h_tensors, uint32_t count) {
+    if (count && !h_tensors) return 0;
+    return enc_layout(count, enc_tiles(h_tensors, count)).bytes;
+}
+
+df_status df_nf12_encode_batch_prepare(const df_nf12_encode_tensor* h_tensors, uint32_t count, void* d_ws,
+                                       size_t ws_bytes, df_nf12_plan* plan, void* stream) {
+    if (!plan || (count && (!h_tensors || !d_ws)) || !df::aligned(d_ws, 16)) return DF_ERR_INVALID_ARG;
+    std::vector<df::Nf12EncDev> dev(count);
+    std::vector<uint64_t> start(static_cast<size_t>(count) + 1, 0);
+    for (uint32_t i = 0; i < count; ++i) {
+        const df_nf12_encode_tensor& t = h_tensors[i];
+        if (t.top > 15 || t.reserved || t.reserved2) return DF_ERR_INVALID_ARG;
+        if (t.n > DF_MAX_WEIGHTS) return DF_ERR_UNSUPPORTED;
+        if (t.n && (!t.in || !t.slots || !t.bitmap)) return DF_ERR_INVALID_ARG;
+        if (t.side_capacity && !t.side) return DF_ERR_INVALID_ARG;
+        if (!df::aligned(t.in, 2) || !df::aligned(t.slots, 4) || !df::aligned(t.bitmap, 4) ||
+            !df::aligned(t.side, 16))
+            return DF_ERR_INVALID_ARG;
+        if ((t.n + 7) / 8 > df::kMaxGroups) return DF_ERR_UNSUPPORTED;
+        df::Nf12EncDev& d = dev[i];
+        d.in = t.in;
+        d.slots = static_cast<uint32_t*>(t.slots);
+        d.bitmap = static_cast<uint32_t*>(t.bitmap);
+        d.side = static_cast<uint4*>(t.side);
+        d.n = t.n;
+        d.cap = t.side_capacity;
+        d.top = t.top;
+        d.in_vec = df::aligned(t.in, 16) ? 1u : 0u;
+        d.pad = 0;
+        start[i + 1] = start[i] + df::tiles_of(t.n);
+    }
+    const uint64_t total = start[count];
+    if (total > 0x7FFFFFFFull) return DF_ERR_UNSUPPORTED;
+    const EncLayout l = enc_layout(count, total);
+    if (ws_bytes < l.bytes) return DF_ERR_WORKSPACE;
+    plan->d_ws = d_ws;
+    plan->count = count;
+    plan->reserved = 0;
+    plan->total_tiles = total;
+    if (!count) return DF_OK;
+    // copies from pageable host memory return once the source has been
+    // staged, so the host vectors may die on return
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(d_ws);
+    cudaError_t e = cudaMemcpyAsync(ws + l.descs, dev.data(), dev.size() * sizeof(df::Nf12EncDev),
+                                    cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(ws + l.starts, start.data(), start.size() * 8, cudaMemcpyHostToDevice, s);
+    return e == cudaSuccess ? DF_OK : cuda_fail(e);
+}
+
+df_status df_nf12_encode_batch_groups(const df_nf12_plan* plan, uint64_t* d_escaped, void* stream) {
+    if (!plan || !d_escaped || (plan->count && !plan->d_ws) || !df::aligned(d_escaped, 8)) return DF_ERR_INVALID_ARG;
+    if (!plan->count) return DF_OK;
+    if (plan->total_tiles > 0x7FFFFFFFull) return DF_ERR_UNSUPPORTED;
+    const EncLayout l = enc_layout(plan->count, plan->total_tiles);
+    uint8_t* ws = static_cast<uint8_t*>(plan->d_ws);
+    const df::Nf12EncDev* descs = reinterpret_cast<const df::Nf12EncDev*>(ws + l.descs);
+    const uint64_t* starts = reinterpret_cast<const uint64_t*>(ws + l.starts);
+    uint64_t* counts = reinterpret_cast<uint64_t*>(ws + l.counts);
+    uint64_t* totals = reinterpret_cast<uint64_t*>(ws + l.totals);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    df_status st;
+    if (plan->total_tiles) {
+        df::pack_batch_kernel<<<static_cast<unsigned>(plan->total_tiles), df::kNfThreads, 0, s>>>(descs, starts,
+                                                                                                 plan->count, counts);
+        if ((st = df::launched()) != DF_OK) return st;
+    }
+    df::scan_batch_kernel<<<plan->count, df::kBatchScanThreads, 0, s>>>(starts, counts, totals);
+    if ((st = df::launched()) != DF_OK) return st;
+    const cudaError_t e = cudaMemcpyAsync(d_escaped, totals, 8 * static_cast<size_t>(plan->count),
+                                          cudaMemcpyDeviceToDevice, s);
+    return e == cudaSuccess ? DF_OK : cuda_fail(e);
+}
+
+df_status df_nf12_encode_batch_escapes(const df_nf12_plan* plan, uint32_t* d_err, void* stream) {
+    if (!plan || (plan->count && !plan->d_ws)) return DF_ERR_INVALID_ARG;
+    if (!plan->count || !plan->total_tiles) return DF_OK;
+    if (plan->total_tiles > 0x7FFFFFFFull) return DF_ERR_UNSUPPORTED;
+    const EncLayout l = enc_layout(plan->count, plan->total_tiles);
+    const uint8_t* ws = static_cast<const uint8_t*>(plan->d_ws);
+    df::escape_batch_kernel<<<static_cast<unsigned>(plan->total_tiles), df::kWordsPerTile, 0,
+                              static_cast<cudaStream_t>(stream)>>>(
+        reinterpret_cast<const df::Nf12EncDev*>(ws + l.descs), reinterpret_cast<const uint64_t*>(ws + l.starts),
+        plan->count, reinterpret_cast<const uint64_t*>(ws + l.counts), reinterpret_cast<const uint64_t*>(ws + l.totals),
+        d_err);
+    return df::launched();
 }
 
 }  // extern "C"

@@ -11,7 +11,7 @@ import numpy as np
 import torch
 
 from . import api
-from ._native import DF_NF12_TOP, DfNf12Tensor
+from ._native import DF_NF12_TOP, DfNf12EncodeTensor, DfNf12Tensor
 from .codec import _as_u16
 
 
@@ -73,6 +73,63 @@ def compress(w: torch.Tensor, top: int = DF_NF12_TOP, d_err: torch.Tensor | None
     if e:
         api.df_nf12_encode_escapes(x, top, slots, bitmap, ws, side, d_err, stream)
     return Nf12(n=n, shape=tuple(w.shape), top=top, slots=slots, bitmap=bitmap, side=side, n_escaped=e)
+
+
+class BatchEncoder:
+    """A grouped encode of many tensors (one launch per step for all of them):
+    run() packs every tensor and counts its escapes, reads the counts (one
+    wait), sizes the side buffers and writes them."""
+
+    def __init__(self, ws: list[torch.Tensor], top: int = DF_NF12_TOP):
+        if not ws:
+            raise ValueError("no tensors")
+        self.xs = [_as_u16(w) for w in ws]
+        self.shapes = [tuple(w.shape) for w in ws]
+        self.top = top
+        dev = self.xs[0].device
+        self.parts = []
+        for x in self.xs:
+            z = api.df_nf12_sizes_for(x.numel())
+            self.parts.append((torch.empty(max(z.slots_bytes, 16), dtype=torch.uint8, device=dev),
+                               torch.empty(max(z.bitmap_bytes, 16), dtype=torch.uint8, device=dev)))
+        self.escaped = torch.empty(len(self.xs), dtype=torch.int64, device=dev)
+        self.sides = [None] * len(self.xs)
+        self.ws = torch.empty(max(api.df_nf12_encode_batch_workspace(self.descriptors()), 16), dtype=torch.uint8,
+                              device=dev)
+        self.plan = api.df_nf12_encode_batch_prepare(self.descriptors(), self.ws)
+
+    def descriptors(self) -> list[DfNf12EncodeTensor]:
+        out = []
+        for i, (x, (slots, bitmap)) in enumerate(zip(self.xs, self.parts)):
+            t = DfNf12EncodeTensor()
+            t.input = x.data_ptr() if x.numel() else None
+            t.n = x.numel()
+            t.slots = slots.data_ptr()
+            t.bitmap = bitmap.data_ptr()
+            side = self.sides[i]
+            t.side = side.data_ptr() if side is not None else None
+            t.side_capacity = side.numel() // 16 if side is not None else 0
+            t.top = self.top
+            out.append(t)
+        return out
+
+    def run(self, d_err: torch.Tensor | None = None, stream=None) -> list[Nf12]:
+        api.df_nf12_encode_batch_groups(self.plan, self.escaped, stream)
+        counts = [int(v) for v in self.escaped.cpu().numpy().view(np.uint64)]  # waits for the stream
+        dev = self.xs[0].device
+        for i, e in enumerate(counts):
+            if self.sides[i] is None or self.sides[i].numel() < 16 * e:
+                self.sides[i] = torch.empty(max(16 * e, 16), dtype=torch.uint8, device=dev)
+        self.plan = api.df_nf12_encode_batch_prepare(self.descriptors(), self.ws, stream)
+        api.df_nf12_encode_batch_escapes(self.plan, d_err, stream)
+        return [Nf12(n=x.numel(), shape=shp, top=self.top, slots=sl, bitmap=bm, side=sd, n_escaped=e)
+                for x, shp, (sl, bm), sd, e in zip(self.xs, self.shapes, self.parts, self.sides, counts)]
+
+
+def compress_batch(ws: list[torch.Tensor], top: int = DF_NF12_TOP, d_err: torch.Tensor | None = None,
+                   stream=None) -> list[Nf12]:
+    """compress() of many tensors with one launch per kernel for all."""
+    return BatchEncoder(ws, top).run(d_err, stream)
 
 
 def decompress(c: Nf12, out: torch.Tensor | None = None, d_err: torch.Tensor | None = None,

@@ -5,7 +5,8 @@
   tails, for 16-byte-aligned and 2-byte-aligned inputs, and another top;
 * decode of the ORACLE's parts (independent of the GPU encoder) gives the
   source back, for aligned and unaligned outputs;
-* the grouped decode over many tensors, empty and tiny ones included;
+* the grouped decode over many tensors, empty and tiny ones included, and the
+  grouped encode (one launch per kernel for all tensors) against the oracle;
 * a side index past the escaped groups and a side buffer too small are
   reported in the error word, and nothing is written outside the outputs;
 * at full size (the 8B-shaped set's largest tensor) the round trip is exact
@@ -202,3 +203,36 @@ def test_full_size_round_trip_and_sampled_groups():
             assert np.array_equal(c.side[16 * idx: 16 * idx + 16].cpu().numpy().view(np.uint16), grp)
         else:
             assert np.array_equal(slots[k], s)
+
+
+def test_grouped_encode_matches_oracle():
+    """nf12.compress_batch (one launch per kernel over every tensor) writes the
+    oracle's bytes for each tensor: empty, tiny, ragged, tile-spanning, all
+    escaped, 2-byte-aligned input; run twice (the side buffers are reused)."""
+    rng = np.random.default_rng(12)
+    base = _weights(3_000_000, heavy=True)
+    ws = [base[:0], base[:1], base[5:12], np.full(40_001, 0x4000, np.uint16)]
+    ws += [base[int(a): int(a) + int(k)] for a, k in zip(rng.integers(0, 2_000_000, 40), rng.integers(1, 70_000, 40))]
+    xs = [dev_u16(w) for w in ws]
+    xs.append(dev_u16(base[:100_001])[1:])  # 2-byte aligned only
+    ws.append(base[1:100_001])
+    enc = nf12.BatchEncoder(xs)
+    for _ in range(2):
+        err = err_word()
+        comps = enc.run(err)
+        assert api.df_read_error(err) == 0
+        for c, w in zip(comps, ws):
+            _check_encode(c, w)
+            if w.size:
+                assert np.array_equal(host_u16(nf12.decompress(c, torch.empty(w.size, dtype=torch.int16, device="cuda"))), w)
+
+
+def test_grouped_encode_short_side_buffer_is_reported():
+    w = _weights(200_000, heavy=True)
+    enc = nf12.BatchEncoder([dev_u16(w)])
+    enc.run()
+    enc.sides[0] = enc.sides[0][: 16 * (enc.sides[0].numel() // 16 // 2)]  # half the room
+    enc.plan = api.df_nf12_encode_batch_prepare(enc.descriptors(), enc.ws)
+    err = err_word()
+    api.df_nf12_encode_batch_escapes(enc.plan, err)
+    assert api.df_read_error(err) & DF_EFLAG_NF12_SIDE
