@@ -26,7 +26,10 @@ Also reported on the same line (N = 1 unless said otherwise):
   encode          device time of the GPU encoder, per call summed
   e2e             through the public API from pinned host memory: containers
                   copied in and BF16 copied out every step, overlapped with the
-                  decode layer by layer (every N)
+                  decode layer by layer (every N); into_hbm: the same with the
+                  BF16 left in HBM for an on-GPU consumer
+  verify          device SHA-256 (leaf tree) and compare throughput on the
+                  decoded set
   roofline        the decode kernel against the measured HBM copy bandwidth
   cpu_baseline    the oracle on the host cores, on a bounded sample
   clocks          SM clocks sampled during the timed region
@@ -567,6 +570,35 @@ def idx8_record(comps, outs, src, args, stream, err, peak, flush):
     return rec
 
 
+def verify_record(outs, dev):
+    """Device throughput of the verify steps on the decoded set: the per-tensor
+    SHA-256 leaf tree (df_sha256_device, leaf digests to the host) and the
+    first-difference compare (df_compare) of every output with itself."""
+    import torch
+
+    from lossless_bf16_weight_huffman_b200 import api
+
+    nbytes = sum(2 * o.numel() for o in outs)
+    ws = torch.empty(max(api.df_sha256_workspace(2 * o.numel()) for o in outs), dtype=torch.uint8, device=dev)
+    first = torch.empty(1, dtype=torch.int64, device=dev)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for o in outs:
+        api.df_sha256_device(o, ws)  # waits for its leaf digests
+    t_sha = time.perf_counter() - t0
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for o in outs:
+        api.df_compare(o, o, first)
+    b.record()
+    torch.cuda.synchronize()
+    t_cmp = a.elapsed_time(b) / 1e3
+    return {"sha256_gbs": round(nbytes / t_sha / 1e9, 2), "sha256_s": round(t_sha, 3),
+            "compare_gbs": round(2 * nbytes / t_cmp / 1e9, 1), "bytes": nbytes,
+            "note": "sha256: wall time per tensor including the host's root hash over the leaf digests; "
+                    "compare: device time, both operands read"}
+
+
 def layer_groups(specs, idx):
     """Indices (into idx) grouped by decoder layer; every other tensor alone."""
     groups = []
@@ -690,6 +722,18 @@ def e2e_record(args, specs, idx, comps, src, dev, world):
     hls.run(consume)
     torch.cuda.synchronize()
     assert hls.errors() == 0
+    # the same stream into HBM only (the consumer keeps the BF16 on the GPU;
+    # the step's result read back is the decode status word)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    hls.run(lambda i, views: None)
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(args.e2e_steps):
+        hls.run(lambda i, views: None)
+        assert hls.errors() == 0  # reads the status word back each step
+    b.record()
+    torch.cuda.synchronize()
+    ms_in = max_over_ranks(a.elapsed_time(b) / args.e2e_steps, world, dev)
     last = groups[-1][1]
     off = 0
     for j in last:
@@ -713,7 +757,11 @@ def e2e_record(args, specs, idx, comps, src, dev, world):
             "d2h_bytes_per_step": int(2 * n_all), "ms_per_step": round(ms, 2), "wall_s": round(wall, 3),
             "how": "jit.HostLayerStreamer: per layer, pinned host container -> HBM on a copy stream, "
                    "df_decode_batch_run on a decode stream, BF16 -> pinned host on the consumer stream; "
-                   "consecutive layers overlap"}
+                   "consecutive layers overlap",
+            "into_hbm": {"value": round(2 * n_all / (ms_in / 1e3) / 1e9, 3), "unit": "GB/s of BF16 decoded",
+                         "ms_per_step": round(ms_in, 2), "d2h_bytes_per_step": 4 * world,
+                         "how": "the same, the BF16 left in HBM for an on-GPU consumer; the decode status "
+                                "word read back every step"}}
 
 
 def run_gpu(args, world, rank, local, pool, ncores):
@@ -825,6 +873,7 @@ def run_gpu(args, world, rank, local, pool, ncores):
         del fl
         if args.workload == "llama8b_shaped":
             extras["jit_layer"] = jit_record(args, all_specs, idx, comps, outs, src, err, dev)
+        extras["verify"] = verify_record(outs, dev)
         torch.cuda.empty_cache()
 
     # ---- e2e through the public API (every N)

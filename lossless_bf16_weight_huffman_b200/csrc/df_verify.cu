@@ -62,10 +62,20 @@ constexpr uint64_t kLeafBytes = 64 * 1024;
 __host__ __device__ __forceinline__ uint32_t rotr(uint32_t x, uint32_t n) { return (x >> n) | (x << (32 - n)); }
 
 // One 512-bit block (16 big-endian words) into the state (FIPS 180-4, 6.2.2).
+// Loop unrolling for the device pass (the host compiler does not know the pragma).
+#ifdef __CUDA_ARCH__
+#define DF_UNROLL _Pragma("unroll")
+#else
+#define DF_UNROLL
+#endif
+
 __host__ __device__ inline void sha256_block(uint32_t h[8], const uint32_t w_in[16]) {
     uint32_t w[16];
+    DF_UNROLL
     for (int i = 0; i < 16; ++i) w[i] = w_in[i];
     uint32_t a = h[0], b = h[1], c = h[2], d = h[3], e = h[4], f = h[5], g = h[6], k = h[7];
+    // unrolled on the device: the schedule's indices are constants, so w stays in registers
+    DF_UNROLL
     for (int t = 0; t < 64; ++t) {
         uint32_t wt;
         if (t < 16) {
@@ -143,7 +153,44 @@ __global__ void __launch_bounds__(128) sha256_leaves_kernel(const uint8_t* __res
     if (i >= leaves) return;
     const uint64_t off = i * kLeafBytes;
     const uint64_t len = nbytes - off < kLeafBytes ? nbytes - off : kLeafBytes;
-    sha256(data + off, len, digests + 32 * i);
+    const uint8_t* p = data + off;
+    if (len != kLeafBytes || (reinterpret_cast<uintptr_t>(p) & 15)) {
+        sha256(p, len, digests + 32 * i);  // the last, shorter leaf or unaligned data: byte loads
+        return;
+    }
+    // a whole aligned leaf: 16-byte loads, then the padding block of FIPS 180-4, 5.1.1
+    uint32_t h[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) h[j] = sha_h0(j);
+    const uint4* q = reinterpret_cast<const uint4*>(p);
+    for (uint64_t blk = 0; blk < kLeafBytes / 64; ++blk) {
+        uint32_t w[16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint4 v = __ldg(q + 4 * blk + j);
+            w[4 * j] = __byte_perm(v.x, 0, 0x0123);
+            w[4 * j + 1] = __byte_perm(v.y, 0, 0x0123);
+            w[4 * j + 2] = __byte_perm(v.z, 0, 0x0123);
+            w[4 * j + 3] = __byte_perm(v.w, 0, 0x0123);
+        }
+        sha256_block(h, w);
+    }
+    uint32_t w[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) w[j] = 0;
+    w[0] = 0x80000000u;
+    const uint64_t bits = static_cast<uint64_t>(kLeafBytes) * 8;
+    w[14] = static_cast<uint32_t>(bits >> 32);
+    w[15] = static_cast<uint32_t>(bits);
+    sha256_block(h, w);
+    uint8_t* out = digests + 32 * i;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        out[4 * j] = static_cast<uint8_t>(h[j] >> 24);
+        out[4 * j + 1] = static_cast<uint8_t>(h[j] >> 16);
+        out[4 * j + 2] = static_cast<uint8_t>(h[j] >> 8);
+        out[4 * j + 3] = static_cast<uint8_t>(h[j]);
+    }
 }
 
 // Structure of one container, no decode: block offsets start at 0, never

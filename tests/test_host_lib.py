@@ -369,3 +369,16 @@ def test_binding_refuses_short_buffers_before_the_library():
         api.df_decode(d, torch.empty(99, dtype=torch.int16))
     with pytest.raises(ValueError, match="d_outs"):
         api.df_decode_batch_prepare([d], [torch.empty(50, dtype=torch.int16)], torch.empty(4096, dtype=torch.uint8))
+
+
+def test_host_sha256_against_hashlib():
+    """df_sha256 (host) is plain SHA-256 (FIPS 180-4): the standard's "abc"
+    example, the empty message, the padding edge lengths, random data."""
+    import hashlib
+
+    assert api.df_sha256(b"abc").hex() == "ba7816bf8f01cfea414140de5dae2223b00361a396177a9cb410ff61f20015ad"
+    assert api.df_sha256(b"") == hashlib.sha256(b"").digest()
+    rng = np.random.default_rng(8)
+    for n in (1, 55, 56, 57, 63, 64, 65, 119, 120, 128, 1000, 65536, 65537):
+        data = rng.integers(0, 256, n, dtype=np.uint8).tobytes()
+        assert api.df_sha256(data) == hashlib.sha256(data).digest(), n
