@@ -213,8 +213,33 @@ __global__ void __launch_bounds__(256) structure_kernel(const uint64_t* __restri
 __global__ void __launch_bounds__(256) compare_kernel(const uint16_t* __restrict__ a, const uint16_t* __restrict__ b,
                                                       uint64_t n, unsigned long long* __restrict__ first) {
     const uint64_t stride = static_cast<uint64_t>(gridDim.x) * blockDim.x;
+    const uint64_t t0 = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     unsigned long long mine = ~0ull;
-    for (uint64_t i = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride)
+    uint64_t done = 0;
+    if (!((reinterpret_cast<uintptr_t>(a) | reinterpret_cast<uintptr_t>(b)) & 15)) {
+        // both 16-byte aligned: 8 weights per load, two loads of each in flight
+        const uint4* a4 = reinterpret_cast<const uint4*>(a);
+        const uint4* b4 = reinterpret_cast<const uint4*>(b);
+        const uint64_t n8 = n / 8;
+        for (uint64_t i = t0; i < n8; i += 2 * stride) {
+            const bool two = i + stride < n8;
+            const uint4 x0 = __ldg(a4 + i), y0 = __ldg(b4 + i);
+            uint4 x1 = x0, y1 = y0;
+            if (two) {
+                x1 = __ldg(a4 + i + stride);
+                y1 = __ldg(b4 + i + stride);
+            }
+            const uint32_t d0[4] = {x0.x ^ y0.x, x0.y ^ y0.y, x0.z ^ y0.z, x0.w ^ y0.w};
+            const uint32_t d1[4] = {x1.x ^ y1.x, x1.y ^ y1.y, x1.z ^ y1.z, x1.w ^ y1.w};
+            for (int k = 0; k < 8 && mine == ~0ull; ++k)
+                if ((d0[k >> 1] >> (16 * (k & 1))) & 0xFFFFu) mine = 8 * i + k;
+            for (int k = 0; k < 8 && two && mine == ~0ull; ++k)
+                if ((d1[k >> 1] >> (16 * (k & 1))) & 0xFFFFu) mine = 8 * (i + stride) + k;
+            if (mine != ~0ull) break;  // later indices of this thread are larger
+        }
+        done = 8 * n8;
+    }
+    for (uint64_t i = done + t0; i < n; i += stride)
         if (a[i] != b[i] && i < mine) mine = i;
     for (int d = 16; d > 0; d >>= 1) {
         const unsigned long long o = __shfl_xor_sync(0xFFFFFFFFu, mine, d);

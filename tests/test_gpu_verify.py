@@ -28,6 +28,31 @@ def test_device_digest_matches_leaf_tree(cuda_device, n):
     assert api.df_sha256_device(d) == leaf_tree(a.tobytes())
 
 
+def test_device_digest_of_unaligned_data(cuda_device):
+    """Whole 64 KiB leaves at an odd address take the byte-load path."""
+    rng = np.random.default_rng(3)
+    a = rng.integers(0, 256, 3 * 65536 + 1001, dtype=np.uint8)
+    d = torch.from_numpy(a).cuda()
+    assert api.df_sha256_device(d[1:]) == leaf_tree(a[1:].tobytes())
+
+
+@pytest.mark.parametrize("n", [1, 7, 8, 9, 4095, 1_000_003])
+def test_compare_first_difference_sizes_and_alignments(cuda_device, n):
+    rng = np.random.default_rng(n)
+    base = torch.from_numpy(rng.integers(-32768, 32767, n + 1, dtype=np.int16)).cuda()
+    for a_src in (base[:n], base[1:]):  # 16-byte aligned and 2-byte aligned
+        a = a_src.contiguous() if a_src.data_ptr() % 16 == 0 else a_src
+        b = a.clone()
+        out = torch.empty(1, dtype=torch.int64, device="cuda")
+        api.df_compare(a, b, out)
+        assert int(out.cpu().numpy().view(np.uint64)[0]) == 2**64 - 1
+        pos = sorted(set(int(p) for p in rng.integers(0, n, 5)))
+        for p in reversed(pos):
+            b[p] ^= 1
+            api.df_compare(a, b, out)
+            assert int(out.item()) == p
+
+
 def test_compare_finds_the_first_difference(cuda_device):
     a = torch.arange(100_000, dtype=torch.int16, device="cuda")
     b = a.clone()
