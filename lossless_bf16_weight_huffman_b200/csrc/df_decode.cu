@@ -32,13 +32,15 @@
 //      previous round left open, so every round starts on a group boundary
 //   3. warp scan of the region sizes: every lane's first stage position
 //   4. an owner map: for every group of 16 outputs, the lane whose region
-//      holds its first exponent
-//   5. merge, in two loops: groups that lie in one region take their 16
-//      exponents from it; then each lane takes the one group, if any, that
-//      its range ends inside, gathering from its region and the next one(s).
-//      Per group: one 16-byte load of sign|fraction bytes, two 16-byte stores.
-//      The round's last group, if the round ends inside it, stays open for the
-//      next round; only a run's first and last groups take element stores.
+//      holds its first exponent; then each lane completes the group its range
+//      ends inside by copying the next lane's first 16 exponents into its
+//      region's slack, so nearly every group lies in one region
+//   5. merge: every group takes its 16 exponents from its owner's region;
+//      one 16-byte load of sign|fraction bytes, two 16-byte stores. Groups
+//      that could not be completed (short or full regions) gather from
+//      several regions in a separate, rarely taken path. The round's last
+//      group, if the round ends inside it, stays open for the next round;
+//      only a run's first and last groups take element stores.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -535,7 +537,7 @@ __global__ void __launch_bounds__(kMaxWarps * kLanes, 1)
 
                 // 4. owner map: group gi (stage positions [16gi, 16gi+16))
                 // belongs to the lane whose range holds 16gi; bit 7 marks a
-                // group that runs past that range (merged in 5b)
+                // group that runs past that range (completed in 4b, else merged in 5b)
                 if (ext) {
                     const uint32_t hi = pos + ext;
                     for (uint32_t gi = (pos + 15) >> 4; 16 * gi < hi; ++gi)
