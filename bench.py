@@ -87,7 +87,8 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-extras", action="store_true",
                    help="headline only: skip the per-set records, layer-by-layer and jit_layer")
-    p.add_argument("--jit-tokens", type=int, default=4096, help="activation rows of the jit_layer GEMM consumer")
+    p.add_argument("--jit-tokens", default="4096,16384",
+                   help="activation rows of the jit_layer GEMM consumer (comma-separated sizes)")
     p.add_argument("--jit-layers", type=int, default=32, help="decoder layers in the jit_layer measurement")
     p.add_argument("--chunk-bytes", type=int, default=0,
                    help="format chunk size C in bytes (0: 32, or 16 where the shortest code is 1 bit)")
@@ -297,7 +298,17 @@ def _oracle_job(job):
     t2 = time.perf_counter()
     if not (out == w).all():
         raise RuntimeError(f"oracle round trip failed on {set_name}[{index}]")
-    return int(w.size), t1 - t0, t2 - t1
+    # the fixed 12-bit format's oracle on the same tensor
+    from oracle import nf12_oracle
+
+    t3 = time.perf_counter()
+    slots, bitmap, side = nf12_oracle.encode(w)
+    t4 = time.perf_counter()
+    back = nf12_oracle.decode(slots, bitmap, side, w.size)
+    t5 = time.perf_counter()
+    if not (back == w).all():
+        raise RuntimeError(f"nf12 oracle round trip failed on {set_name}[{index}]")
+    return int(w.size), t1 - t0, t2 - t1, t4 - t3, t5 - t4
 
 
 def _cpu_model() -> str:
@@ -313,7 +324,8 @@ def _cpu_model() -> str:
 def cpu_baseline(pool, ncores):
     """The oracle encoder and decoder on bounded samples of every weight set,
     one process (one host thread) per tensor across all host cores; a
-    worker's own times give the one-thread rates. The 8B-shaped set is
+    worker's own times give the one-thread rates. The fixed 12-bit format's
+    oracle (numpy) runs on the same tensors in the same workers. The 8B-shaped set is
     extrapolated from a decoder layer (same shapes and distributions) by
     weight count."""
     from lossless_bf16_weight_huffman_b200 import synth
@@ -338,7 +350,9 @@ def cpu_baseline(pool, ncores):
         dec_s = sum(m[2] for m in multi)
         rec.update({"one_thread_encode_gbs": round(2 * n / enc_s / 1e9, 4),
                     "one_thread_decode_gbs": round(2 * n / dec_s / 1e9, 4),
-                    "one_thread_weights_per_s": round(n / dec_s, 1)})
+                    "one_thread_weights_per_s": round(n / dec_s, 1),
+                    "nf12_one_thread_encode_gbs": round(2 * n / max(sum(m[3] for m in multi), 1e-9) / 1e9, 4),
+                    "nf12_one_thread_decode_gbs": round(2 * n / max(sum(m[4] for m in multi), 1e-9) / 1e9, 4)})
         if name == "mixed_2000":
             rec["sample"] = "every 8th tensor (250 of 2000)"
         per[name] = rec
@@ -615,7 +629,9 @@ def layer_groups(specs, idx):
 def jit_record(args, specs, idx, comps, outs, src, err, dev):
     """Per-pass time of a GEMM consumer over the decoder layers with weights
     (a) resident as BF16, (b) decoded just in time at run-ahead depth 0, 1, 2,
-    (c) the same from the fixed 12-bit format."""
+    (c) the same from the fixed 12-bit format; for every consumer size in
+    --jit-tokens (the overhead is the decode time over the GEMM time, so it
+    shrinks as the consumer grows)."""
     import torch
 
     from lossless_bf16_weight_huffman_b200 import jit, nf12
@@ -623,23 +639,12 @@ def jit_record(args, specs, idx, comps, outs, src, err, dev):
     groups = [(k, g) for k, g in layer_groups(specs, idx) if k is not None][: args.jit_layers]
     if not groups:
         return None
-    B = args.jit_tokens
     layer_specs = [[specs[idx[j]] for j in g] for _, g in groups]
     ins = sorted({s.shape[1] for l in layer_specs for s in l if len(s.shape) == 2})
     outs_f = sorted({s.shape[0] for l in layer_specs for s in l if len(s.shape) == 2})
-    gen = torch.Generator(device=dev).manual_seed(0xDF11)
-    x_in = {k: torch.randn(B, k, generator=gen, device=dev, dtype=torch.float32).to(torch.bfloat16) for k in ins}
-    y_out = {k: torch.empty(B, k, device=dev, dtype=torch.bfloat16) for k in outs_f}
-    flops = sum(2 * B * s.numel for l in layer_specs for s in l if len(s.shape) == 2)
-
-    def consume(l, views):
-        for s, v in zip(layer_specs[l], views):
-            if len(s.shape) != 2:
-                continue
-            w = v.view(torch.bfloat16).view(s.shape[0], s.shape[1])
-            torch.matmul(x_in[s.shape[1]], w.t(), out=y_out[s.shape[0]])
-
     resident = [[outs[j] for j in g] for _, g in groups]
+    layers = [[comps[j] for j in g] for _, g in groups]
+    n12 = [[nf12.compress(src[j]) for j in g] for _, g in groups]
 
     def timed(fn, reps=3):
         fn()
@@ -652,49 +657,56 @@ def jit_record(args, specs, idx, comps, outs, src, err, dev):
         torch.cuda.synchronize()
         return a.elapsed_time(b) / reps
 
-    t_res = timed(lambda: [consume(l, resident[l]) for l in range(len(groups))])
-    layers = [[comps[j] for j in g] for _, g in groups]
-    rec = {"consumer": f"per layer, y = x W^T for each linear weight (cuBLAS bf16), x: {B} rows",
-           "layers": len(groups), "tokens": B, "gemm_tflops_resident": round(flops / t_res / 1e9, 1),
-           "resident_ms_per_pass": round(t_res, 3)}
-    for depth in (0, 1, 2):
-        st = jit.LayerStreamer(layers, depth=depth, device=dev)
-        t = timed(lambda: st.run(consume))
-        assert st.errors() == 0
-        rec[f"depth{depth}_ms_per_pass"] = round(t, 3)
-        rec[f"depth{depth}_overhead_pct"] = round(100.0 * (t - t_res) / t_res, 2)
-        del st
+    def one_size(B):
+        gen = torch.Generator(device=dev).manual_seed(0xDF11)
+        x_in = {k: torch.randn(B, k, generator=gen, device=dev, dtype=torch.float32).to(torch.bfloat16) for k in ins}
+        y_out = {k: torch.empty(B, k, device=dev, dtype=torch.bfloat16) for k in outs_f}
+        flops = sum(2 * B * s.numel for l in layer_specs for s in l if len(s.shape) == 2)
+
+        def consume(l, views):
+            for s, v in zip(layer_specs[l], views):
+                if len(s.shape) != 2:
+                    continue
+                w = v.view(torch.bfloat16).view(s.shape[0], s.shape[1])
+                torch.matmul(x_in[s.shape[1]], w.t(), out=y_out[s.shape[0]])
+
+        t_res = timed(lambda: [consume(l, resident[l]) for l in range(len(groups))])
+        rec = {"consumer": f"per layer, y = x W^T for each linear weight (cuBLAS bf16), x: {B} rows",
+               "layers": len(groups), "tokens": B, "gemm_tflops_resident": round(flops / t_res / 1e9, 1),
+               "resident_ms_per_pass": round(t_res, 3)}
+        for fmt, ls in (("", layers), ("nf12_", n12)):
+            for depth in (0, 1, 2):
+                st = jit.LayerStreamer(ls, depth=depth, device=dev)
+                t = timed(lambda: st.run(consume))
+                assert st.errors() == 0
+                rec[f"{fmt}depth{depth}_ms_per_pass"] = round(t, 3)
+                rec[f"{fmt}depth{depth}_overhead_pct"] = round(100.0 * (t - t_res) / t_res, 2)
+                del st
+        return rec
+
+    sizes = [int(b) for b in str(args.jit_tokens).split(",") if b]
+    recs = [one_size(B) for B in sizes]
+    rec = dict(recs[0])
+    if len(recs) > 1:
+        rec["more_tokens"] = recs[1:]
     # the decode alone, layer by layer, for scale
-    st = jit.LayerStreamer(layers, depth=0, device=dev)
-    rec["decode_alone_ms_per_pass"] = round(timed(lambda: st.run(lambda l, v: None)), 3)
-    del st
-    # the same schedule from the fixed 12-bit format
-    n12 = [[nf12.compress(src[j]) for j in g] for _, g in groups]
-    for depth in (0, 1, 2):
-        st = jit.LayerStreamer(n12, depth=depth, device=dev)
-        t = timed(lambda: st.run(consume))
-        assert st.errors() == 0
-        rec[f"nf12_depth{depth}_ms_per_pass"] = round(t, 3)
-        rec[f"nf12_depth{depth}_overhead_pct"] = round(100.0 * (t - t_res) / t_res, 2)
+    for fmt, ls in (("", layers), ("nf12_", n12)):
+        st = jit.LayerStreamer(ls, depth=0, device=dev)
+        rec[f"{fmt}decode_alone_ms_per_pass"] = round(timed(lambda: st.run(lambda l, v: None)), 3)
         del st
-    st = jit.LayerStreamer(n12, depth=0, device=dev)
-    rec["nf12_decode_alone_ms_per_pass"] = round(timed(lambda: st.run(lambda l, v: None)), 3)
+
+    # every just-in-time layer equals the resident weights (depth 1, both formats)
     def check(l, views):
         for a, b in zip(views, resident[l]):
             if not torch.equal(a, b.view(torch.int16).reshape(-1)):
-                raise SystemExit(f"nf12 just-in-time decode mismatch, layer {l}")
+                raise SystemExit(f"just-in-time decode differs from the resident weights, layer {l}")
 
-    st.run(check)
-    torch.cuda.synchronize()
-    del st, n12
-    # check the just-in-time weights against the resident ones on the last layer
-    st1 = jit.LayerStreamer(layers, depth=1, device=dev)
-    seen = {}
-    st1.run(lambda l, v: seen.__setitem__(l, [t.clone() for t in v]) if l == len(groups) - 1 else None)
-    torch.cuda.synchronize()
-    for a, b in zip(seen[len(groups) - 1], resident[-1]):
-        if not torch.equal(a, b.view(torch.int16).reshape(-1)):
-            raise SystemExit("jit_layer decode differs from the resident weights")
+    for ls in (layers, n12):
+        st = jit.LayerStreamer(ls, depth=1, device=dev)
+        st.run(check)
+        torch.cuda.synchronize()
+        del st
+    del n12
     return rec
 
 
