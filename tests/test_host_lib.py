@@ -382,3 +382,40 @@ def test_host_sha256_against_hashlib():
     for n in (1, 55, 56, 57, 63, 64, 65, 119, 120, 128, 1000, 65536, 65537):
         data = rng.integers(0, 256, n, dtype=np.uint8).tobytes()
         assert api.df_sha256(data) == hashlib.sha256(data).digest(), n
+
+
+def test_new_entry_points_refuse_bad_arguments_before_any_device_work():
+    """The fixed 12-bit format's and the compact index's calls check their
+    arguments on the host and return before touching a device (no GPU here)."""
+    import ctypes
+
+    L = _native.lib()
+    z = _native.DfNf12Sizes()
+    assert L.df_nf12_sizes_for((1 << 48) + 1, ctypes.byref(z)) == _native.DF_ERR_UNSUPPORTED  # DF_MAX_WEIGHTS + 1
+    assert L.df_nf12_sizes_for(10, None) == _native.DF_ERR_INVALID_ARG
+    # decode: top above 15, a reserved field set, misaligned slots
+    t = _native.DfNf12Tensor()
+    t.n, t.slots, t.bitmap, t.out, t.top = 16, 256, 512, 1024, 16
+    assert L.df_nf12_decode(ctypes.byref(t), None, None) == _native.DF_ERR_INVALID_ARG
+    t.top, t.reserved = 7, 1
+    assert L.df_nf12_decode(ctypes.byref(t), None, None) == _native.DF_ERR_INVALID_ARG
+    t.reserved, t.slots = 0, 258
+    assert L.df_nf12_decode(ctypes.byref(t), None, None) == _native.DF_ERR_INVALID_ARG
+    # grouped encode: workspace size, then a descriptor with top 16
+    e = (_native.DfNf12EncodeTensor * 2)()
+    e[0].n, e[1].n = 16384 * 3 + 5, 9  # 4 tiles and 1 tile
+    for x in e:
+        x.input, x.slots, x.bitmap, x.top = 256, 512, 1024, 7
+    ws = L.df_nf12_encode_batch_workspace(e, 2)
+    assert ws == 2 * 64 + 8 * 3 + 8 * 5 + 8 * 2
+    plan = _native.DfNf12Plan()
+    e[1].top = 16
+    assert L.df_nf12_encode_batch_prepare(e, 2, 4096, ws, ctypes.byref(plan), None) == _native.DF_ERR_INVALID_ARG
+    e[1].top = 7
+    assert L.df_nf12_encode_batch_prepare(e, 2, 4096, ws - 8, ctypes.byref(plan), None) == _native.DF_ERR_WORKSPACE
+    # compact index: misaligned buffer, too small a buffer, too many blocks
+    wide = 4096
+    assert L.df_index8_build(256, 10, 260, 76, wide, None, None) == _native.DF_ERR_INVALID_ARG
+    assert L.df_index8_build(256, 100, 512, 76, wide, None, None) == _native.DF_ERR_INVALID_ARG  # needs 152
+    assert L.df_index8_build(256, 1 << 32, 512, 1 << 40, wide, None, None) == _native.DF_ERR_UNSUPPORTED
+    assert L.df_index8_expand(512, 64, 2, 256, None, None) == _native.DF_ERR_INVALID_ARG  # 2 wide of 1 superblock
