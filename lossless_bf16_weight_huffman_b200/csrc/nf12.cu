@@ -16,9 +16,13 @@
 //
 // Encode writes side entries in group order. The pass over the groups counts
 // escapes per tile; a one-block scan turns the counts into tile bases; a
-// second pass over the bitmap (one block per tile with escapes, usually a few
-// percent of groups) writes side entries and side indices. The caller reads
-// the total between the passes to size the side buffer.
+// second pass over the bitmap (a 64-thread CUDA block per tile, which returns
+// at once when its tile has no escapes; escapes are usually 1-2% of groups)
+// writes side entries and side indices. The caller reads the total between
+// the passes to size the side buffer. The grouped encode runs the same three
+// steps once for many tensors: tiles of every tensor in one launch (a tile
+// finds its tensor by binary search over the tensors' first tiles), one
+// CUDA block per tensor for the scans.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
