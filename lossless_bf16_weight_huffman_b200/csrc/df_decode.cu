@@ -932,6 +932,48 @@ df_status df_decode_batch_prepare(const df_tensor* tensors, uint16_t* const* d_o
     if (st != DF_OK) return st;
     plan->cta_threads = warps * kLanes;
     plan->smem_bytes = static_cast<uint32_t>(smem_bytes(cfg, warps));
+    // A CUDA block decodes a contiguous range of format blocks, restaging the
+    // tables (and waiting for all its warps) at every tensor; a tensor of
+    // fewer format blocks than warps leaves most warps idle until the next
+    // restage. When such small tensors outnumber the resident CUDA blocks,
+    // spread them evenly between the large ones, so every range holds its
+    // share instead of a few ranges holding clusters of them (the descriptors
+    // carry their own outputs, so their order is free). A few small tensors
+    // stay where they are: moving one only adds a restage.
+    int sms = 0, max_smem = 0, per_sm = 0;
+    st = device_limits(&sms, &max_smem, &per_sm);
+    if (st != DF_OK) return st;
+    const uint64_t resident = static_cast<uint64_t>(sms) *
+                              std::max<uint64_t>(1, static_cast<uint64_t>(per_sm) / (plan->smem_bytes + 1024));
+    {
+        std::vector<uint32_t> small, large;
+        uint64_t large_blocks = 0;
+        for (uint32_t i = 0; i < dev.size(); ++i) {
+            if (dev[i].n_blocks < warps) {
+                small.push_back(i);
+            } else {
+                large.push_back(i);
+                large_blocks += dev[i].n_blocks;
+            }
+        }
+        if (small.size() >= resident && !large.empty()) {
+            std::vector<DevTensor> order;
+            order.reserve(dev.size());
+            uint64_t done = 0;  // large blocks placed so far
+            size_t si = 0;
+            for (uint32_t li : large) {
+                order.push_back(dev[li]);
+                done += dev[li].n_blocks;
+                // small tensor k belongs after (k + 1/2) / small.size() of the large blocks
+                while (si < small.size() && static_cast<unsigned __int128>(2 * si + 1) * large_blocks <=
+                                                static_cast<unsigned __int128>(2 * done) * small.size())
+                    order.push_back(dev[small[si++]]);
+            }
+            while (si < small.size()) order.push_back(dev[small[si++]]);
+            dev.swap(order);
+            for (size_t i = 0; i < dev.size(); ++i) start[i + 1] = start[i] + dev[i].n_blocks;
+        }
+    }
     // layout: the live descriptors (rounded up to 256 bytes), then the block
     // prefix sums. Copies from pageable host memory return once the source has
     // been staged, so the host vectors may die on return.
