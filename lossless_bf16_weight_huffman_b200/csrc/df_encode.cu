@@ -20,7 +20,8 @@
 // boundary, the block offset. Whole words go out with plain stores, the
 // words a tile shares with its neighbours with atomic ORs into the zeroed
 // buffers. The input is read three times in all: by the histogram and by
-// both passes.
+// both passes; each pass asks for its input two warp tiles ahead (an L2
+// prefetch hint).
 #include <cuda_runtime.h>
 
 #include <cstring>
@@ -96,6 +97,12 @@ __device__ __forceinline__ uint32_t load16(const uint16_t* __restrict__ in, uint
         }
     }
     return full ? kPerThread : (i0 < n ? static_cast<uint32_t>(n - i0) : 0u);
+}
+
+// Hint that weight i (below n) of `in` will be read soon: its line is
+// fetched into L2 now. No effect on results.
+__device__ __forceinline__ void prefetch_l2(const uint16_t* in, uint64_t n, uint64_t i) {
+    if (i < n) asm volatile("prefetch.global.L2 [%0];" ::"l"(in + i));
 }
 
 struct EncArgs {
@@ -250,6 +257,7 @@ __device__ __forceinline__ uint32_t pack64(const uint2* s_cl, const uint32_t wv[
 }
 
 constexpr uint32_t kWarpTile = 32 * kPerThread;      // 512 weights: a warp, 16 consecutive weights per lane
+constexpr uint32_t kPrefetchTiles = 2;  // both passes ask for the input this many warp tiles ahead
 constexpr uint32_t kEncWarps = kEncThreads / 32;
 constexpr uint32_t kWarpWords = kWarpTile + 2;       // a warp tile holds at most 512 codes of at most 32 bits
 // gap fields a warp tile can hold (every code 32 bits, 16-byte chunks) as
@@ -297,8 +305,11 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(EncArgs a, EncTable
     // 1. sign|fraction bytes and the bit count of this warp's sub-range
     uint64_t lsum = 0;
     bool missing = false;
+    for (uint32_t d = 1; d < kPrefetchTiles; ++d)
+        if (t_begin + d < t_end) prefetch_l2(a.in, a.n, (t_begin + d) * kWarpTile + lane * kPerThread);
     for (uint64_t t = t_begin; t < t_end; ++t) {
         const uint64_t i0 = t * kWarpTile + lane * kPerThread;
+        if (t + kPrefetchTiles < t_end) prefetch_l2(a.in, a.n, i0 + kPrefetchTiles * kWarpTile);
         uint32_t wv[kPerThread / 2];
         const uint32_t cnt = load16(a.in, a.n, i0, a.in_vec != 0, wv);
         uint32_t smw[kPerThread / 4];
@@ -341,8 +352,11 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(EncArgs a, EncTable
     uint32_t rr = static_cast<uint32_t>(bit0 % cbits);  // bit0 = jc * cbits + rr
     uint64_t jc = bit0 / cbits;
     uint32_t jcT = static_cast<uint32_t>(jc % T);
+    for (uint32_t d = 1; d < kPrefetchTiles; ++d)
+        if (t_begin + d < t_end) prefetch_l2(a.in, a.n, (t_begin + d) * kWarpTile + lane * kPerThread);
     for (uint64_t t = t_begin; t < t_end; ++t) {
         const uint64_t i0 = t * kWarpTile + lane * kPerThread;
+        if (t + kPrefetchTiles < t_end) prefetch_l2(a.in, a.n, i0 + kPrefetchTiles * kWarpTile);
         uint32_t wv[kPerThread / 2];
         const uint32_t cnt = load16(a.in, a.n, i0, a.in_vec != 0, wv);
         unsigned long long v, ends;
