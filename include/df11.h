@@ -59,7 +59,7 @@ typedef int df_status;
 #define DF_ERR_INVALID_ARG 1 /* a null, misaligned or inconsistent argument     */
 #define DF_ERR_CUDA 2        /* a CUDA call failed; see df_last_cuda_error()   */
 #define DF_ERR_CORRUPT 3     /* the device error word reported corrupt data     */
-#define DF_ERR_UNSUPPORTED 4 /* valid but outside this build's limits           */
+#define DF_ERR_UNSUPPORTED 4 /* valid but outside this library's limits         */
 #define DF_ERR_WORKSPACE 5   /* workspace too small                             */
 
 /* bits of the device error word */
