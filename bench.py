@@ -454,6 +454,52 @@ def encode_set(specs, dev, args, staging):
     return src, comps, hist_ms, enc_ms
 
 
+def grouped_encode_record(src, comps, args, peak, steps=5):
+    """The grouped encoder (codec.BatchEncoder: one histogram launch, then one
+    zeroing launch and one encode launch for all tensors) on the same tensors:
+    its containers against those of the per-tensor calls, and its device time
+    per step (CUDA events around each part, median of `steps`; inputs not
+    flushed from L2 between steps)."""
+    import statistics
+
+    import torch
+
+    from lossless_bf16_weight_huffman_b200 import api, codec
+
+    n = sum(x.numel() for x in src)
+    enc = codec.BatchEncoder(src, chunk_bytes=args.chunk_bytes, threads_per_block=args.threads_per_block)
+    got = enc.prepare()
+    err = torch.zeros(1, dtype=torch.int32, device=src[0].device)
+    enc.run(err)
+    torch.cuda.synchronize()
+    flags = api.df_read_error(err)
+    equal = flags == 0 and all(
+        a.total_bits == b.total_bits and torch.equal(a.stream, b.stream) and torch.equal(a.gaps, b.gaps)
+        and torch.equal(a.offsets, b.offsets) and torch.equal(a.sm[: a.n], b.sm[: b.n])
+        for a, b in zip(got, comps))
+    hist_t, enc_t = [], []
+    for _ in range(steps):
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e0.record()
+        enc.run_histograms()
+        e1.record()
+        enc.run(err)
+        e2.record()
+        torch.cuda.synchronize()
+        hist_t.append(e0.elapsed_time(e1))
+        enc_t.append(e1.elapsed_time(e2))
+    h, e = statistics.median(hist_t), statistics.median(enc_t)
+    algo = 4 * n + n + sum(c.sizes["stream_bytes"] for c in comps)
+    del enc, got
+    torch.cuda.empty_cache()
+    return {"value": round(2 * n / ((h + e) / 1e3) / 1e9, 2), "unit": "GB/s of BF16 input",
+            "histogram_ms": round(h, 4), "encode_ms": round(e, 4),
+            "roofline_frac": round(algo / ((h + e) / 1e3) / 1e9 / peak, 4),
+            "equal_to_per_tensor_calls": bool(equal), "error_flags": flags, "tensors": len(src),
+            "note": "df_histogram_batch_run (a memset, one kernel) and df_encode_batch_run (a zeroing kernel, a "
+                    "memset, one encode kernel) over all tensors; algorithmic bytes as the per-tensor record"}
+
+
 def time_launches(run, steps, warmup, stream, flush=None):
     """Per-step device ms of run() (CUDA events on `stream`). With `flush`, a
     write larger than L2 precedes every step, outside its events."""
@@ -885,6 +931,7 @@ def run_gpu(args, world, rank, local, pool, ncores):
         cfg[args.workload]["nf12"] = nf12_record(src, outs, args, stream, err, peak, fl)
         torch.cuda.empty_cache()
         cfg[args.workload]["idx8"] = idx8_record(comps, outs, src, args, stream, err, peak, fl)
+        extras["encode_grouped"] = grouped_encode_record(src, comps, args, peak)
         for name in ("single_1024x4096", "llama_layer", "heavy_tail_64m", "mixed_2000"):
             if name == args.workload:
                 continue
@@ -895,6 +942,7 @@ def run_gpu(args, world, rank, local, pool, ncores):
             cfg[name] = decode_record(s_comps, s_outs, args, stream, err, peak, fl)
             verify(s_src, s_outs, [s.name for s in sp])
             cfg[name]["nf12"] = nf12_record(s_src, s_outs, args, stream, err, peak, fl)
+            cfg[name]["encode_grouped"] = grouped_encode_record(s_src, s_comps, args, peak)
             del s_src, s_comps, s_outs, stg
         extras["configs"] = cfg
         del fl

@@ -134,6 +134,36 @@ typedef struct df_batch_plan {
     uint64_t total_blocks;     /* format blocks over all tensors                */
 } df_batch_plan;
 
+/* One tensor of a grouped encode (host array; read by
+ * df_encode_batch_prepare before it returns). Inputs and outputs as
+ * df_encode's arguments of the same names. A table whose `code` entries are
+ * all NULL plans the histograms only; a table with every code set (and its
+ * outputs) plans the encode as well. */
+typedef struct df_encode_tensor {
+    const uint16_t* in;        /* device, n BF16 bit patterns, 2-byte aligned   */
+    uint64_t n;
+    const df_code* code;       /* host; NULL until the histogram is known      */
+    uint64_t total_bits;       /* df_plan's value for this tensor and code     */
+    uint32_t chunk_bytes;      /* C: multiple of 16 in 16..4096                */
+    uint32_t threads_per_block; /* T: multiple of 32 in 32..1024               */
+    uint8_t* stream;           /* device, sizes.stream_bytes, 16-byte aligned  */
+    uint8_t* gaps;             /* device, sizes.gap_bytes, 4-byte aligned      */
+    uint64_t* block_offsets;   /* device, n_blocks + 1, 8-byte aligned         */
+    uint8_t* sm;               /* device, n bytes                              */
+} df_encode_tensor;
+
+/* Host plan of a grouped encode, filled by df_encode_batch_prepare. */
+typedef struct df_encode_plan {
+    void* d_ws;                /* the workspace holding the device tables       */
+    uint32_t count;            /* tensors                                       */
+    uint32_t has_codes;        /* 1: every tensor has its code and outputs      */
+    uint64_t sum_tiles;        /* sum of ceil(n / 4096) (sizes the workspace)   */
+    uint64_t hist_tiles;       /* CUDA blocks of the grouped histogram          */
+    uint64_t hist_tile_weights; /* weights per histogram CUDA block             */
+    uint64_t ranges;           /* encode ranges over all tensors               */
+    uint64_t zero_tiles;       /* CUDA blocks that zero the outputs             */
+} df_encode_plan;
+
 /* Human-readable name of a status. Static string; never NULL.
  * Source: none on the pages (an error-reporting helper of this ABI). */
 const char* df_status_string(df_status s);
@@ -261,6 +291,47 @@ df_status df_encode(const df_code* code, const uint16_t* d_in, uint64_t n, uint6
 df_status df_encode_noalloc(const df_code* code, const uint16_t* d_in, uint64_t n, uint64_t total_bits,
                             uint32_t chunk_bytes, uint32_t threads_per_block, uint8_t* d_stream, uint8_t* d_gaps,
                             uint64_t* d_block_offsets, uint8_t* d_sm, uint32_t* d_err, void* stream);
+
+/* ---- grouped encode (device) ---------------------------------------------------
+ * df_histogram and df_encode over many tensors with one launch per step for
+ * all of them, so that many small tensors (biases, norms, small linears) cost
+ * a few launches instead of several each. Every tensor's histogram and
+ * container bytes equal those of df_histogram and df_encode on it alone.
+ * Source: df11pack, intro (the codebook from each tensor's exponent
+ * frequencies; the compressor's speed over a whole model's tensors is the
+ * page's headline, "Measured"); grouping them into one launch is this
+ * library's own.
+ *
+ * df_encode_batch_workspace: device workspace bytes for these tensors (only
+ * their n is read, so one workspace serves both prepare calls). */
+size_t df_encode_batch_workspace(const df_encode_tensor* h_tensors, uint32_t count);
+
+/* df_encode_batch_prepare: validate the table, copy the device descriptors
+ * (and the codes, when every tensor has one) into d_ws (16-byte aligned)
+ * asynchronously on `stream`, and fill *plan. Call it once with the codes
+ * NULL to run the histograms, then again with every code and output set
+ * (after df_build_code and df_plan on the host) to run the encode. Errors:
+ * DF_ERR_INVALID_ARG (a bad pointer, alignment or format, a code length over
+ * 32, codes set for some tensors only), DF_ERR_WORKSPACE, DF_ERR_UNSUPPORTED
+ * (n > DF_MAX_WEIGHTS; more than 2^31 - 1 CUDA blocks or ranges), DF_ERR_CUDA.
+ * Source: as the section above. */
+df_status df_encode_batch_prepare(const df_encode_tensor* h_tensors, uint32_t count, void* d_ws, size_t ws_bytes,
+                                  df_encode_plan* plan, void* stream);
+
+/* df_histogram_batch_run: d_hist[256 t + e] = the number of weights of tensor
+ * t whose exponent bits equal e, for every tensor of the plan (d_hist: count
+ * x 256 uint64, device, 8-byte aligned; overwritten). One launch over fixed
+ * tiles of every tensor. Source: as df_histogram. Errors: DF_ERR_INVALID_ARG,
+ * DF_ERR_CUDA. */
+df_status df_histogram_batch_run(const df_encode_plan* plan, uint64_t* d_hist, void* stream);
+
+/* df_encode_batch_run: write every tensor's container, as df_encode does for
+ * one: a launch that zeroes all outputs, then one over ranges of every tensor
+ * (a tensor's look-back stays within its own ranges). Needs a plan prepared
+ * with every code. A wrong total_bits or an exponent without a code sets
+ * DF_EFLAG_ENC_* in d_err (nullable), as in df_encode. Source: as df_encode.
+ * Errors: DF_ERR_INVALID_ARG, DF_ERR_CUDA. */
+df_status df_encode_batch_run(const df_encode_plan* plan, uint32_t* d_err, void* stream);
 
 /* ---- decode (device) ---------------------------------------------------------
  * df_decode: d_out[0..t->n) = the original BF16 bit patterns (uint16, device;

@@ -38,8 +38,9 @@ DF_ENCODE_NOALLOC_MAX_WEIGHTS = 1 << 29
 EXPORTS = (
     "df_status_string", "df_last_cuda_error", "df_build_code", "df_code_from_lengths", "df_lut_words", "df_build_lut", "df_plan",
     "df_container_sizes",
-    "df_histogram", "df_encode", "df_encode_noalloc", "df_decode", "df_decode_batch_workspace", "df_decode_batch_prepare",
-    "df_decode_batch_run", "df_decode_batch", "df_read_error", "df_check_structure", "df_compare",
+    "df_histogram", "df_encode", "df_encode_noalloc", "df_encode_batch_workspace", "df_encode_batch_prepare",
+    "df_histogram_batch_run", "df_encode_batch_run", "df_decode", "df_decode_batch_workspace",
+    "df_decode_batch_prepare", "df_decode_batch_run", "df_decode_batch", "df_read_error", "df_check_structure", "df_compare",
     "df_sha256_workspace", "df_sha256_device", "df_sha256", "df_index8_bytes", "df_index8_build",
     "df_index8_expand",
     "df_nf12_sizes_for", "df_nf12_encode_groups", "df_nf12_encode_escapes", "df_nf12_decode",
@@ -111,6 +112,34 @@ class DfBatchPlan(ctypes.Structure):
         ("max_ctas", ctypes.c_uint32),
         ("reserved", ctypes.c_uint32),
         ("total_blocks", ctypes.c_uint64),
+    ]
+
+
+class DfEncodeTensor(ctypes.Structure):
+    _fields_ = [
+        ("input", ctypes.c_void_p),
+        ("n", ctypes.c_uint64),
+        ("code", ctypes.POINTER(DfCode)),
+        ("total_bits", ctypes.c_uint64),
+        ("chunk_bytes", ctypes.c_uint32),
+        ("threads_per_block", ctypes.c_uint32),
+        ("stream", ctypes.c_void_p),
+        ("gaps", ctypes.c_void_p),
+        ("block_offsets", ctypes.c_void_p),
+        ("sm", ctypes.c_void_p),
+    ]
+
+
+class DfEncodePlan(ctypes.Structure):
+    _fields_ = [
+        ("d_ws", ctypes.c_void_p),
+        ("count", ctypes.c_uint32),
+        ("has_codes", ctypes.c_uint32),
+        ("sum_tiles", ctypes.c_uint64),
+        ("hist_tiles", ctypes.c_uint64),
+        ("hist_tile_weights", ctypes.c_uint64),
+        ("ranges", ctypes.c_uint64),
+        ("zero_tiles", ctypes.c_uint64),
     ]
 
 
@@ -198,6 +227,15 @@ def lib() -> ctypes.CDLL:
     L.df_encode.restype = i32
     L.df_encode_noalloc.argtypes = [ctypes.POINTER(DfCode), vp, u64, u64, u32, u32, vp, vp, vp, vp, vp, vp]
     L.df_encode_noalloc.restype = i32
+    L.df_encode_batch_workspace.argtypes = [ctypes.POINTER(DfEncodeTensor), u32]
+    L.df_encode_batch_workspace.restype = sz
+    L.df_encode_batch_prepare.argtypes = [ctypes.POINTER(DfEncodeTensor), u32, vp, sz, ctypes.POINTER(DfEncodePlan),
+                                          vp]
+    L.df_encode_batch_prepare.restype = i32
+    L.df_histogram_batch_run.argtypes = [ctypes.POINTER(DfEncodePlan), vp, vp]
+    L.df_histogram_batch_run.restype = i32
+    L.df_encode_batch_run.argtypes = [ctypes.POINTER(DfEncodePlan), vp, vp]
+    L.df_encode_batch_run.restype = i32
     L.df_decode.argtypes = [ctypes.POINTER(DfTensor), vp, vp, vp]
     L.df_decode.restype = i32
     L.df_decode_batch_workspace.argtypes = [u32]

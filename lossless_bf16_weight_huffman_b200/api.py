@@ -9,8 +9,8 @@ import ctypes
 import numpy as np
 import torch
 
-from ._native import (DfBatchPlan, DfCode, DfNf12EncodeTensor, DfNf12Plan, DfNf12Sizes, DfNf12Tensor, DfSizes,
-                      DfTensor, check, lib)
+from ._native import (DfBatchPlan, DfCode, DfEncodePlan, DfEncodeTensor, DfNf12EncodeTensor, DfNf12Plan,
+                      DfNf12Sizes, DfNf12Tensor, DfSizes, DfTensor, check, lib)
 
 
 def _stream_ptr(stream=None):
@@ -136,6 +136,37 @@ def df_encode(code: DfCode, d_in: torch.Tensor, total_bits: int, chunk_bytes: in
         ctypes.byref(code), _dev(d_in, "d_in"), d_in.numel(), total_bits, chunk_bytes, threads_per_block,
         _dev(d_stream, "d_stream"), _dev(d_gaps, "d_gaps"), _dev(d_block_offsets, "d_block_offsets"),
         _dev(d_sm, "d_sm"), _dev(d_ws, "d_ws"), ws_bytes, _dev(d_err, "d_err"), _stream_ptr(stream)))
+
+
+def _encode_array(tensors):
+    return (DfEncodeTensor * max(1, len(tensors)))(*tensors)
+
+
+def df_encode_batch_workspace(tensors) -> int:
+    return int(lib().df_encode_batch_workspace(_encode_array(tensors), len(tensors)))
+
+
+def df_encode_batch_prepare(tensors, d_ws: torch.Tensor, stream=None) -> DfEncodePlan:
+    """tensors: DfEncodeTensor list (device pointers as ints; `code` a
+    pointer to a DfCode the caller keeps alive until the call returns)."""
+    _need(d_ws, df_encode_batch_workspace(tensors), "d_ws")
+    plan = DfEncodePlan()
+    check("df_encode_batch_prepare", lib().df_encode_batch_prepare(
+        _encode_array(tensors), len(tensors), _dev(d_ws, "d_ws"), d_ws.numel() * d_ws.element_size(),
+        ctypes.byref(plan), _stream_ptr(stream)))
+    return plan
+
+
+def df_histogram_batch_run(plan: DfEncodePlan, d_hist: torch.Tensor, stream=None) -> None:
+    _need(d_hist, 2048 * plan.count, "d_hist")
+    check("df_histogram_batch_run", lib().df_histogram_batch_run(
+        ctypes.byref(plan), _dev(d_hist, "d_hist"), _stream_ptr(stream)))
+
+
+def df_encode_batch_run(plan: DfEncodePlan, d_err: torch.Tensor | None = None, stream=None) -> None:
+    _need_err(d_err)
+    check("df_encode_batch_run", lib().df_encode_batch_run(ctypes.byref(plan), _dev(d_err, "d_err"),
+                                                           _stream_ptr(stream)))
 
 
 def df_encode_noalloc(code: DfCode, d_in: torch.Tensor, total_bits: int, chunk_bytes: int, threads_per_block: int,

@@ -2,17 +2,20 @@
 container held in torch CUDA buffers, and decode one or many containers.
 
 PyTorch only allocates memory here; every step of the codec runs in
-libdf11.so (df_histogram, df_encode, df_decode, df_decode_batch_*). Building
+libdf11.so (df_histogram, df_encode, df_encode_batch_*, df_decode,
+df_decode_batch_*). Building
 the code table is host work done by df_build_code / df_build_lut in the same
 library. There is no CPU fallback: CPU tensors are rejected.
 """
 from __future__ import annotations
 
+import ctypes
+
 import numpy as np
 import torch
 
 from . import api
-from ._native import DfTensor
+from ._native import DfEncodeTensor, DfTensor
 
 DEFAULT_MAX_LEN = 32
 DEFAULT_CHUNK_BYTES = 32
@@ -220,6 +223,105 @@ def compress(w: torch.Tensor, max_len: int = DEFAULT_MAX_LEN, chunk_bytes: int |
         if api.df_read_error(err, stream) or int(first.cpu().numpy().view(np.uint64)[0]) != 2**64 - 1:
             raise SafeCheckError("the container does not decode to its source")
     return c
+
+
+def _per_tensor(value, count: int, name: str) -> list:
+    if isinstance(value, (list, tuple)):
+        if len(value) != count:
+            raise ValueError(f"{name}: one value per tensor")
+        return list(value)
+    return [value] * count
+
+
+class BatchEncoder:
+    """A grouped encode of many tensors (df_encode_batch_*): one launch for
+    all the exponent histograms, the codes built on the host (one wait for
+    the histograms), then one launch that zeroes every output and one that
+    encodes every tensor. Each container equals compress()'s for the same
+    tensor and format. chunk_bytes (None: auto_chunk_bytes per tensor) and
+    threads_per_block may be one value or one per tensor. prepare() reads the
+    histograms and allocates the containers; run() encodes into them (again
+    on every call, e.g. to time it)."""
+
+    def __init__(self, ws: list[torch.Tensor], max_len: int = DEFAULT_MAX_LEN, chunk_bytes=None,
+                 threads_per_block=DEFAULT_THREADS_PER_BLOCK, stream=None):
+        if not ws:
+            raise ValueError("no tensors")
+        self.xs = [_as_u16(w) for w in ws]
+        self.shapes = [tuple(w.shape) for w in ws]
+        self.dev = self.xs[0].device
+        if any(x.device != self.dev for x in self.xs):
+            raise ValueError("all tensors must be on one device")
+        self.max_len = max_len
+        self.chunk_bytes = _per_tensor(chunk_bytes, len(self.xs), "chunk_bytes")
+        self.tpb = _per_tensor(threads_per_block, len(self.xs), "threads_per_block")
+        self.hist = torch.empty((len(self.xs), 256), dtype=torch.int64, device=self.dev)
+        descs = self._descriptors()
+        self.ws = torch.empty(max(api.df_encode_batch_workspace(descs), 16), dtype=torch.uint8, device=self.dev)
+        self.plan = api.df_encode_batch_prepare(descs, self.ws, stream)
+        self.comps: list[Compressed] | None = None
+
+    def _descriptors(self, comps: list[Compressed] | None = None) -> list[DfEncodeTensor]:
+        out = []
+        for i, x in enumerate(self.xs):
+            t = DfEncodeTensor()
+            t.input = x.data_ptr() if x.numel() else None
+            t.n = x.numel()
+            if comps is not None:
+                c = comps[i]
+                t.code = ctypes.pointer(c.code)
+                t.total_bits = c.total_bits
+                t.chunk_bytes = c.chunk_bytes
+                t.threads_per_block = c.threads_per_block
+                t.stream = c.stream.data_ptr()
+                t.gaps = c.gaps.data_ptr()
+                t.block_offsets = c.offsets.data_ptr()
+                t.sm = c.sm.data_ptr()
+            out.append(t)
+        return out
+
+    def run_histograms(self, stream=None) -> None:
+        """Every tensor's exponent histogram into self.hist (one launch)."""
+        api.df_histogram_batch_run(self.plan, self.hist, stream)
+
+    def histograms(self, stream=None) -> np.ndarray:
+        self.run_histograms(stream)
+        if stream is not None:
+            stream.synchronize()
+        return self.hist.cpu().numpy().view(np.uint64)
+
+    def prepare(self, stream=None) -> list[Compressed]:
+        hist = self.histograms(stream)
+        comps = []
+        for i, x in enumerate(self.xs):
+            n = x.numel()
+            code = api.df_build_code(hist[i], self.max_len)
+            C = self.chunk_bytes[i] or auto_chunk_bytes(code)
+            T = self.tpb[i]
+            lut = torch.from_numpy(api.df_build_lut(code).view(np.int32)).to(self.dev)
+            z = api.df_plan(code, hist[i], n, C, T).as_dict()
+            comps.append(Compressed(
+                n=n, shape=self.shapes[i], code=code, lut=lut, sizes=z, chunk_bytes=C, threads_per_block=T,
+                stream=torch.empty(z["stream_bytes"], dtype=torch.uint8, device=self.dev),
+                gaps=torch.empty(z["gap_bytes"], dtype=torch.uint8, device=self.dev),
+                offsets=torch.empty(z["n_blocks"] + 1, dtype=torch.int64, device=self.dev),
+                sm=torch.empty(max(n, 16), dtype=torch.uint8, device=self.dev)))
+        self.plan = api.df_encode_batch_prepare(self._descriptors(comps), self.ws, stream)
+        self.comps = comps
+        return comps
+
+    def run(self, d_err: torch.Tensor | None = None, stream=None) -> list[Compressed]:
+        if self.comps is None:
+            self.prepare(stream)
+        api.df_encode_batch_run(self.plan, d_err, stream)
+        return self.comps
+
+
+def compress_batch(ws: list[torch.Tensor], max_len: int = DEFAULT_MAX_LEN, chunk_bytes=None,
+                   threads_per_block=DEFAULT_THREADS_PER_BLOCK, d_err: torch.Tensor | None = None,
+                   stream=None) -> list[Compressed]:
+    """compress() of many tensors with one launch per step for all of them."""
+    return BatchEncoder(ws, max_len, chunk_bytes, threads_per_block, stream).run(d_err, stream)
 
 
 def decompress(c: Compressed, out: torch.Tensor | None = None, d_err: torch.Tensor | None = None,

@@ -24,8 +24,10 @@
 // prefetch hint).
 #include <cuda_runtime.h>
 
+#include <cstddef>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "df_internal.h"
 
@@ -105,7 +107,7 @@ __device__ __forceinline__ void prefetch_l2(const uint16_t* in, uint64_t n, uint
     if (i < n) asm volatile("prefetch.global.L2 [%0];" ::"l"(in + i));
 }
 
-struct EncArgs {
+struct alignas(16) EncArgs {
     const uint16_t* in;
     uint64_t n;
     uint32_t* stream32;     // the stream as 32-bit words (zeroed)
@@ -281,20 +283,25 @@ constexpr uint32_t kWarpGapWords = (5 * (kWarpTile * 32 / 128 + 2) + 31) / 32 + 
 //      format-block boundary, the block offset). The tile's stream and gap
 //      words go out with coalesced stores, except the end words shared with
 //      the neighbouring tiles, which are OR-ed into the zeroed buffers.
-__global__ void __launch_bounds__(kEncThreads) encode_kernel(EncArgs a, EncTables tab) {
-    __shared__ uint2 s_cl[256];  // per exponent: (code right-aligned, length)
-    __shared__ uint32_t s_range;
-    __shared__ unsigned long long s_sum[kEncWarps];
-    __shared__ unsigned long long s_pre[kEncWarps];
-    __shared__ uint32_t s_words[kEncWarps][kWarpWords];
-    __shared__ uint32_t s_gaps[kEncWarps][kWarpGapWords];
+//
+// encode_range does one range with the whole CUDA block: range `range` of
+// the R into which the tensor `a` describes is split, sh.cl holding its code.
+// It has two block-wide barriers of its own (after pass 1 and after the
+// look-back) and none at its start or end: the caller fills sh.cl and a
+// before a barrier and synchronises again before it overwrites them.
+struct EncShared {
+    uint2 cl[256];  // per exponent: (code right-aligned, length)
+    unsigned long long sum[kEncWarps];
+    unsigned long long pre[kEncWarps];
+    uint32_t words[kEncWarps][kWarpWords];
+    uint32_t gaps[kEncWarps][kWarpGapWords];
+};
+
+__device__ __forceinline__ void encode_range(const EncArgs& a, EncShared& sh, uint64_t range, uint64_t R) {
     const uint32_t tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    if (tid == 0) s_range = atomicAdd(a.ticket, 1u);  // ranges start in index order
-    for (uint32_t i = tid; i < 256; i += kEncThreads) {
-        s_cl[i] = make_uint2(tab.codes[i], tab.lengths[i]);
-    }
-    __syncthreads();
-    const uint64_t range = s_range, R = gridDim.x;
+    const uint2* s_cl = sh.cl;
+    unsigned long long* s_sum = sh.sum;
+    unsigned long long* s_pre = sh.pre;
     const uint64_t wtiles = (a.n + kWarpTile - 1) / kWarpTile;
     // balanced contiguous splits (no products that could overflow)
     const uint64_t r_begin = (wtiles / R) * range + min(range, wtiles % R);
@@ -345,8 +352,8 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(EncArgs a, EncTable
     __syncthreads();
 
     // 2. pack, warp tile by warp tile
-    uint32_t* words = s_words[warp];
-    uint32_t* gapw = s_gaps[warp];
+    uint32_t* words = sh.words[warp];
+    uint32_t* gapw = sh.gaps[warp];
     const uint32_t cbits = a.chunk_bits, T = a.threads_per_block, csh = a.cb_shift, tsh = a.t_shift;
     uint64_t bit0 = s_pre[warp];              // the first stream bit of the next tile
     uint32_t rr = static_cast<uint32_t>(bit0 % cbits);  // bit0 = jc * cbits + rr
@@ -530,6 +537,143 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(EncArgs a, EncTable
     }
 }
 
+// One tensor: one range per CUDA block, taken in launch order.
+__global__ void __launch_bounds__(kEncThreads) encode_kernel(EncArgs a, EncTables tab) {
+    __shared__ EncShared sh;
+    __shared__ uint32_t s_range;
+    const uint32_t tid = threadIdx.x;
+    if (tid == 0) s_range = atomicAdd(a.ticket, 1u);  // ranges start in index order
+    for (uint32_t i = tid; i < 256; i += kEncThreads) sh.cl[i] = make_uint2(tab.codes[i], tab.lengths[i]);
+    __syncthreads();
+    encode_range(a, sh, s_range, gridDim.x);
+}
+
+// The index t of the entry with starts[t] <= g < starts[t + 1] (starts
+// non-decreasing, starts[0] = 0 <= g < starts[count]): the tensor that holds
+// unit g of a grouped launch; tensors without units are skipped.
+__device__ __forceinline__ uint32_t tensor_at(const uint64_t* __restrict__ starts, uint32_t count, uint64_t g) {
+    uint32_t lo = 0, hi = count;
+    while (hi - lo > 1) {
+        const uint32_t mid = (lo + hi) >> 1;
+        if (__ldg(starts + mid) <= g)
+            lo = mid;
+        else
+            hi = mid;
+    }
+    return lo;
+}
+
+// Grouped encode of many tensors in one launch: persistent CUDA blocks take
+// ranges from one counter in index order (a tensor's ranges are consecutive,
+// rstart[t] .. rstart[t + 1]); a range's tensor comes from a binary search,
+// its descriptor and code are copied to shared memory, and the range is
+// encoded as encode_kernel does it. Each descriptor's look-back state is its
+// own, so a tensor's first range publishes its prefix at once and no range
+// waits on another tensor's.
+__global__ void __launch_bounds__(kEncThreads)
+    encode_batch_kernel(const EncArgs* __restrict__ descs, const uint2* __restrict__ codes,
+                        const uint64_t* __restrict__ rstart, uint32_t count, uint32_t* ticket, uint32_t* err) {
+    __shared__ EncShared sh;
+    __shared__ EncArgs s_a;
+    __shared__ unsigned long long s_g, s_range, s_R;
+    __shared__ uint32_t s_t;
+    constexpr uint32_t kArgWords = sizeof(EncArgs) / 4;
+    constexpr uint32_t kErrWord = offsetof(EncArgs, err) / 4;
+    const uint32_t tid = threadIdx.x;
+    const uint64_t total = __ldg(rstart + count);
+    for (;;) {
+        if (tid == 0) {
+            const uint64_t g = atomicAdd(ticket, 1u);  // ranges start in index order
+            s_g = g;
+            if (g < total) {
+                const uint32_t t = tensor_at(rstart, count, g);
+                s_t = t;
+                s_range = g - __ldg(rstart + t);
+                s_R = __ldg(rstart + t + 1) - __ldg(rstart + t);
+            }
+        }
+        __syncthreads();  // the last range is done with s_a and sh
+        if (s_g >= total) break;
+        const uint32_t t = s_t;
+        const uint32_t* src = reinterpret_cast<const uint32_t*>(descs + t);
+        uint32_t* dst = reinterpret_cast<uint32_t*>(&s_a);
+        for (uint32_t i = tid; i < kArgWords; i += kEncThreads)
+            if (i != kErrWord && i != kErrWord + 1) dst[i] = __ldg(src + i);
+        if (tid == 0) s_a.err = err;
+        for (uint32_t i = tid; i < 256; i += kEncThreads) sh.cl[i] = __ldg(codes + 256ull * t + i);
+        const uint64_t range = s_range, R = s_R;
+        __syncthreads();
+        encode_range(s_a, sh, range, R);
+    }
+}
+
+// Zeroes the stream, gap and block-offset words of every tensor of a grouped
+// encode (the encoder ORs the words that neighbouring warp tiles share): one
+// CUDA block per kZeroTileWords words of one tensor, zstart[t] .. zstart[t+1]
+// being tensor t's tiles.
+constexpr uint32_t kZeroTileWords = 4096;
+
+__global__ void __launch_bounds__(256)
+    zero_batch_kernel(const EncArgs* __restrict__ descs, const uint64_t* __restrict__ zstart, uint32_t count) {
+    const uint32_t t = tensor_at(zstart, count, blockIdx.x);
+    const EncArgs& d = descs[t];
+    const uint64_t zs = d.stream_words, zg = d.gap_words, zo = 2 * (d.n_blocks + 1);
+    const uint64_t w0 = (blockIdx.x - __ldg(zstart + t)) * kZeroTileWords;
+    const uint64_t w1 = min(w0 + kZeroTileWords, zs + zg + zo);
+    uint32_t* stream32 = d.stream32;
+    uint32_t* gaps32 = d.gaps32;
+    uint32_t* offs32 = reinterpret_cast<uint32_t*>(d.offsets);
+    for (uint64_t w = w0 + threadIdx.x; w < w1; w += blockDim.x) {
+        if (w < zs)
+            stream32[w] = 0;
+        else if (w < zs + zg)
+            gaps32[w - zs] = 0;
+        else
+            offs32[w - zs - zg] = 0;
+    }
+}
+
+// Exponent histograms of every tensor of a grouped encode: one CUDA block per
+// `tile` weights of one tensor (hstart[t] .. hstart[t+1] being tensor t's
+// tiles), per-warp shared counters as in hist_kernel, the block's nonzero
+// counts added to hist[256 t ..]. tile is a multiple of 8, so a 16-byte
+// aligned input stays aligned at every tile start.
+__global__ void __launch_bounds__(256)
+    hist_batch_kernel(const EncArgs* __restrict__ descs, const uint64_t* __restrict__ hstart, uint32_t count,
+                      uint64_t tile, unsigned long long* __restrict__ hist) {
+    __shared__ uint32_t sh[8][256];
+    const uint32_t warp = threadIdx.x >> 5;
+    for (uint32_t i = threadIdx.x; i < 8 * 256; i += blockDim.x) (&sh[0][0])[i] = 0;
+    const uint32_t t = tensor_at(hstart, count, blockIdx.x);
+    const uint16_t* in = descs[t].in;
+    const uint64_t n = descs[t].n;
+    const uint64_t b = (blockIdx.x - __ldg(hstart + t)) * tile;
+    const uint64_t e = min(n, b + tile);
+    __syncthreads();
+    uint64_t done = b;
+    if (descs[t].in_vec) {
+        const uint4* in4 = reinterpret_cast<const uint4*>(in);
+        for (uint64_t i = b / 8 + threadIdx.x; i < e / 8; i += blockDim.x) {
+            const uint4 v = __ldg(in4 + i);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                atomicAdd(&sh[warp][(w[k] >> 7) & 0xFFu], 1u);
+                atomicAdd(&sh[warp][(w[k] >> 23) & 0xFFu], 1u);
+            }
+        }
+        done = e / 8 * 8;
+    }
+    for (uint64_t i = done + threadIdx.x; i < e; i += blockDim.x) atomicAdd(&sh[warp][(__ldg(in + i) >> 7) & 0xFFu], 1u);
+    __syncthreads();
+    for (uint32_t s = threadIdx.x; s < 256; s += blockDim.x) {
+        uint32_t c = 0;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) c += sh[w][s];
+        if (c) atomicAdd(hist + 256ull * t + s, static_cast<unsigned long long>(c));
+    }
+}
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 df_status sm_count(int* sms) {
@@ -539,6 +683,92 @@ df_status sm_count(int* sms) {
     e = cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return cuda_fail(e);
     return DF_OK;
+}
+
+// The descriptor of one tensor's encode for a container of total_bits code
+// bits under chunk_bytes and tpb (the sizes df_container_sizes gives); the
+// look-back state, the range counter and the error word are left to the caller.
+EncArgs make_args(const uint16_t* in, uint64_t n, uint64_t total_bits, uint32_t chunk_bytes, uint32_t tpb,
+                  uint8_t* stream, uint8_t* gaps, uint64_t* offsets, uint8_t* sm) {
+    const uint64_t cbits = 8ull * chunk_bytes;
+    const uint64_t n_chunks = total_bits ? (total_bits + cbits - 1) / cbits : 1;
+    EncArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.in = in;
+    a.n = n;
+    a.stream32 = reinterpret_cast<uint32_t*>(stream);
+    a.gaps32 = reinterpret_cast<uint32_t*>(gaps);
+    a.offsets = offsets;
+    a.sm = sm;
+    a.state = nullptr;
+    a.ticket = nullptr;
+    a.total_bits = total_bits;
+    a.n_chunks = n_chunks;
+    a.stream_words = (n_chunks * chunk_bytes + 16) / 4;
+    a.gap_words = ((((5 * n_chunks + 7) / 8) + 1 + 15) & ~15ull) / 4;
+    a.n_blocks = (n_chunks + tpb - 1) / tpb;
+    a.chunk_bits = static_cast<uint32_t>(cbits);
+    a.threads_per_block = tpb;
+    a.tiles = static_cast<uint32_t>((n + kTile - 1) / kTile);
+    a.err = nullptr;
+    a.in_vec = aligned(in, 16) ? 1u : 0u;
+    a.sm_vec = aligned(sm, 16) ? 1u : 0u;
+    a.cb_shift = a.t_shift = 32;
+    for (uint32_t k = 0; k < 32; ++k) {
+        if ((1ull << k) == cbits) a.cb_shift = k;
+        if ((1u << k) == tpb) a.t_shift = k;
+    }
+    return a;
+}
+
+bool format_ok(uint32_t chunk_bytes, uint32_t tpb) {
+    return chunk_bytes >= 16 && chunk_bytes <= 4096 && chunk_bytes % 16 == 0 && tpb >= 32 && tpb <= 1024 &&
+           tpb % 32 == 0;
+}
+
+// Workspace of a grouped encode: descriptors, codes as (code, length) pairs,
+// the unit prefix sums of the histogram, range and zeroing launches, the
+// range counter and the look-back states (one per range, at most one per 4096
+// weights), each part 16-byte aligned.
+struct EncBatchLayout {
+    size_t descs, codes, hstart, rstart, zstart, ticket, state, bytes;
+};
+
+size_t round16(size_t x) { return (x + 15) & ~static_cast<size_t>(15); }
+
+EncBatchLayout enc_batch_layout(uint32_t count, uint64_t sum_tiles) {
+    EncBatchLayout l;
+    const size_t c = count;
+    size_t o = 0;
+    l.descs = o;
+    o += round16(sizeof(EncArgs) * c);
+    l.codes = o;
+    o += sizeof(uint2) * 256 * c;
+    l.hstart = o;
+    o += round16(8 * (c + 1));
+    l.rstart = o;
+    o += round16(8 * (c + 1));
+    l.zstart = o;
+    o += round16(8 * (c + 1));
+    l.ticket = o;
+    o += 16;
+    l.state = o;
+    o += 8 * static_cast<size_t>(sum_tiles);
+    l.bytes = round16(o);
+    return l;
+}
+
+// Ranges of one tensor in a grouped encode: at most kBatchRangeTiles warp
+// tiles each (several per large tensor, so that CUDA blocks interleave over
+// tensors), at most one per 4096 weights (the look-back state's size).
+constexpr uint64_t kBatchRangeTiles = 64;
+
+uint64_t ranges_of(uint64_t n) {
+    if (n == 0) return 0;
+    const uint64_t wtiles = (n + kWarpTile - 1) / kWarpTile;
+    const uint64_t tiles = (n + kTile - 1) / kTile;
+    const uint64_t r = (wtiles + kBatchRangeTiles - 1) / kBatchRangeTiles;
+    return r < tiles ? r : tiles;
 }
 
 // Scratch of df_encode_noalloc: per-tile bit counts and bases for at most
@@ -617,21 +847,17 @@ df_status df_encode(const df_code* code, const uint16_t* d_in, uint64_t n, uint6
     if (!aligned(d_stream, 16) || !aligned(d_gaps, 4) || !aligned(d_block_offsets, 8) || !aligned(d_in, 2))
         return DF_ERR_INVALID_ARG;
     if (n > DF_MAX_WEIGHTS) return DF_ERR_UNSUPPORTED;
-    const uint64_t cbits = 8ull * chunk_bytes;
-    const uint64_t n_chunks = total_bits ? (total_bits + cbits - 1) / cbits : 1;
-    const uint64_t stream_bytes = n_chunks * chunk_bytes + 16;
-    const uint64_t gap_bytes = (((5 * n_chunks + 7) / 8) + 1 + 15) & ~15ull;
-    const uint64_t n_blocks = (n_chunks + tpb - 1) / tpb;
     const uint64_t tiles = (n + kTile - 1) / kTile;
     const uint64_t need_ws = 16 * (tiles + 2) + 256;
     if (n && (ws_bytes < need_ws || !d_ws)) return DF_ERR_WORKSPACE;
     if (n && !aligned(d_ws, 16)) return DF_ERR_INVALID_ARG;
     if (tiles > 0x7FFFFFFFull) return DF_ERR_UNSUPPORTED;
+    EncArgs a = make_args(d_in, n, total_bits, chunk_bytes, tpb, d_stream, d_gaps, d_block_offsets, d_sm);
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = cudaMemsetAsync(d_stream, 0, stream_bytes, s);
-    if (e == cudaSuccess) e = cudaMemsetAsync(d_gaps, 0, gap_bytes, s);
-    if (e == cudaSuccess) e = cudaMemsetAsync(d_block_offsets, 0, 8 * (n_blocks + 1), s);
+    cudaError_t e = cudaMemsetAsync(d_stream, 0, 4 * a.stream_words, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(d_gaps, 0, 4 * a.gap_words, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(d_block_offsets, 0, 8 * (a.n_blocks + 1), s);
     if (e != cudaSuccess) return cuda_fail(e);
     if (n == 0) return DF_OK;  // empty stream, zero gap, offsets {0, 0}
 
@@ -641,31 +867,9 @@ df_status df_encode(const df_code* code, const uint16_t* d_in, uint64_t n, uint6
     // workspace: per-tile look-back state, then the tile counter; both zeroed
     e = cudaMemsetAsync(d_ws, 0, 8 * tiles + 16, s);
     if (e != cudaSuccess) return cuda_fail(e);
-    EncArgs a;
-    a.in = d_in;
-    a.n = n;
-    a.stream32 = reinterpret_cast<uint32_t*>(d_stream);
-    a.gaps32 = reinterpret_cast<uint32_t*>(d_gaps);
-    a.offsets = d_block_offsets;
-    a.sm = d_sm;
     a.state = static_cast<unsigned long long*>(d_ws);
     a.ticket = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(d_ws) + 8 * tiles);
-    a.total_bits = total_bits;
-    a.n_chunks = n_chunks;
-    a.stream_words = stream_bytes / 4;
-    a.gap_words = gap_bytes / 4;
-    a.n_blocks = n_blocks;
-    a.chunk_bits = static_cast<uint32_t>(cbits);
-    a.threads_per_block = tpb;
-    a.tiles = static_cast<uint32_t>(tiles);
     a.err = d_err;
-    a.in_vec = aligned(d_in, 16) ? 1u : 0u;
-    a.sm_vec = aligned(d_sm, 16) ? 1u : 0u;
-    a.cb_shift = a.t_shift = 32;
-    for (uint32_t k = 0; k < 32; ++k) {
-        if ((1ull << k) == cbits) a.cb_shift = k;
-        if ((1u << k) == tpb) a.t_shift = k;
-    }
     // persistent CUDA blocks: as many as are resident at once, at most one per tile
     int per_sm = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, encode_kernel, kEncThreads, 0);
@@ -690,6 +894,146 @@ df_status df_encode_noalloc(const df_code* code, const uint16_t* d_in, uint64_t 
     if (st != DF_OK) return st;
     return df_encode(code, d_in, n, total_bits, chunk_bytes, tpb, d_stream, d_gaps, d_block_offsets, d_sm, ws,
                      sizeof(g_noalloc_scratch), d_err, stream);
+}
+
+size_t df_encode_batch_workspace(const df_encode_tensor* h_tensors, uint32_t count) {
+    if (count && !h_tensors) return 0;
+    uint64_t sum_tiles = 0;
+    for (uint32_t i = 0; i < count; ++i) sum_tiles += (h_tensors[i].n + kTile - 1) / kTile;
+    return enc_batch_layout(count, sum_tiles).bytes;
+}
+
+df_status df_encode_batch_prepare(const df_encode_tensor* h_tensors, uint32_t count, void* d_ws, size_t ws_bytes,
+                                  df_encode_plan* plan, void* stream) {
+    if (!plan || (count && (!h_tensors || !d_ws)) || !aligned(d_ws, 16)) return DF_ERR_INVALID_ARG;
+    uint32_t with_code = 0;
+    uint64_t sum_tiles = 0, total_n = 0;
+    for (uint32_t i = 0; i < count; ++i) {
+        const df_encode_tensor& t = h_tensors[i];
+        if (t.n > DF_MAX_WEIGHTS) return DF_ERR_UNSUPPORTED;
+        if ((t.n && !t.in) || !aligned(t.in, 2)) return DF_ERR_INVALID_ARG;
+        with_code += t.code ? 1u : 0u;
+        sum_tiles += (t.n + kTile - 1) / kTile;
+        total_n += t.n;
+    }
+    if (with_code && with_code != count) return DF_ERR_INVALID_ARG;
+    const bool has_codes = count && with_code == count;
+    for (uint32_t i = 0; has_codes && i < count; ++i) {
+        const df_encode_tensor& t = h_tensors[i];
+        if (!format_ok(t.chunk_bytes, t.threads_per_block)) return DF_ERR_INVALID_ARG;
+        if (!t.stream || !t.gaps || !t.block_offsets || (t.n && !t.sm)) return DF_ERR_INVALID_ARG;
+        if (!aligned(t.stream, 16) || !aligned(t.gaps, 4) || !aligned(t.block_offsets, 8)) return DF_ERR_INVALID_ARG;
+        for (uint32_t e = 0; e < 256; ++e)
+            if (t.code->lengths[e] > 32) return DF_ERR_INVALID_ARG;
+    }
+    const EncBatchLayout l = enc_batch_layout(count, sum_tiles);
+    if (ws_bytes < l.bytes) return DF_ERR_WORKSPACE;
+
+    // histogram tiles: about four CUDA blocks per resident slot over the whole
+    // set, 2^16 to 2^20 weights each (a power of two, so a multiple of 8)
+    int sms = 0;
+    df_status st = sm_count(&sms);
+    if (st != DF_OK) return st;
+    const uint64_t want = total_n / (4ull * 8 * static_cast<uint64_t>(sms)) + 1;
+    uint64_t tile = 1ull << 16;
+    while (tile < want && tile < (1ull << 20)) tile <<= 1;
+
+    std::vector<EncArgs> descs(count);
+    std::vector<uint2> codes(has_codes ? 256 * static_cast<size_t>(count) : 0);
+    std::vector<uint64_t> hstart(static_cast<size_t>(count) + 1, 0), rstart(hstart), zstart(hstart);
+    uint8_t* ws = static_cast<uint8_t*>(d_ws);
+    for (uint32_t i = 0; i < count; ++i) {
+        const df_encode_tensor& t = h_tensors[i];
+        if (has_codes) {
+            for (uint32_t e = 0; e < 256; ++e)
+                codes[256 * static_cast<size_t>(i) + e] = make_uint2(t.code->codes[e], t.code->lengths[e]);
+            descs[i] = make_args(t.in, t.n, t.total_bits, t.chunk_bytes, t.threads_per_block, t.stream, t.gaps,
+                                 t.block_offsets, t.sm);
+            descs[i].state = reinterpret_cast<unsigned long long*>(ws + l.state) + rstart[i];
+            const uint64_t words = descs[i].stream_words + descs[i].gap_words + 2 * (descs[i].n_blocks + 1);
+            zstart[i + 1] = zstart[i] + (words + kZeroTileWords - 1) / kZeroTileWords;
+            rstart[i + 1] = rstart[i] + ranges_of(t.n);
+        } else {
+            std::memset(&descs[i], 0, sizeof(EncArgs));
+            descs[i].in = t.in;
+            descs[i].n = t.n;
+            descs[i].in_vec = aligned(t.in, 16) ? 1u : 0u;
+        }
+        hstart[i + 1] = hstart[i] + (t.n + tile - 1) / tile;
+    }
+    if (hstart[count] > 0x7FFFFFFFull || rstart[count] > 0x7FFFFFFFull || zstart[count] > 0x7FFFFFFFull)
+        return DF_ERR_UNSUPPORTED;
+    plan->d_ws = d_ws;
+    plan->count = count;
+    plan->has_codes = has_codes ? 1u : 0u;
+    plan->sum_tiles = sum_tiles;
+    plan->hist_tiles = hstart[count];
+    plan->hist_tile_weights = tile;
+    plan->ranges = rstart[count];
+    plan->zero_tiles = zstart[count];
+    if (!count) return DF_OK;
+    // copies from pageable host memory return once the source has been
+    // staged, so the host vectors may die on return
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(ws + l.descs, descs.data(), sizeof(EncArgs) * descs.size(),
+                                    cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess && has_codes)
+        e = cudaMemcpyAsync(ws + l.codes, codes.data(), sizeof(uint2) * codes.size(), cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(ws + l.hstart, hstart.data(), 8 * hstart.size(), cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(ws + l.rstart, rstart.data(), 8 * rstart.size(), cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(ws + l.zstart, zstart.data(), 8 * zstart.size(), cudaMemcpyHostToDevice, s);
+    return e == cudaSuccess ? DF_OK : cuda_fail(e);
+}
+
+df_status df_histogram_batch_run(const df_encode_plan* plan, uint64_t* d_hist, void* stream) {
+    if (!plan || (plan->count && (!plan->d_ws || !d_hist)) || !aligned(d_hist, 8)) return DF_ERR_INVALID_ARG;
+    if (!plan->count) return DF_OK;
+    if (plan->hist_tiles > 0x7FFFFFFFull || plan->hist_tile_weights % 8) return DF_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(d_hist, 0, 256 * sizeof(uint64_t) * plan->count, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (!plan->hist_tiles) return DF_OK;
+    const EncBatchLayout l = enc_batch_layout(plan->count, plan->sum_tiles);
+    const uint8_t* ws = static_cast<const uint8_t*>(plan->d_ws);
+    hist_batch_kernel<<<static_cast<unsigned>(plan->hist_tiles), 256, 0, s>>>(
+        reinterpret_cast<const EncArgs*>(ws + l.descs), reinterpret_cast<const uint64_t*>(ws + l.hstart),
+        plan->count, plan->hist_tile_weights, reinterpret_cast<unsigned long long*>(d_hist));
+    e = cudaGetLastError();
+    return e == cudaSuccess ? DF_OK : cuda_fail(e);
+}
+
+df_status df_encode_batch_run(const df_encode_plan* plan, uint32_t* d_err, void* stream) {
+    if (!plan || (plan->count && !plan->d_ws)) return DF_ERR_INVALID_ARG;
+    if (!plan->count) return DF_OK;
+    if (!plan->has_codes || plan->ranges > 0x7FFFFFFFull || plan->zero_tiles > 0x7FFFFFFFull)
+        return DF_ERR_INVALID_ARG;
+    const EncBatchLayout l = enc_batch_layout(plan->count, plan->sum_tiles);
+    uint8_t* ws = static_cast<uint8_t*>(plan->d_ws);
+    const EncArgs* descs = reinterpret_cast<const EncArgs*>(ws + l.descs);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (plan->zero_tiles) {
+        zero_batch_kernel<<<static_cast<unsigned>(plan->zero_tiles), 256, 0, s>>>(
+            descs, reinterpret_cast<const uint64_t*>(ws + l.zstart), plan->count);
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    if (!plan->ranges) return DF_OK;
+    // the range counter and one look-back state per range, zeroed
+    cudaError_t e = cudaMemsetAsync(ws + l.ticket, 0, 16 + 8 * plan->ranges, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, encode_batch_kernel, kEncThreads, 0);
+    if (e != cudaSuccess) return cuda_fail(e);
+    int sms = 0;
+    const df_status st = sm_count(&sms);
+    if (st != DF_OK) return st;
+    const uint64_t slots = static_cast<uint64_t>(sms) * static_cast<uint64_t>(per_sm < 1 ? 1 : per_sm);
+    const uint64_t grid = plan->ranges < slots ? plan->ranges : slots;
+    encode_batch_kernel<<<static_cast<unsigned>(grid), kEncThreads, 0, s>>>(
+        descs, reinterpret_cast<const uint2*>(ws + l.codes), reinterpret_cast<const uint64_t*>(ws + l.rstart),
+        plan->count, reinterpret_cast<uint32_t*>(ws + l.ticket), d_err);
+    e = cudaGetLastError();
+    return e == cudaSuccess ? DF_OK : cuda_fail(e);
 }
 
 }  // extern "C"

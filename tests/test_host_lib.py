@@ -65,6 +65,8 @@ def test_struct_sizes_match_header_layout():
     assert ctypes.sizeof(_native.DfSizes) == 9 * 8
     assert ctypes.sizeof(_native.DfTensor) == 16 + 16 + 5 * 8 + 256 + 16
     assert ctypes.sizeof(_native.DfBatchPlan) == 8 + 8 * 4 + 8
+    assert ctypes.sizeof(_native.DfEncodeTensor) == 4 * 8 + 2 * 4 + 4 * 8
+    assert ctypes.sizeof(_native.DfEncodePlan) == 8 + 2 * 4 + 5 * 8
     assert ctypes.sizeof(_native.DfNf12Sizes) == 5 * 8
     assert ctypes.sizeof(_native.DfNf12Tensor) == 16 + 4 * 8 + 8
     assert ctypes.sizeof(_native.DfNf12Plan) == 8 + 8 + 8
@@ -419,3 +421,40 @@ def test_new_entry_points_refuse_bad_arguments_before_any_device_work():
     assert L.df_index8_build(256, 100, 512, 76, wide, None, None) == _native.DF_ERR_INVALID_ARG  # needs 152
     assert L.df_index8_build(256, 1 << 32, 512, 1 << 40, wide, None, None) == _native.DF_ERR_UNSUPPORTED
     assert L.df_index8_expand(512, 64, 2, 256, None, None) == _native.DF_ERR_INVALID_ARG  # 2 wide of 1 superblock
+
+
+def test_grouped_encode_refuses_bad_tables_before_any_device_work():
+    """df_encode_batch_prepare checks every descriptor, the codes and the
+    workspace on the host before it touches a device (no GPU here); the runs
+    refuse a plan they cannot use."""
+    import ctypes
+
+    L = _native.lib()
+    code = api.df_build_code(np.full(256, 1, np.uint64), 32)
+    t = (_native.DfEncodeTensor * 2)()
+    for x, n in zip(t, (100_000, 4096 * 5)):
+        x.input, x.n, x.total_bits, x.chunk_bytes, x.threads_per_block = 256, n, 8 * n, 32, 32
+        x.stream, x.gaps, x.block_offsets, x.sm = 4096, 8192, 16384, 32768
+    ws_hist = L.df_encode_batch_workspace(t, 2)
+    assert ws_hist > 0
+    one = L.df_encode_batch_workspace(t, 1)
+    assert 0 < one < ws_hist
+    plan = _native.DfEncodePlan()
+    t[0].code = ctypes.pointer(code)  # a code for one tensor only
+    assert L.df_encode_batch_prepare(t, 2, 4096, ws_hist, ctypes.byref(plan), None) == _native.DF_ERR_INVALID_ARG
+    t[1].code = ctypes.pointer(code)
+    t[1].chunk_bytes = 8  # not a multiple of 16
+    assert L.df_encode_batch_prepare(t, 2, 4096, ws_hist, ctypes.byref(plan), None) == _native.DF_ERR_INVALID_ARG
+    t[1].chunk_bytes, t[1].stream = 32, 4100  # stream not 16-byte aligned
+    assert L.df_encode_batch_prepare(t, 2, 4096, ws_hist, ctypes.byref(plan), None) == _native.DF_ERR_INVALID_ARG
+    t[1].stream = 4096
+    assert L.df_encode_batch_prepare(t, 2, 4096, ws_hist - 16, ctypes.byref(plan), None) == _native.DF_ERR_WORKSPACE
+    assert L.df_encode_batch_prepare(t, 2, 4100, ws_hist, ctypes.byref(plan), None) == _native.DF_ERR_INVALID_ARG
+    t[0].input = 257  # input not 2-byte aligned
+    assert L.df_encode_batch_prepare(t, 2, 4096, ws_hist, ctypes.byref(plan), None) == _native.DF_ERR_INVALID_ARG
+    t[0].input, t[0].n = 256, (1 << 48) + 1  # DF_MAX_WEIGHTS + 1
+    assert L.df_encode_batch_prepare(t, 2, 4096, ws_hist, ctypes.byref(plan), None) == _native.DF_ERR_UNSUPPORTED
+    # runs: a plan without codes cannot encode; no histogram buffer
+    plan.d_ws, plan.count, plan.has_codes = 4096, 2, 0
+    assert L.df_encode_batch_run(ctypes.byref(plan), None, None) == _native.DF_ERR_INVALID_ARG
+    assert L.df_histogram_batch_run(ctypes.byref(plan), None, None) == _native.DF_ERR_INVALID_ARG
