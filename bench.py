@@ -500,6 +500,15 @@ def grouped_encode_record(src, comps, args, peak, steps=5):
                     "memset, one encode kernel) over all tensors; algorithmic bytes as the per-tensor record"}
 
 
+def recorded(fn, *args):
+    """fn(*args), or the exception it raised as the record (so that one
+    secondary measurement cannot cost the whole bench line)."""
+    try:
+        return fn(*args)
+    except Exception as e:  # reported in the JSON line, not hidden
+        return {"error": f"{type(e).__name__}: {e}"}
+
+
 def time_launches(run, steps, warmup, stream, flush=None):
     """Per-step device ms of run() (CUDA events on `stream`). With `flush`, a
     write larger than L2 precedes every step, outside its events."""
@@ -931,7 +940,7 @@ def run_gpu(args, world, rank, local, pool, ncores):
         cfg[args.workload]["nf12"] = nf12_record(src, outs, args, stream, err, peak, fl)
         torch.cuda.empty_cache()
         cfg[args.workload]["idx8"] = idx8_record(comps, outs, src, args, stream, err, peak, fl)
-        extras["encode_grouped"] = grouped_encode_record(src, comps, args, peak)
+        extras["encode_grouped"] = recorded(grouped_encode_record, src, comps, args, peak)
         for name in ("single_1024x4096", "llama_layer", "heavy_tail_64m", "mixed_2000"):
             if name == args.workload:
                 continue
@@ -942,7 +951,7 @@ def run_gpu(args, world, rank, local, pool, ncores):
             cfg[name] = decode_record(s_comps, s_outs, args, stream, err, peak, fl)
             verify(s_src, s_outs, [s.name for s in sp])
             cfg[name]["nf12"] = nf12_record(s_src, s_outs, args, stream, err, peak, fl)
-            cfg[name]["encode_grouped"] = grouped_encode_record(s_src, s_comps, args, peak)
+            cfg[name]["encode_grouped"] = recorded(grouped_encode_record, s_src, s_comps, args, peak)
             del s_src, s_comps, s_outs, stg
         extras["configs"] = cfg
         del fl
