@@ -22,6 +22,12 @@
 // buffers. The input is read three times in all: by the histogram and by
 // both passes; each pass asks for its input two warp tiles ahead (an L2
 // prefetch hint).
+//
+// The grouped encode does the same for many tensors with one launch per
+// step: a histogram kernel over fixed tiles of every tensor, a kernel that
+// zeroes every tensor's outputs, and an encode kernel whose persistent CUDA
+// blocks take ranges of every tensor from one counter and run the same range
+// code (encode_range) on each, the range's tensor found by binary search.
 #include <cuda_runtime.h>
 
 #include <cstddef>
