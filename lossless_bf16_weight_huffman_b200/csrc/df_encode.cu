@@ -933,7 +933,10 @@ df_status df_encode_batch_prepare(const df_encode_tensor* h_tensors, uint32_t co
             if (t.code->lengths[e] > 32) return DF_ERR_INVALID_ARG;
     }
     const EncBatchLayout l = enc_batch_layout(count, sum_tiles);
-    if (ws_bytes < l.bytes) return DF_ERR_WORKSPACE;
+    if (count && ws_bytes < l.bytes) return DF_ERR_WORKSPACE;
+    std::memset(plan, 0, sizeof(*plan));
+    plan->d_ws = d_ws;
+    if (!count) return DF_OK;
 
     // histogram tiles: about four CUDA blocks per resident slot over the whole
     // set, 2^16 to 2^20 weights each (a power of two, so a multiple of 8)
@@ -969,7 +972,6 @@ df_status df_encode_batch_prepare(const df_encode_tensor* h_tensors, uint32_t co
     }
     if (hstart[count] > 0x7FFFFFFFull || rstart[count] > 0x7FFFFFFFull || zstart[count] > 0x7FFFFFFFull)
         return DF_ERR_UNSUPPORTED;
-    plan->d_ws = d_ws;
     plan->count = count;
     plan->has_codes = has_codes ? 1u : 0u;
     plan->sum_tiles = sum_tiles;
@@ -977,7 +979,6 @@ df_status df_encode_batch_prepare(const df_encode_tensor* h_tensors, uint32_t co
     plan->hist_tile_weights = tile;
     plan->ranges = rstart[count];
     plan->zero_tiles = zstart[count];
-    if (!count) return DF_OK;
     // copies from pageable host memory return once the source has been
     // staged, so the host vectors may die on return
     cudaStream_t s = static_cast<cudaStream_t>(stream);

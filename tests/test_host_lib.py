@@ -454,6 +454,12 @@ def test_grouped_encode_refuses_bad_tables_before_any_device_work():
     assert L.df_encode_batch_prepare(t, 2, 4096, ws_hist, ctypes.byref(plan), None) == _native.DF_ERR_INVALID_ARG
     t[0].input, t[0].n = 256, (1 << 48) + 1  # DF_MAX_WEIGHTS + 1
     assert L.df_encode_batch_prepare(t, 2, 4096, ws_hist, ctypes.byref(plan), None) == _native.DF_ERR_UNSUPPORTED
+    # an empty table needs no device: an empty plan, and runs that do nothing
+    assert L.df_encode_batch_workspace(t, 0) > 0
+    assert L.df_encode_batch_prepare(t, 0, None, 0, ctypes.byref(plan), None) == _native.DF_OK
+    assert plan.count == 0 and plan.ranges == 0
+    assert L.df_encode_batch_run(ctypes.byref(plan), None, None) == _native.DF_OK
+    assert L.df_histogram_batch_run(ctypes.byref(plan), None, None) == _native.DF_OK
     # runs: a plan without codes cannot encode; no histogram buffer
     plan.d_ws, plan.count, plan.has_codes = 4096, 2, 0
     assert L.df_encode_batch_run(ctypes.byref(plan), None, None) == _native.DF_ERR_INVALID_ARG
