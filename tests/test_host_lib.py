@@ -464,3 +464,25 @@ def test_grouped_encode_refuses_bad_tables_before_any_device_work():
     plan.d_ws, plan.count, plan.has_codes = 4096, 2, 0
     assert L.df_encode_batch_run(ctypes.byref(plan), None, None) == _native.DF_ERR_INVALID_ARG
     assert L.df_histogram_batch_run(ctypes.byref(plan), None, None) == _native.DF_ERR_INVALID_ARG
+
+
+def test_tensor_level_encoders_refuse_cpu_tensors_and_empty_lists():
+    """There is no CPU path: the grouped encoders reject host tensors (and an
+    empty list) before any library call."""
+    import torch
+
+    from lossless_bf16_weight_huffman_b200 import codec, nf12
+
+    w = torch.zeros(100, dtype=torch.bfloat16)
+    with pytest.raises(TypeError, match="CUDA"):
+        codec.compress_batch([w])
+    with pytest.raises(TypeError, match="CUDA"):
+        codec.compress(w)
+    with pytest.raises(ValueError, match="no tensors"):
+        codec.BatchEncoder([])
+    with pytest.raises(ValueError, match="no tensors"):
+        nf12.BatchEncoder([])
+    with pytest.raises(TypeError):
+        nf12.compress(w)
+    with pytest.raises(ValueError, match="no tensors"):
+        codec.BatchDecoder([])
