@@ -256,12 +256,14 @@ class BatchEncoder:
         self.chunk_bytes = _per_tensor(chunk_bytes, len(self.xs), "chunk_bytes")
         self.tpb = _per_tensor(threads_per_block, len(self.xs), "threads_per_block")
         self.hist = torch.empty((len(self.xs), 256), dtype=torch.int64, device=self.dev)
-        descs = self._descriptors()
+        descs = self.descriptors()
         self.ws = torch.empty(max(api.df_encode_batch_workspace(descs), 16), dtype=torch.uint8, device=self.dev)
         self.plan = api.df_encode_batch_prepare(descs, self.ws, stream)
         self.comps: list[Compressed] | None = None
 
-    def _descriptors(self, comps: list[Compressed] | None = None) -> list[DfEncodeTensor]:
+    def descriptors(self, comps: list[Compressed] | None = None) -> list[DfEncodeTensor]:
+        """The C descriptors of the inputs, with each container's code,
+        format and outputs when `comps` is given (histograms only otherwise)."""
         out = []
         for i, x in enumerate(self.xs):
             t = DfEncodeTensor()
@@ -306,7 +308,7 @@ class BatchEncoder:
                 gaps=torch.empty(z["gap_bytes"], dtype=torch.uint8, device=self.dev),
                 offsets=torch.empty(z["n_blocks"] + 1, dtype=torch.int64, device=self.dev),
                 sm=torch.empty(max(n, 16), dtype=torch.uint8, device=self.dev)))
-        self.plan = api.df_encode_batch_prepare(self._descriptors(comps), self.ws, stream)
+        self.plan = api.df_encode_batch_prepare(self.descriptors(comps), self.ws, stream)
         self.comps = comps
         return comps
 

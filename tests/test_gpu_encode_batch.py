@@ -94,7 +94,7 @@ def test_grouped_encode_reports_a_wrong_total_and_keeps_the_others_intact():
     ws = [base[:200_000], base[200_000:450_001], base[500_000:530_000]]
     enc = codec.BatchEncoder([dev_u16(w) for w in ws], chunk_bytes=32)
     comps = enc.prepare()
-    descs = enc._descriptors(comps)
+    descs = enc.descriptors(comps)
     descs[1].total_bits = comps[1].total_bits - 1  # the buffers stay large enough: one bit less
     enc.plan = api.df_encode_batch_prepare(descs, enc.ws)
     err = err_word()
