@@ -670,7 +670,8 @@ __global__ void __launch_bounds__(256)
         }
         done = e / 8 * 8;
     }
-    for (uint64_t i = done + threadIdx.x; i < e; i += blockDim.x) atomicAdd(&sh[warp][(__ldg(in + i) >> 7) & 0xFFu], 1u);
+    for (uint64_t i = done + threadIdx.x; i < e; i += blockDim.x)
+        atomicAdd(&sh[warp][(__ldg(in + i) >> 7) & 0xFFu], 1u);
     __syncthreads();
     for (uint32_t s = threadIdx.x; s < 256; s += blockDim.x) {
         uint32_t c = 0;
@@ -986,9 +987,12 @@ df_status df_encode_batch_prepare(const df_encode_tensor* h_tensors, uint32_t co
                                     cudaMemcpyHostToDevice, s);
     if (e == cudaSuccess && has_codes)
         e = cudaMemcpyAsync(ws + l.codes, codes.data(), sizeof(uint2) * codes.size(), cudaMemcpyHostToDevice, s);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(ws + l.hstart, hstart.data(), 8 * hstart.size(), cudaMemcpyHostToDevice, s);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(ws + l.rstart, rstart.data(), 8 * rstart.size(), cudaMemcpyHostToDevice, s);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(ws + l.zstart, zstart.data(), 8 * zstart.size(), cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(ws + l.hstart, hstart.data(), 8 * hstart.size(), cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(ws + l.rstart, rstart.data(), 8 * rstart.size(), cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(ws + l.zstart, zstart.data(), 8 * zstart.size(), cudaMemcpyHostToDevice, s);
     return e == cudaSuccess ? DF_OK : cuda_fail(e);
 }
 
